@@ -1,0 +1,226 @@
+/*
+ * kta_oracle.c -- plain fp64 CPU oracle for the Hybrid Linear Temporal Attention operator.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark load this file's library. The CUDA product path never links, loads or calls it,
+ * and this file includes nothing from the CUDA path.
+ *
+ * Source pages (cited by title and section):
+ *   [K1] paper-read "Kairos: A Native World Model Stack for Physical AI" (yingwang.github.io),
+ *        section 2 "Method", second pillar (hybrid linear temporal attention): the SWA, DSWA
+ *        and GLA paragraphs and the four gated delta-rule equations that follow them.
+ *   [K2] ai-papers.net summary of Kairos, section "3-layer hybrid temporal architecture".
+ *
+ * Each function evaluates its definition directly:
+ *   - softmax branches: every key s < N is tested with the visibility predicate by brute force,
+ *     scores are fp64 dot products, and softmax subtracts the row maximum;
+ *   - GLA: the per-token recurrence, one token at a time, with an fp64 d x d state;
+ *   - gated delta rule: the four recurrence lines in the order the page gives them.
+ * No blocking, chunking or reordering beyond that. Inputs are the stored values (bf16 or fp32)
+ * passed as float and widened to double on read; every sum is taken in double.
+ *
+ * Layouts (row-major): q, k, v, o are [B][N][H][d] (token-major, heads interleaved, the
+ * page's (B, F*L, D) with D = H*d). Heads h0 <= h < h1 are computed; other heads of o are left
+ * untouched. Gates cover only the computed heads: vector alpha [B][N][h1-h0][d]; scalar alpha
+ * and beta [B][N][h1-h0]. States S0 / S_out are [B][h1-h0][d][d], stored key-major:
+ * S[i][j] with i over the key dimension and j over the value dimension.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <omp.h>
+
+#define IDX4(b, n, h, c, N, H, D) ((((int64_t)(b) * (N) + (n)) * (H) + (h)) * (D) + (c))
+
+static int g_threads = 0;
+
+void oracle_set_threads(int n) { g_threads = n; }
+
+int oracle_get_threads(void) {
+    return g_threads > 0 ? g_threads : omp_get_max_threads();
+}
+
+/* [K1] SWA paragraph: standard attention inside a window of L x window_size tokens, L being
+ * the tokens of one frame. Reading: the window is W whole frames ending at the query's own
+ * frame (the own frame is fully visible, no later frame is). */
+static int swa_visible(int64_t t, int64_t s, int64_t P, int64_t W) {
+    int64_t ft = t / P, fs = s / P;
+    return fs <= ft && fs > ft - W;
+}
+
+/* [K1] DSWA paragraph: the same window size as SWA, but frames taken every dil-th step back
+ * from the query frame: frames ft, ft-dil, ..., ft-(W-1)*dil. */
+static int dswa_visible(int64_t t, int64_t s, int64_t P, int64_t W, int64_t dil) {
+    int64_t ft = t / P, fs = s / P;
+    if (fs > ft) return 0;
+    int64_t gap = ft - fs;
+    return (gap % dil) == 0 && (gap / dil) < W;
+}
+
+/* One softmax-attention output row o[b, t, h, :] over the keys that vis() admits. */
+static void softmax_row(const float* q, const float* k, const float* v, double* o,
+                        int64_t B, int64_t N, int64_t H, int64_t d,
+                        int64_t b, int64_t h, int64_t t, int64_t P, int64_t W, int64_t dil,
+                        int dilated, double scale, double* score, double* acc) {
+    (void)B;
+    const float* qt = q + IDX4(b, t, h, 0, N, H, d);
+    double mx = -INFINITY;
+    for (int64_t s = 0; s < N; ++s) {
+        int vis = dilated ? dswa_visible(t, s, P, W, dil) : swa_visible(t, s, P, W);
+        if (!vis) { score[s] = NAN; continue; }
+        const float* ks = k + IDX4(b, s, h, 0, N, H, d);
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += (double)qt[c] * (double)ks[c];
+        score[s] = scale * dot;
+        if (score[s] > mx) mx = score[s];
+    }
+    double denom = 0.0;
+    for (int64_t c = 0; c < d; ++c) acc[c] = 0.0;
+    for (int64_t s = 0; s < N; ++s) {
+        if (isnan(score[s])) continue;
+        double p = exp(score[s] - mx);
+        denom += p;
+        const float* vs = v + IDX4(b, s, h, 0, N, H, d);
+        for (int64_t c = 0; c < d; ++c) acc[c] += p * (double)vs[c];
+    }
+    double* ot = o + IDX4(b, t, h, 0, N, H, d);
+    for (int64_t c = 0; c < d; ++c) ot[c] = acc[c] / denom;
+}
+
+static int softmax_branch(const float* q, const float* k, const float* v, double* o,
+                          int B, int N, int H, int d, int h0, int h1,
+                          int P, int W, int dil, int dilated, double scale,
+                          const int64_t* rows, int64_t nrows) {
+    if (B < 1 || N < 1 || H < 1 || d < 1 || P < 1 || W < 1 || dil < 1) return 1;
+    if (h0 < 0 || h1 > H || h0 >= h1) return 1;
+    int64_t nr = rows ? nrows : (int64_t)N;
+    int64_t nh = h1 - h0;
+    int64_t total = (int64_t)B * nh * nr;
+    int nt = oracle_get_threads();
+#pragma omp parallel num_threads(nt)
+    {
+        double* score = (double*)malloc(sizeof(double) * (size_t)N);
+        double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t w = 0; w < total; ++w) {
+            int64_t r = w % nr;
+            int64_t h = h0 + (w / nr) % nh;
+            int64_t b = w / (nr * nh);
+            int64_t t = rows ? rows[r] : r;
+            if (t < 0 || t >= N) continue;
+            softmax_row(q, k, v, o, B, N, H, d, b, h, t, P, W, dil, dilated, scale, score, acc);
+        }
+        free(score);
+        free(acc);
+    }
+    return 0;
+}
+
+int oracle_swa(const float* q, const float* k, const float* v, double* o,
+               int B, int N, int H, int d, int h0, int h1,
+               int P, int W, double scale, const int64_t* rows, int64_t nrows) {
+    return softmax_branch(q, k, v, o, B, N, H, d, h0, h1, P, W, 1, 0, scale, rows, nrows);
+}
+
+int oracle_dswa(const float* q, const float* k, const float* v, double* o,
+                int B, int N, int H, int d, int h0, int h1,
+                int P, int W, int dil, double scale, const int64_t* rows, int64_t nrows) {
+    return softmax_branch(q, k, v, o, B, N, H, d, h0, h1, P, W, dil, 1, scale, rows, nrows);
+}
+
+/* Visibility predicates exported for the mask tests: out[i] = visible(t[i], s[i]). */
+void oracle_visible(const int64_t* t, const int64_t* s, int64_t n, int P, int W, int dil,
+                    int dilated, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = (uint8_t)(dilated ? dswa_visible(t[i], s[i], P, W, dil)
+                                   : swa_visible(t[i], s[i], P, W));
+}
+
+/* GLA with a vector forget gate, one token at a time (the form S_t = diag(alpha_t) S_{t-1}
+ * + k_t^T v_t, o_t = scale * q_t S_t; row convention, S is d_k x d_v). [K1] GLA paragraph
+ * gives the gated state update; the per-key-dimension gate is the configs' reading. */
+int oracle_gla(const float* q, const float* k, const float* v, const float* alpha,
+               const double* S0, double* o, double* S_out,
+               int B, int N, int H, int d, int h0, int h1, double scale) {
+    if (B < 1 || N < 0 || H < 1 || d < 1 || h0 < 0 || h1 > H || h0 >= h1) return 1;
+    int64_t nh = h1 - h0;
+    int nt = oracle_get_threads();
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+    for (int64_t w = 0; w < (int64_t)B * nh; ++w) {
+        int64_t b = w / nh, hg = w % nh, h = h0 + hg;
+        double* S = (double*)malloc(sizeof(double) * (size_t)d * (size_t)d);
+        if (S0) memcpy(S, S0 + w * d * d, sizeof(double) * (size_t)d * (size_t)d);
+        else memset(S, 0, sizeof(double) * (size_t)d * (size_t)d);
+        for (int64_t t = 0; t < N; ++t) {
+            const float* qt = q + IDX4(b, t, h, 0, N, H, d);
+            const float* kt = k + IDX4(b, t, h, 0, N, H, d);
+            const float* vt = v + IDX4(b, t, h, 0, N, H, d);
+            const float* at = alpha + IDX4(b, t, hg, 0, N, nh, d);
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j)
+                    S[i * d + j] = (double)at[i] * S[i * d + j] + (double)kt[i] * (double)vt[j];
+            double* ot = o + IDX4(b, t, h, 0, N, H, d);
+            for (int64_t j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += (double)qt[i] * S[i * d + j];
+                ot[j] = scale * acc;
+            }
+        }
+        if (S_out) memcpy(S_out + w * d * d, S, sizeof(double) * (size_t)d * (size_t)d);
+        free(S);
+    }
+    return 0;
+}
+
+/* Gated delta rule, the four lines of [K1] in the page's column convention (its state M is
+ * d_v x d_k; here M[j][i] is held as S[i][j]):
+ *   v_old = M_{t-1} k_t
+ *   v_new = beta_t v_t + (1 - beta_t) v_old
+ *   M_t   = alpha_t M_{t-1} - v_old k_t^T + v_new k_t^T
+ *   o_t   = scale * M_t q_t
+ * alpha_t and beta_t are scalars per token and head. */
+int oracle_delta(const float* q, const float* k, const float* v,
+                 const float* alpha, const float* beta, const double* S0,
+                 double* o, double* S_out,
+                 int B, int N, int H, int d, int h0, int h1, double scale) {
+    if (B < 1 || N < 0 || H < 1 || d < 1 || h0 < 0 || h1 > H || h0 >= h1) return 1;
+    int64_t nh = h1 - h0;
+    int nt = oracle_get_threads();
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+    for (int64_t w = 0; w < (int64_t)B * nh; ++w) {
+        int64_t b = w / nh, hg = w % nh, h = h0 + hg;
+        double* S = (double*)malloc(sizeof(double) * (size_t)d * (size_t)d);
+        double* vold = (double*)malloc(sizeof(double) * (size_t)d);
+        double* vnew = (double*)malloc(sizeof(double) * (size_t)d);
+        if (S0) memcpy(S, S0 + w * d * d, sizeof(double) * (size_t)d * (size_t)d);
+        else memset(S, 0, sizeof(double) * (size_t)d * (size_t)d);
+        for (int64_t t = 0; t < N; ++t) {
+            const float* qt = q + IDX4(b, t, h, 0, N, H, d);
+            const float* kt = k + IDX4(b, t, h, 0, N, H, d);
+            const float* vt = v + IDX4(b, t, h, 0, N, H, d);
+            double a = (double)alpha[((int64_t)b * N + t) * nh + hg];
+            double be = (double)beta[((int64_t)b * N + t) * nh + hg];
+            for (int64_t j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += S[i * d + j] * (double)kt[i];
+                vold[j] = acc;
+            }
+            for (int64_t j = 0; j < d; ++j) vnew[j] = be * (double)vt[j] + (1.0 - be) * vold[j];
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j)
+                    S[i * d + j] = a * S[i * d + j] - vold[j] * (double)kt[i] + vnew[j] * (double)kt[i];
+            double* ot = o + IDX4(b, t, h, 0, N, H, d);
+            for (int64_t j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += S[i * d + j] * (double)qt[i];
+                ot[j] = scale * acc;
+            }
+        }
+        if (S_out) memcpy(S_out + w * d * d, S, sizeof(double) * (size_t)d * (size_t)d);
+        free(S);
+        free(vold);
+        free(vnew);
+    }
+    return 0;
+}
