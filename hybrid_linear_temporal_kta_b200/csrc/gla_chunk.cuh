@@ -1,0 +1,325 @@
+// gla_chunk.cuh -- chunked gated linear attention with a vector forget gate (bf16 in / out,
+// fp32 state and gates), on warp-level bf16 tensor-core tiles.
+//
+// Operator (paper-read "Kairos: A Native World Model Stack for Physical AI", section 2, second
+// pillar, GLA paragraph): S_t = diag(alpha_t) S_{t-1} + k_t^T v_t, o_t = scale * q_t S_t.
+//
+// Chunked form used here (exact algebra, C tokens per chunk, chunks aligned to multiples of C
+// from token 0). Let b_t = sum_{r <= t in chunk} log2 alpha_r (a vector over key dims), m the
+// chunk's middle token and S_0 the state at the chunk start:
+//   o_t   = scale * [ (q_t * 2^{b_t}) S_0 + sum_{s <= t} ((q_t * 2^{b_t - b_m}) . (k_s * 2^{b_m - b_s})) v_s ]
+//   S_end = diag(2^{b_C}) S_0 + sum_s (k_s * 2^{b_C - b_s})^T v_s
+// The middle reference point keeps both factors of the intra-chunk product within 2^{|b| over
+// half a chunk}; the state and inter-chunk factors are <= 1.
+//
+// Sequence parallelism: the tokens of a sequence are split into segments of whole chunks.
+//   pass 1 (OUTPUT = false): each segment's end state from a zero start, and its total log2 decay;
+//   pass 2 (OUTPUT = true):  each segment folds S0 and the earlier segments' pass-1 results into
+//                            its start state, then runs the chunks and writes o.
+// The value dimension is split in BV = 64 column slices (columns of S are independent).
+// CTA = 4 warps. Warp w computes output rows [16w, 16w+16) of a chunk and state rows
+// [w*D/4, (w+1)*D/4).
+#pragma once
+
+#include "mma_sync.cuh"
+
+namespace kta {
+
+struct GlaParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* alpha;      // [B][rows][H][D]
+  __nv_bfloat16* o;
+  long long ld;            // q / k / v / o row stride (elements)
+  int rows_b;              // rows per sequence in q / k / v / o / alpha
+  int N;                   // tokens per sequence in this call
+  int H;                   // heads in this call
+  int seg_len;             // tokens per segment (multiple of C)
+  int nseg;
+  float scale;
+  const float* S0;         // [B][H][D][D] key-major, or null
+  float* S_out;            // [B][H][D][D], or null
+  float* ws_S;             // [B*H][nseg][D][D] segment end states (pass 1)
+  float* ws_L;             // [B*H][nseg][D] segment total log2 decay (pass 1)
+};
+
+template <int D, int C>
+struct GlaSmem {
+  static constexpr int BV = 64;
+  static constexpr int LDK = D + 8;   // padded rows: conflict-free ldmatrix
+  static constexpr int LDV = BV + 8;
+  __nv_bfloat16 q[C * LDK];   // raw q, then the intra-chunk query operand
+  __nv_bfloat16 qg[C * LDK];  // query decayed from the chunk start (inter-chunk operand)
+  __nv_bfloat16 k[C * LDK];   // raw k, then the intra-chunk key operand
+  __nv_bfloat16 kc[C * LDK];  // key decayed to the chunk end (state-update operand)
+  __nv_bfloat16 v[C * LDV];
+  __nv_bfloat16 s[D * LDV];   // bf16 copy of the chunk-start state slice
+  float g[C * D];             // alpha, then the cumulative log2 gate b_t
+  float gend[D];              // 2^{b_C}
+};
+
+template <int D, int C, bool OUTPUT>
+__global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
+  using SM = GlaSmem<D, C>;
+  constexpr int BV = SM::BV, LDK = SM::LDK, LDV = SM::LDV;
+  constexpr int RW = D / 4;           // state rows per warp
+  constexpr int MT = RW / 16;         // m16 tiles of state per warp
+  constexpr int NT = BV / 8;          // n8 tiles across the value slice
+  constexpr int RT = C / 16;          // 16-row query tiles per chunk
+  constexpr int MID = C / 2;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SM& sm = *reinterpret_cast<SM*>(smem_raw);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g4 = lane >> 2, t4 = lane & 3;
+  const int seg = blockIdx.x, slice = blockIdx.y, bh = blockIdx.z;
+  const int b = bh / p.H, h = bh % p.H;
+  const int j0 = slice * BV;
+  const int t_begin = seg * p.seg_len;
+  const int t_end = min(p.N, t_begin + p.seg_len);
+  const long long row_b = static_cast<long long>(b) * p.rows_b;
+
+  // ---- state fragment registers: st[mt][nt][r] = S[row][j0 + col]
+  float st[MT][NT][4];
+  auto srow = [&](int mt, int r) { return warp * RW + mt * 16 + g4 + (r >= 2 ? 8 : 0); };
+  auto scol = [&](int nt, int r) { return nt * 8 + 2 * t4 + (r & 1); };
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) st[mt][nt][r] = 0.f;
+
+  if (OUTPUT) {
+    const long long sb = static_cast<long long>(bh) * D * D;
+    if (p.S0) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            st[mt][nt][r] = p.S0[sb + srow(mt, r) * D + j0 + scol(nt, r)];
+    }
+    for (int s2 = 0; s2 < seg; ++s2) {
+      const float* L = p.ws_L + (static_cast<long long>(bh) * p.nseg + s2) * D;
+      const float* Sl = p.ws_S + (static_cast<long long>(bh) * p.nseg + s2) * D * D;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int row = srow(mt, r);
+          const float dec = exp2f(L[row]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            st[mt][nt][r] = fmaf(dec, st[mt][nt][r], Sl[row * D + j0 + scol(nt, r)]);
+        }
+    }
+  }
+  float ltot = 0.f;  // this thread's key dim (tid < D): total log2 decay over the segment
+
+  auto write_state_smem = [&]() {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int r0 = srow(mt, 0), c0 = scol(nt, 0);
+        *reinterpret_cast<uint32_t*>(&sm.s[r0 * LDV + c0]) = bf16x2(st[mt][nt][0], st[mt][nt][1]);
+        *reinterpret_cast<uint32_t*>(&sm.s[(r0 + 8) * LDV + c0]) = bf16x2(st[mt][nt][2], st[mt][nt][3]);
+      }
+  };
+  if (OUTPUT) write_state_smem();
+
+  for (int c0 = t_begin; c0 < t_end; c0 += C) {
+    const int n = min(C, t_end - c0);
+    // ---- load the chunk: q, k (OUTPUT only for q), v slice, alpha (rows >= n: zeros / alpha = 1)
+    {
+      constexpr int QCH = D / 8;  // 16-byte pieces per bf16 row
+      for (int idx = tid; idx < C * QCH; idx += 128) {
+        const int t = idx / QCH, c = (idx % QCH) * 8;
+        const long long grow = row_b + c0 + min(t, n - 1);
+        const int bytes = t < n ? 16 : 0;
+        const long long off = grow * p.ld + static_cast<long long>(h) * D + c;
+        if (OUTPUT) cp_async16(&sm.q[t * LDK + c], p.q + off, bytes);
+        cp_async16(&sm.k[t * LDK + c], p.k + off, bytes);
+      }
+      constexpr int VCH = BV / 8;
+      for (int idx = tid; idx < C * VCH; idx += 128) {
+        const int t = idx / VCH, c = (idx % VCH) * 8;
+        const long long grow = row_b + c0 + min(t, n - 1);
+        cp_async16(&sm.v[t * LDV + c], p.v + grow * p.ld + static_cast<long long>(h) * D + j0 + c,
+                   t < n ? 16 : 0);
+      }
+      constexpr int ACH = D / 4;  // 16-byte pieces per fp32 row
+      for (int idx = tid; idx < C * ACH; idx += 128) {
+        const int t = idx / ACH, c = (idx % ACH) * 4;
+        if (t < n) {
+          const long long grow = row_b + c0 + t;
+          cp_async16(&sm.g[t * D + c], p.alpha + (grow * p.H + h) * D + c, 16);
+        } else {
+          *reinterpret_cast<float4*>(&sm.g[t * D + c]) = make_float4(1.f, 1.f, 1.f, 1.f);
+        }
+      }
+      cp_async_wait_all();
+    }
+    __syncthreads();
+    // ---- cumulative log2 gate per key dim
+    if (tid < D) {
+      float acc = 0.f;
+#pragma unroll 8
+      for (int t = 0; t < C; ++t) {
+        acc += __log2f(sm.g[t * D + tid]);
+        sm.g[t * D + tid] = acc;
+      }
+      sm.gend[tid] = exp2f(acc);
+      ltot += acc;
+    }
+    __syncthreads();
+    // ---- decayed operands
+    for (int idx = tid; idx < C * D; idx += 128) {
+      const int t = idx / D, i = idx % D;
+      const float bt = sm.g[t * D + i];
+      const float bl = sm.g[(C - 1) * D + i];
+      const float kv = __bfloat162float(sm.k[t * LDK + i]);
+      sm.kc[t * LDK + i] = __float2bfloat16_rn(kv * exp2f(bl - bt));
+      if (OUTPUT) {
+        const float bm = sm.g[MID * D + i];
+        const float qv = __bfloat162float(sm.q[t * LDK + i]);
+        const float e = exp2f(bt - bm);
+        sm.q[t * LDK + i] = __float2bfloat16_rn(qv * e);
+        sm.qg[t * LDK + i] = __float2bfloat16_rn(qv * exp2f(bt));
+        sm.k[t * LDK + i] = __float2bfloat16_rn(kv * exp2f(bm - bt));
+      }
+    }
+    __syncthreads();
+
+    if (OUTPUT && warp < RT) {
+      const int r0 = warp * 16;
+      // intra-chunk scores A = Qi Ki^T, causal part only (key tiles up to this warp's rows)
+      uint32_t aq[D / 16][4];
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) ldsm_x4(aq[kk], &sm.q[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
+      float acc[C / 8][4];
+#pragma unroll
+      for (int nt = 0; nt < C / 8; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[nt][r] = 0.f;
+#pragma unroll
+      for (int np = 0; np < C / 16; ++np) {
+        if (np > warp) break;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          uint32_t bk[4];
+          ldsm_x4(bk, &sm.k[frag_b_nmajor(lane, np * 16, kk * 16, LDK)]);
+          mma16816(acc[2 * np], aq[kk], bk[0], bk[1]);
+          mma16816(acc[2 * np + 1], aq[kk], bk[2], bk[3]);
+        }
+      }
+      // causal mask (s <= t) and conversion to bf16 A fragments
+      uint32_t pa[C / 16][4];
+#pragma unroll
+      for (int nt = 0; nt < C / 8; ++nt) {
+        const int col = nt * 8 + 2 * t4;
+        const int ra = r0 + g4, rb = r0 + g4 + 8;
+        const float x0 = col <= ra ? acc[nt][0] : 0.f;
+        const float x1 = col + 1 <= ra ? acc[nt][1] : 0.f;
+        const float x2 = col <= rb ? acc[nt][2] : 0.f;
+        const float x3 = col + 1 <= rb ? acc[nt][3] : 0.f;
+        pa[nt >> 1][(nt & 1) * 2 + 0] = bf16x2(x0, x1);
+        pa[nt >> 1][(nt & 1) * 2 + 1] = bf16x2(x2, x3);
+      }
+      float ov[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) ov[nt][r] = 0.f;
+      // O = A V  (tokens up to this warp's rows)
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+        if (kk > warp) break;
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t bv[4];
+          ldsm_x4_t(bv, &sm.v[frag_b_kmajor(lane, kk * 16, np * 16, LDV)]);
+          mma16816(ov[2 * np], pa[kk], bv[0], bv[1]);
+          mma16816(ov[2 * np + 1], pa[kk], bv[2], bv[3]);
+        }
+      }
+      // O += Qg S_0
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t ag[4];
+        ldsm_x4(ag, &sm.qg[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t bs[4];
+          ldsm_x4_t(bs, &sm.s[frag_b_kmajor(lane, kk * 16, np * 16, LDV)]);
+          mma16816(ov[2 * np], ag, bs[0], bs[1]);
+          mma16816(ov[2 * np + 1], ag, bs[2], bs[3]);
+        }
+      }
+      // store rows < n
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int t = r0 + g4 + hr * 8;
+        if (t < n) {
+          __nv_bfloat16* orow = p.o + (row_b + c0 + t) * p.ld + static_cast<long long>(h) * D + j0;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            *reinterpret_cast<uint32_t*>(orow + nt * 8 + 2 * t4) =
+                bf16x2(ov[nt][2 * hr] * p.scale, ov[nt][2 * hr + 1] * p.scale);
+        }
+      }
+    }
+
+    // ---- state update: S = diag(2^{b_C}) S + Kc^T V  (all warps)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float dec = sm.gend[srow(mt, r)];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) st[mt][nt][r] *= dec;
+      }
+#pragma unroll
+    for (int kk = 0; kk < C / 16; ++kk) {
+      uint32_t bv[NT / 2][4];
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) ldsm_x4_t(bv[np], &sm.v[frag_b_kmajor(lane, kk * 16, np * 16, LDV)]);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        uint32_t ak[4];
+        ldsm_x4_t(ak, &sm.kc[frag_a_kmajor(lane, warp * RW + mt * 16, kk * 16, LDK)]);
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          mma16816(st[mt][2 * np], ak, bv[np][0], bv[np][1]);
+          mma16816(st[mt][2 * np + 1], ak, bv[np][2], bv[np][3]);
+        }
+      }
+    }
+    __syncthreads();
+    if (OUTPUT) write_state_smem();
+  }
+
+  if (!OUTPUT) {
+    float* Sl = p.ws_S + (static_cast<long long>(bh) * p.nseg + seg) * D * D;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) Sl[srow(mt, r) * D + j0 + scol(nt, r)] = st[mt][nt][r];
+    if (slice == 0 && tid < D) p.ws_L[(static_cast<long long>(bh) * p.nseg + seg) * D + tid] = ltot;
+  } else if (seg == p.nseg - 1 && p.S_out) {
+    float* So = p.S_out + static_cast<long long>(bh) * D * D;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) So[srow(mt, r) * D + j0 + scol(nt, r)] = st[mt][nt][r];
+  }
+}
+
+}  // namespace kta

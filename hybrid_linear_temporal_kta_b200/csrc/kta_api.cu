@@ -1,0 +1,992 @@
+// kta_api.cu -- the C ABI of libkta.so (declared in include/kta.h): argument validation, tensor
+// map encoding, work decomposition and kernel launches for the Hybrid Linear Temporal Attention
+// operator. All kernels of the library are compiled into this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+
+#include "kta.h"
+#include "kta_ptx.cuh"
+#include "win_attn_tc.cuh"
+#include "simt_f32.cuh"
+#include "gla_chunk.cuh"
+#include "delta_chunk.cuh"
+
+namespace {
+
+using kta::WinParams;
+
+thread_local std::string g_last_error;
+
+kta_status fail(kta_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+#define KTA_CUDA(call)                                                                 \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    if (e_ != cudaSuccess)                                                             \
+      return fail(KTA_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));       \
+  } while (0)
+
+inline size_t elem_size(kta_dtype dt) { return dt == KTA_BF16 ? 2 : 4; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over a token-major buffer: dim0 = d (contiguous), dim1 = heads (stride d),
+// dim2 = rows (stride ld elements); box = 64 columns x 1 head x 128 rows, 128-byte swizzle,
+// zero fill outside the tensor.
+kta_status make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows,
+                    long long ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return KTA_OK;
+}
+
+// ------------------------------------------------------------------------- per-device state
+
+struct DeviceRes {
+  void* ws = nullptr;        // GLA segment workspace (grown on demand)
+  size_t ws_bytes = 0;
+  std::mutex mu;
+};
+
+DeviceRes& device_res(int dev) {
+  static std::mutex mu;
+  static std::map<int, DeviceRes*> m;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = m.find(dev);
+  if (it == m.end()) it = m.emplace(dev, new DeviceRes()).first;
+  return *it->second;
+}
+
+struct ThreadStreams {  // per host thread and device: side stream + events for the hybrid fork
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+kta_status thread_streams(ThreadStreams** out) {
+  thread_local std::map<int, ThreadStreams> m;
+  int dev = 0;
+  KTA_CUDA(cudaGetDevice(&dev));
+  ThreadStreams& t = m[dev];
+  if (!t.side) {
+    KTA_CUDA(cudaStreamCreateWithFlags(&t.side, cudaStreamNonBlocking));
+    KTA_CUDA(cudaEventCreateWithFlags(&t.fork, cudaEventDisableTiming));
+    KTA_CUDA(cudaEventCreateWithFlags(&t.join, cudaEventDisableTiming));
+  }
+  *out = &t;
+  return KTA_OK;
+}
+
+kta_status workspace(size_t bytes, void** out) {
+  int dev = 0;
+  KTA_CUDA(cudaGetDevice(&dev));
+  DeviceRes& r = device_res(dev);
+  std::lock_guard<std::mutex> lk(r.mu);
+  if (r.ws_bytes < bytes) {
+    if (r.ws) {
+      KTA_CUDA(cudaDeviceSynchronize());
+      KTA_CUDA(cudaFree(r.ws));
+      r.ws = nullptr;
+      r.ws_bytes = 0;
+    }
+    KTA_CUDA(cudaMalloc(&r.ws, bytes));
+    r.ws_bytes = bytes;
+  }
+  *out = r.ws;
+  return KTA_OK;
+}
+
+// Raise a kernel's dynamic shared memory limit once per (kernel, device).
+template <typename K>
+kta_status set_smem_attr(K kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, bool> done;
+  int dev = 0;
+  KTA_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  if (!done[key]) {
+    KTA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)));
+    done[key] = true;
+  }
+  return KTA_OK;
+}
+
+// ------------------------------------------------------------------------- softmax launches
+
+struct WinGroup {
+  int H = 0, W = 1, dil = 1;
+  const void* k = nullptr;   // key buffer of the group (head coordinate = h - kh_off)
+  const void* v = nullptr;
+  long long k_ld = 0;        // row stride (elements)
+  long long k_rows = 0;      // rows in the buffer
+  int k_heads = 0;           // heads in one row of the buffer addressed by the map
+  int kh_off = 0;
+  int kb_frames = 0, kmod = 1;
+};
+
+struct WinLaunch {
+  int B = 0, P = 0, Fq = 0, f_base = 0, d = 0;
+  kta_dtype dt = KTA_BF16;
+  const void* q = nullptr;
+  long long q_ld = 0;
+  int q_rows_b = 0;
+  void* o = nullptr;
+  long long o_ld = 0;
+  float scale = 1.f;
+  WinGroup g[2];
+};
+
+template <int D>
+kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
+  const int Htot = L.g[0].H + L.g[1].H;
+  CUtensorMap tq, tk0, tv0, tk1, tv1;
+  kta_status s;
+  if ((s = make_map(&tq, L.q, D, Htot, static_cast<long long>(L.B) * L.q_rows_b, L.q_ld))) return s;
+  const WinGroup& g0 = L.g[0];
+  const WinGroup& g1 = L.g[1].H > 0 ? L.g[1] : L.g[0];
+  if ((s = make_map(&tk0, g0.k, D, g0.k_heads, g0.k_rows, g0.k_ld))) return s;
+  if ((s = make_map(&tv0, g0.v, D, g0.k_heads, g0.k_rows, g0.k_ld))) return s;
+  if ((s = make_map(&tk1, g1.k, D, g1.k_heads, g1.k_rows, g1.k_ld))) return s;
+  if ((s = make_map(&tv1, g1.v, D, g1.k_heads, g1.k_rows, g1.k_ld))) return s;
+  WinParams p{};
+  p.B = L.B;
+  p.P = L.P;
+  p.Fq = L.Fq;
+  p.f_base = L.f_base;
+  p.n_qt = (L.P + 127) / 128;
+  p.Htot = Htot;
+  p.H0 = L.g[0].H;
+  for (int i = 0; i < 2; ++i) {
+    const WinGroup& g = L.g[i].H > 0 ? L.g[i] : L.g[0];
+    p.W[i] = g.W;
+    p.dil[i] = g.dil;
+    p.kh_off[i] = g.kh_off;
+    p.kb_frames[i] = g.kb_frames;
+    p.kmod[i] = g.kmod;
+  }
+  p.q_rows_b = L.q_rows_b;
+  p.scale_log2 = L.scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(L.o);
+  p.o_ld = L.o_ld;
+  const long long nblk = static_cast<long long>(L.Fq) * Htot * L.B * p.n_qt;
+  if (nblk <= 0) return KTA_OK;
+  if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "grid too large (%lld CTAs)", nblk);
+  const size_t smem = kta::win_smem_bytes<D>();
+  if ((s = set_smem_attr(kta::win_attn_tc_kernel<D>, smem))) return s;
+  kta::win_attn_tc_kernel<D><<<static_cast<unsigned>(nblk), 192, smem, st>>>(tq, tk0, tv0, tk1,
+                                                                             tv1, p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+kta_status launch_win_f32(const WinLaunch& L, cudaStream_t st) {
+  kta::WinSimtParams p{};
+  p.B = L.B;
+  p.P = L.P;
+  p.Fq = L.Fq;
+  p.f_base = L.f_base;
+  p.Htot = L.g[0].H + L.g[1].H;
+  p.H0 = L.g[0].H;
+  for (int i = 0; i < 2; ++i) {
+    const WinGroup& g = L.g[i].H > 0 ? L.g[i] : L.g[0];
+    p.W[i] = g.W;
+    p.dil[i] = g.dil;
+    p.kh_off[i] = g.kh_off;
+    p.kb_frames[i] = g.kb_frames;
+    p.kmod[i] = g.kmod;
+    p.k_ld[i] = g.k_ld;
+  }
+  p.q_rows_b = L.q_rows_b;
+  p.q_ld = L.q_ld;
+  p.o_ld = L.o_ld;
+  p.scale = L.scale;
+  p.d = L.d;
+  const WinGroup& g1 = L.g[1].H > 0 ? L.g[1] : L.g[0];
+  dim3 grid((L.Fq * L.P + 3) / 4, p.Htot, L.B);
+  if (grid.y > 65535 || grid.z > 65535) return fail(KTA_ERR_UNSUPPORTED, "too many heads/batches");
+  kta::win_attn_f32_kernel<<<grid, 128, 0, st>>>(
+      static_cast<const float*>(L.q), static_cast<const float*>(L.g[0].k),
+      static_cast<const float*>(L.g[0].v), static_cast<const float*>(g1.k),
+      static_cast<const float*>(g1.v), static_cast<float*>(L.o), p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+kta_status launch_win(const WinLaunch& L, cudaStream_t st) {
+  if (L.g[0].H + L.g[1].H == 0 || L.Fq == 0) return KTA_OK;
+  if (L.dt == KTA_F32) return launch_win_f32(L, st);
+  if (L.d == 128) return launch_win_tc<128>(L, st);
+  if (L.d == 64) return launch_win_tc<64>(L, st);
+  return fail(KTA_ERR_UNSUPPORTED, "bf16 softmax branches need d in {64, 128} (got %d)", L.d);
+}
+
+// ------------------------------------------------------------------------- GLA launches
+
+struct LinLaunch {
+  int B = 0, N = 0, H = 0, d = 0, rows_b = 0, chunk = 64;
+  kta_dtype dt = KTA_BF16;
+  const void *q = nullptr, *k = nullptr, *v = nullptr;
+  void* o = nullptr;
+  long long ld = 0;
+  const float* alpha = nullptr;
+  const float* beta = nullptr;
+  const float* S0 = nullptr;
+  float* S_out = nullptr;
+  float scale = 1.f;
+  bool delta = false;
+  bool allow_segments = true;
+};
+
+template <int D, int C>
+kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
+  using SM = kta::GlaSmem<D, C>;
+  const int slices = D / SM::BV;
+  const long long base = static_cast<long long>(L.B) * L.H * slices;
+  const int nchunks = (L.N + C - 1) / C;
+  int nseg = 1;
+  if (L.allow_segments) {
+    const long long want = (4LL * 148 + base - 1) / base;
+    nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
+  }
+  const int seg_chunks = (nchunks + nseg - 1) / nseg;
+  const int seg_len = seg_chunks * C;
+  nseg = (L.N + seg_len - 1) / seg_len;
+  kta::GlaParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(L.q);
+  p.k = static_cast<const __nv_bfloat16*>(L.k);
+  p.v = static_cast<const __nv_bfloat16*>(L.v);
+  p.alpha = L.alpha;
+  p.o = static_cast<__nv_bfloat16*>(L.o);
+  p.ld = L.ld;
+  p.rows_b = L.rows_b;
+  p.N = L.N;
+  p.H = L.H;
+  p.seg_len = seg_len;
+  p.nseg = nseg;
+  p.scale = L.scale;
+  p.S0 = L.S0;
+  p.S_out = L.S_out;
+  if (nseg > 1) {
+    void* ws = nullptr;
+    const size_t bytes = static_cast<size_t>(L.B) * L.H * nseg * (size_t(D) * D + D) * 4;
+    kta_status s = workspace(bytes, &ws);
+    if (s) return s;
+    p.ws_S = static_cast<float*>(ws);
+    p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * nseg * D * D;
+  }
+  const size_t smem = sizeof(SM);
+  kta_status sa;
+  if ((sa = set_smem_attr(kta::gla_chunk_kernel<D, C, false>, smem)) ||
+      (sa = set_smem_attr(kta::gla_chunk_kernel<D, C, true>, smem)))
+    return sa;
+  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
+  dim3 grid(nseg, slices, L.B * L.H);
+  if (nseg > 1) {
+    kta::gla_chunk_kernel<D, C, false><<<grid, 128, smem, st>>>(p);
+    KTA_CUDA(cudaGetLastError());
+  }
+  kta::gla_chunk_kernel<D, C, true><<<grid, 128, smem, st>>>(p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+template <int D>
+kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
+  using SM = kta::DeltaSmem<D>;
+  kta::DeltaParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(L.q);
+  p.k = static_cast<const __nv_bfloat16*>(L.k);
+  p.v = static_cast<const __nv_bfloat16*>(L.v);
+  p.alpha = L.alpha;
+  p.beta = L.beta;
+  p.o = static_cast<__nv_bfloat16*>(L.o);
+  p.ld = L.ld;
+  p.rows_b = L.rows_b;
+  p.N = L.N;
+  p.H = L.H;
+  p.scale = L.scale;
+  p.S0 = L.S0;
+  p.S_out = L.S_out;
+  const size_t smem = sizeof(SM);
+  kta_status sa;
+  if ((sa = set_smem_attr(kta::delta_chunk_kernel<D>, smem))) return sa;
+  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
+  dim3 grid(D / SM::BV, L.B * L.H);
+  kta::delta_chunk_kernel<D><<<grid, 128, smem, st>>>(p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+template <int D>
+kta_status launch_rec_f32(const LinLaunch& L, cudaStream_t st) {
+  kta::RecF32Params p{};
+  p.B = L.B;
+  p.N = L.N;
+  p.H = L.H;
+  p.d = D;
+  p.ld = L.ld;
+  p.rows_b = L.rows_b;
+  p.scale = L.scale;
+  p.S0 = L.S0;
+  p.S_out = L.S_out;
+  if (L.B > 65535) return fail(KTA_ERR_UNSUPPORTED, "B > 65535");
+  dim3 grid(L.H, L.B);
+  if (L.delta)
+    kta::delta_rec_f32_kernel<D><<<grid, D, 0, st>>>(
+        static_cast<const float*>(L.q), static_cast<const float*>(L.k),
+        static_cast<const float*>(L.v), L.alpha, L.beta, static_cast<float*>(L.o), p);
+  else
+    kta::gla_rec_f32_kernel<D><<<grid, D, 0, st>>>(
+        static_cast<const float*>(L.q), static_cast<const float*>(L.k),
+        static_cast<const float*>(L.v), L.alpha, static_cast<float*>(L.o), p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+kta_status launch_lin(const LinLaunch& L, cudaStream_t st) {
+  if (L.H == 0 || L.N == 0) return KTA_OK;
+  if (L.dt == KTA_F32) {
+    if (L.d == 32) return launch_rec_f32<32>(L, st);
+    if (L.d == 64) return launch_rec_f32<64>(L, st);
+    return launch_rec_f32<128>(L, st);
+  }
+  if (L.delta) {
+    if (L.d == 128) return launch_delta_chunk<128>(L, st);
+    if (L.d == 64) return launch_delta_chunk<64>(L, st);
+    return fail(KTA_ERR_UNSUPPORTED, "bf16 delta rule needs d in {64, 128} (got %d)", L.d);
+  }
+  if (L.d == 128) {
+    if (L.chunk == 64) return launch_gla_chunk<128, 64>(L, st);
+    if (L.chunk == 32) return launch_gla_chunk<128, 32>(L, st);
+    return launch_gla_chunk<128, 16>(L, st);
+  }
+  if (L.d == 64) {
+    if (L.chunk == 64) return launch_gla_chunk<64, 64>(L, st);
+    if (L.chunk == 32) return launch_gla_chunk<64, 32>(L, st);
+    return launch_gla_chunk<64, 16>(L, st);
+  }
+  return fail(KTA_ERR_UNSUPPORTED, "bf16 GLA needs d in {64, 128} (got %d)", L.d);
+}
+
+// ------------------------------------------------------------------------- validation
+
+kta_status check_shape(const kta_shape& s) {
+  if (s.B < 1 || s.F < 1 || s.P < 1) return fail(KTA_ERR_INVALID_ARG, "B, F, P must be >= 1");
+  if (s.d != 32 && s.d != 64 && s.d != 128)
+    return fail(KTA_ERR_UNSUPPORTED, "d must be 32, 64 or 128 (got %d)", s.d);
+  if (s.dtype != KTA_BF16 && s.dtype != KTA_F32) return fail(KTA_ERR_INVALID_ARG, "bad dtype");
+  const long long N = static_cast<long long>(s.F) * s.P;
+  if (N >= (1LL << 31) || static_cast<long long>(s.B) * N >= (1LL << 31))
+    return fail(KTA_ERR_UNSUPPORTED, "B*F*P must be < 2^31");
+  return KTA_OK;
+}
+
+kta_status check_heads(int H, int ld_heads, const kta_shape& s) {
+  if (H < 1 || ld_heads < H) return fail(KTA_ERR_INVALID_ARG, "need 1 <= H <= ld_heads");
+  if ((static_cast<long long>(ld_heads) * s.d * elem_size(s.dtype)) % 16)
+    return fail(KTA_ERR_ALIGNMENT, "row stride ld_heads*d*elem must be a multiple of 16 bytes");
+  return KTA_OK;
+}
+
+kta_status check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return fail(KTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(p)) return fail(KTA_ERR_ALIGNMENT, "tensor pointer not 16-byte aligned");
+  }
+  return KTA_OK;
+}
+
+kta_status check_softmax_dtype(const kta_shape& s) {
+  if (s.dtype == KTA_BF16 && s.d == 32)
+    return fail(KTA_ERR_UNSUPPORTED, "bf16 softmax branches need d in {64, 128}");
+  return KTA_OK;
+}
+
+WinLaunch seq_win_launch(const void* q, const void* k, const void* v, void* o, const kta_shape& s,
+                         int ld_heads, float scale) {
+  WinLaunch L;
+  L.B = s.B;
+  L.P = s.P;
+  L.Fq = s.F;
+  L.f_base = 0;
+  L.d = s.d;
+  L.dt = s.dtype;
+  L.q = q;
+  L.q_ld = static_cast<long long>(ld_heads) * s.d;
+  L.q_rows_b = s.F * s.P;
+  L.o = o;
+  L.o_ld = L.q_ld;
+  L.scale = scale;
+  return L;
+}
+
+WinGroup seq_group(const void* k, const void* v, const kta_shape& s, int H, int Htot, int ld_heads,
+                   int W, int dil) {
+  WinGroup g;
+  g.H = H;
+  g.W = W;
+  g.dil = dil;
+  g.k = k;
+  g.v = v;
+  g.k_ld = static_cast<long long>(ld_heads) * s.d;
+  g.k_rows = static_cast<long long>(s.B) * s.F * s.P;
+  g.k_heads = Htot;
+  g.kh_off = 0;
+  g.kb_frames = s.F;
+  g.kmod = s.F;
+  return g;
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+// =========================================================================== C ABI
+
+extern "C" {
+
+const char* kta_status_str(kta_status s) {
+  switch (s) {
+    case KTA_OK: return "KTA_OK";
+    case KTA_ERR_INVALID_ARG: return "KTA_ERR_INVALID_ARG";
+    case KTA_ERR_UNSUPPORTED: return "KTA_ERR_UNSUPPORTED";
+    case KTA_ERR_ALIGNMENT: return "KTA_ERR_ALIGNMENT";
+    case KTA_ERR_CUDA: return "KTA_ERR_CUDA";
+    case KTA_ERR_TIMEOUT: return "KTA_ERR_TIMEOUT";
+    case KTA_ERR_STATE: return "KTA_ERR_STATE";
+  }
+  return "KTA_ERR_UNKNOWN";
+}
+
+const char* kta_last_error(void) { return g_last_error.c_str(); }
+
+int kta_version(void) { return KTA_VERSION; }
+
+kta_status kta_swa_fwd(const void* q, const void* k, const void* v, void* o, kta_shape s, int H,
+                       int ld_heads, int W, float scale, void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) || (r = check_ptrs({q, k, v, o})) ||
+      (r = check_softmax_dtype(s)))
+    return r;
+  if (W < 1) return fail(KTA_ERR_INVALID_ARG, "W must be >= 1");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be > 0");
+  WinLaunch L = seq_win_launch(q, k, v, o, s, ld_heads, scale);
+  L.g[0] = seq_group(k, v, s, H, H, ld_heads, W, 1);
+  return launch_win(L, as_stream(stream));
+}
+
+kta_status kta_dswa_fwd(const void* q, const void* k, const void* v, void* o, kta_shape s, int H,
+                        int ld_heads, int W, int dil, float scale, void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) || (r = check_ptrs({q, k, v, o})) ||
+      (r = check_softmax_dtype(s)))
+    return r;
+  if (W < 1 || dil < 1) return fail(KTA_ERR_INVALID_ARG, "W and dil must be >= 1");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be > 0");
+  WinLaunch L = seq_win_launch(q, k, v, o, s, ld_heads, scale);
+  L.g[0] = seq_group(k, v, s, H, H, ld_heads, W, dil);
+  return launch_win(L, as_stream(stream));
+}
+
+static kta_status lin_common(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, float* S_out, void* o,
+                             kta_shape s, int H, int ld_heads, int chunk, float scale, bool delta,
+                             void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) || (r = check_ptrs({q, k, v, o})))
+    return r;
+  if (!alpha || (delta && !beta)) return fail(KTA_ERR_INVALID_ARG, "null gate pointer");
+  if (!aligned16(alpha) || (S0 && !aligned16(S0)) || (S_out && !aligned16(S_out)))
+    return fail(KTA_ERR_ALIGNMENT, "gate / state pointers must be 16-byte aligned");
+  if (chunk != 16 && chunk != 32 && chunk != 64)
+    return fail(KTA_ERR_INVALID_ARG, "chunk must be 16, 32 or 64");
+  if (!std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be finite");
+  LinLaunch L;
+  L.B = s.B;
+  L.N = s.F * s.P;
+  L.H = H;
+  L.d = s.d;
+  L.rows_b = L.N;
+  L.chunk = chunk;
+  L.dt = s.dtype;
+  L.q = q;
+  L.k = k;
+  L.v = v;
+  L.o = o;
+  L.ld = static_cast<long long>(ld_heads) * s.d;
+  L.alpha = alpha;
+  L.beta = beta;
+  L.S0 = S0;
+  L.S_out = S_out;
+  L.scale = scale;
+  L.delta = delta;
+  return launch_lin(L, as_stream(stream));
+}
+
+kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* S0, float* S_out, void* o, kta_shape s, int H,
+                             int ld_heads, int chunk, float scale, void* stream) {
+  return lin_common(q, k, v, alpha, nullptr, S0, S_out, o, s, H, ld_heads, chunk, scale, false,
+                    stream);
+}
+
+kta_status kta_gla_delta_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, float* S_out, void* o,
+                             kta_shape s, int H, int ld_heads, int chunk, float scale,
+                             void* stream) {
+  return lin_common(q, k, v, alpha, beta, S0, S_out, o, s, H, ld_heads, chunk, scale, true, stream);
+}
+
+static kta_status check_cfg(const kta_hybrid_cfg* c) {
+  if (!c) return fail(KTA_ERR_INVALID_ARG, "null cfg");
+  kta_status r;
+  if ((r = check_shape(c->s))) return r;
+  if (c->n_swa < 0 || c->n_dswa < 0 || c->n_gla < 0 || c->n_swa + c->n_dswa + c->n_gla < 1)
+    return fail(KTA_ERR_INVALID_ARG, "head counts must be >= 0 with at least one head");
+  if (c->n_swa + c->n_dswa > 0) {
+    if ((r = check_softmax_dtype(c->s))) return r;
+    if ((c->n_swa && c->W_swa < 1) || (c->n_dswa && (c->W_dswa < 1 || c->dil < 1)))
+      return fail(KTA_ERR_INVALID_ARG, "windows and dilation must be >= 1");
+    if (!(c->scale_softmax > 0.f) || !std::isfinite(c->scale_softmax))
+      return fail(KTA_ERR_INVALID_ARG, "scale_softmax must be > 0");
+  }
+  if (c->n_gla > 0) {
+    if (c->chunk != 16 && c->chunk != 32 && c->chunk != 64)
+      return fail(KTA_ERR_INVALID_ARG, "chunk must be 16, 32 or 64");
+    if (!std::isfinite(c->scale_gla)) return fail(KTA_ERR_INVALID_ARG, "scale_gla must be finite");
+  }
+  const int H = c->n_swa + c->n_dswa + c->n_gla;
+  return check_heads(H, H, c->s);
+}
+
+kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* beta, void* o, void* stream) {
+  kta_status r;
+  if ((r = check_cfg(cfg)) || (r = check_ptrs({q, k, v, o}))) return r;
+  const kta_shape& s = cfg->s;
+  const int H = cfg->n_swa + cfg->n_dswa + cfg->n_gla;
+  if (cfg->n_gla > 0) {
+    if (!alpha || (cfg->gla_delta && !beta)) return fail(KTA_ERR_INVALID_ARG, "null gate pointer");
+    if (!aligned16(alpha)) return fail(KTA_ERR_ALIGNMENT, "alpha not 16-byte aligned");
+  }
+  const size_t es = elem_size(s.dtype);
+  const long long ld = static_cast<long long>(H) * s.d;
+  cudaStream_t st = as_stream(stream);
+
+  WinLaunch W = seq_win_launch(q, k, v, o, s, H, cfg->scale_softmax);
+  W.g[0] = seq_group(k, v, s, cfg->n_swa, cfg->n_swa + cfg->n_dswa, H, cfg->W_swa, 1);
+  W.g[1] = seq_group(k, v, s, cfg->n_dswa, cfg->n_swa + cfg->n_dswa, H, cfg->W_dswa, cfg->dil);
+  if (cfg->n_swa == 0) {  // DSWA heads only: make them group 0
+    W.g[0] = W.g[1];
+    W.g[1] = WinGroup();
+  }
+
+  LinLaunch L;
+  L.B = s.B;
+  L.N = s.F * s.P;
+  L.H = cfg->n_gla;
+  L.d = s.d;
+  L.rows_b = L.N;
+  L.chunk = cfg->chunk;
+  L.dt = s.dtype;
+  const size_t hoff = static_cast<size_t>(cfg->n_swa + cfg->n_dswa) * s.d * es;
+  L.q = static_cast<const char*>(q) + hoff;
+  L.k = static_cast<const char*>(k) + hoff;
+  L.v = static_cast<const char*>(v) + hoff;
+  L.o = static_cast<char*>(o) + hoff;
+  L.ld = ld;
+  L.alpha = alpha;
+  L.beta = beta;
+  L.scale = cfg->scale_gla;
+  L.delta = cfg->gla_delta != 0;
+
+  const bool both = (cfg->n_swa + cfg->n_dswa) > 0 && cfg->n_gla > 0;
+  if (!both) {
+    if ((r = launch_win(W, st))) return r;
+    return launch_lin(L, st);
+  }
+  ThreadStreams* ts = nullptr;
+  if ((r = thread_streams(&ts))) return r;
+  KTA_CUDA(cudaEventRecord(ts->fork, st));
+  KTA_CUDA(cudaStreamWaitEvent(ts->side, ts->fork, 0));
+  kta_status r_lin = launch_lin(L, ts->side);
+  KTA_CUDA(cudaEventRecord(ts->join, ts->side));
+  kta_status r_win = launch_win(W, st);
+  KTA_CUDA(cudaStreamWaitEvent(st, ts->join, 0));
+  if (r_lin) return r_lin;
+  return r_win;
+}
+
+// --------------------------------------------------------------------------- streaming
+
+}  // extern "C"
+
+struct kta_stream_s {
+  kta_hybrid_cfg cfg;
+  int device = 0;
+  int64_t frame = 0;
+  int R_swa = 0, R_dswa = 0;    // ring slots (SWA ring is stored twice: 2 * R_swa frames)
+  size_t es = 2;
+  char* arena = nullptr;        // [header | swa k | swa v | dswa k | dswa v | state 0 | state 1]
+  size_t arena_bytes = 0;
+  size_t off_swa_k = 0, off_swa_v = 0, off_dswa_k = 0, off_dswa_v = 0, off_state[2] = {0, 0};
+  size_t ring_swa_bytes = 0, ring_dswa_bytes = 0, state_bytes = 0;
+  int cur = 0;
+  uint32_t magic = 0x6b746131u;
+};
+
+namespace {
+
+constexpr size_t kHeader = 256;
+
+struct BlobHeader {
+  uint32_t magic;
+  uint32_t cur;
+  int64_t frame;
+  int32_t B, P, d, n_swa, n_dswa, n_gla, W_swa, W_dswa, dil, dtype, gla_delta;
+};
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+std::mutex g_streams_mu;
+std::map<const kta_stream_s*, bool> g_streams;  // live handles
+
+kta_status valid_stream(kta_stream_t st) {
+  std::lock_guard<std::mutex> lk(g_streams_mu);
+  if (!st || !g_streams.count(st)) return fail(KTA_ERR_STATE, "invalid or destroyed stream handle");
+  return KTA_OK;
+}
+
+// Copy heads [h0, h0+nh) of one frame ([B][P][H][d]) into ring slot `slot` ([B][RR][P][nh][d]).
+kta_status ring_put(const kta_stream_s* s, const void* src, char* ring, int h0, int nh, int RR,
+                    int slot, cudaStream_t st) {
+  const kta_shape& sh = s->cfg.s;
+  const int H = s->cfg.n_swa + s->cfg.n_dswa + s->cfg.n_gla;
+  const size_t row_src = static_cast<size_t>(H) * sh.d * s->es;
+  const size_t row_dst = static_cast<size_t>(nh) * sh.d * s->es;
+  for (int b = 0; b < sh.B; ++b) {
+    const char* sp = static_cast<const char*>(src) + static_cast<size_t>(b) * sh.P * row_src +
+                     static_cast<size_t>(h0) * sh.d * s->es;
+    char* dp = ring + (static_cast<size_t>(b) * RR + slot) * sh.P * row_dst;
+    KTA_CUDA(cudaMemcpy2DAsync(dp, row_dst, sp, row_src, row_dst, sh.P, cudaMemcpyDeviceToDevice, st));
+  }
+  return KTA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kta_status kta_stream_create(const kta_hybrid_cfg* cfg, kta_stream_t* out) {
+  if (!out) return fail(KTA_ERR_INVALID_ARG, "null output handle");
+  *out = nullptr;
+  kta_hybrid_cfg c = *cfg;
+  c.s.F = 1;
+  kta_status r;
+  if ((r = check_cfg(&c))) return r;
+  kta_stream_s* s = new kta_stream_s();
+  s->cfg = c;
+  KTA_CUDA(cudaGetDevice(&s->device));
+  s->es = elem_size(c.s.dtype);
+  s->R_swa = c.n_swa ? c.W_swa : 0;
+  s->R_dswa = c.n_dswa ? (c.W_dswa - 1) * c.dil + 1 : 0;
+  const size_t frame_bytes_swa = static_cast<size_t>(c.s.P) * c.n_swa * c.s.d * s->es;
+  const size_t frame_bytes_dswa = static_cast<size_t>(c.s.P) * c.n_dswa * c.s.d * s->es;
+  s->ring_swa_bytes = round_up(static_cast<size_t>(c.s.B) * 2 * s->R_swa * frame_bytes_swa, 256);
+  s->ring_dswa_bytes = round_up(static_cast<size_t>(c.s.B) * s->R_dswa * frame_bytes_dswa, 256);
+  s->state_bytes = round_up(static_cast<size_t>(c.s.B) * c.n_gla * c.s.d * c.s.d * 4, 256);
+  size_t off = kHeader;
+  s->off_swa_k = off; off += s->ring_swa_bytes;
+  s->off_swa_v = off; off += s->ring_swa_bytes;
+  s->off_dswa_k = off; off += s->ring_dswa_bytes;
+  s->off_dswa_v = off; off += s->ring_dswa_bytes;
+  s->off_state[0] = off; off += s->state_bytes;
+  s->off_state[1] = off; off += s->state_bytes;
+  s->arena_bytes = off;
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&s->arena), s->arena_bytes);
+  if (e != cudaSuccess) {
+    delete s;
+    return fail(KTA_ERR_CUDA, "cudaMalloc of %zu stream bytes failed: %s", off, cudaGetErrorString(e));
+  }
+  e = cudaMemset(s->arena, 0, s->arena_bytes);
+  if (e != cudaSuccess) {
+    cudaFree(s->arena);
+    delete s;
+    return fail(KTA_ERR_CUDA, "cudaMemset failed: %s", cudaGetErrorString(e));
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_streams_mu);
+    g_streams[s] = true;
+  }
+  *out = s;
+  return KTA_OK;
+}
+
+kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, const void* v_f,
+                           const float* alpha_f, const float* beta_f, void* o_f, void* stream) {
+  kta_status r;
+  if ((r = valid_stream(s)) || (r = check_ptrs({q_f, k_f, v_f, o_f}))) return r;
+  const kta_hybrid_cfg& c = s->cfg;
+  if (c.n_gla > 0 && (!alpha_f || (c.gla_delta && !beta_f)))
+    return fail(KTA_ERR_INVALID_ARG, "null gate pointer");
+  if (s->frame >= (1LL << 30)) return fail(KTA_ERR_STATE, "frame counter exhausted");
+  int dev = 0;
+  KTA_CUDA(cudaGetDevice(&dev));
+  if (dev != s->device) return fail(KTA_ERR_STATE, "stream handle belongs to device %d", s->device);
+  cudaStream_t st = as_stream(stream);
+  const kta_shape& sh = c.s;
+  const int H = c.n_swa + c.n_dswa + c.n_gla;
+  const int f = static_cast<int>(s->frame);
+  char* swa_k = s->arena + s->off_swa_k;
+  char* swa_v = s->arena + s->off_swa_v;
+  char* dswa_k = s->arena + s->off_dswa_k;
+  char* dswa_v = s->arena + s->off_dswa_v;
+  // 1. append this frame's keys and values to the rings
+  if (c.n_swa) {
+    const int slot = f % s->R_swa;
+    if ((r = ring_put(s, k_f, swa_k, 0, c.n_swa, 2 * s->R_swa, slot, st)) ||
+        (r = ring_put(s, k_f, swa_k, 0, c.n_swa, 2 * s->R_swa, slot + s->R_swa, st)) ||
+        (r = ring_put(s, v_f, swa_v, 0, c.n_swa, 2 * s->R_swa, slot, st)) ||
+        (r = ring_put(s, v_f, swa_v, 0, c.n_swa, 2 * s->R_swa, slot + s->R_swa, st)))
+      return r;
+  }
+  if (c.n_dswa) {
+    const int slot = f % s->R_dswa;
+    if ((r = ring_put(s, k_f, dswa_k, c.n_swa, c.n_dswa, s->R_dswa, slot, st)) ||
+        (r = ring_put(s, v_f, dswa_v, c.n_swa, c.n_dswa, s->R_dswa, slot, st)))
+      return r;
+  }
+  // 2. softmax heads: queries of this frame against the rings
+  if (c.n_swa + c.n_dswa > 0) {
+    WinLaunch L;
+    L.B = sh.B;
+    L.P = sh.P;
+    L.Fq = 1;
+    L.f_base = f;
+    L.d = sh.d;
+    L.dt = sh.dtype;
+    L.q = q_f;
+    L.q_ld = static_cast<long long>(H) * sh.d;
+    L.q_rows_b = sh.P;
+    L.o = o_f;
+    L.o_ld = L.q_ld;
+    L.scale = c.scale_softmax;
+    int gi = 0;
+    if (c.n_swa) {
+      WinGroup& g = L.g[gi++];
+      g.H = c.n_swa;
+      g.W = c.W_swa;
+      g.dil = 1;
+      g.k = swa_k;
+      g.v = swa_v;
+      g.k_ld = static_cast<long long>(c.n_swa) * sh.d;
+      g.k_rows = static_cast<long long>(sh.B) * 2 * s->R_swa * sh.P;
+      g.k_heads = c.n_swa;
+      g.kh_off = 0;
+      g.kb_frames = 2 * s->R_swa;
+      g.kmod = s->R_swa;
+    }
+    if (c.n_dswa) {
+      WinGroup& g = L.g[gi++];
+      g.H = c.n_dswa;
+      g.W = c.W_dswa;
+      g.dil = c.dil;
+      g.k = dswa_k;
+      g.v = dswa_v;
+      g.k_ld = static_cast<long long>(c.n_dswa) * sh.d;
+      g.k_rows = static_cast<long long>(sh.B) * s->R_dswa * sh.P;
+      g.k_heads = c.n_dswa;
+      g.kh_off = c.n_swa;
+      g.kb_frames = s->R_dswa;
+      g.kmod = s->R_dswa;
+    }
+    if ((r = launch_win(L, st))) return r;
+  }
+  // 3. GLA heads: this frame's tokens from the carried state (ping-pong state buffers)
+  if (c.n_gla) {
+    LinLaunch L;
+    L.B = sh.B;
+    L.N = sh.P;
+    L.H = c.n_gla;
+    L.d = sh.d;
+    L.rows_b = sh.P;
+    L.chunk = c.chunk;
+    L.dt = sh.dtype;
+    const size_t hoff = static_cast<size_t>(c.n_swa + c.n_dswa) * sh.d * s->es;
+    L.q = static_cast<const char*>(q_f) + hoff;
+    L.k = static_cast<const char*>(k_f) + hoff;
+    L.v = static_cast<const char*>(v_f) + hoff;
+    L.o = static_cast<char*>(o_f) + hoff;
+    L.ld = static_cast<long long>(H) * sh.d;
+    L.alpha = alpha_f;
+    L.beta = beta_f;
+    L.S0 = reinterpret_cast<const float*>(s->arena + s->off_state[s->cur]);
+    L.S_out = reinterpret_cast<float*>(s->arena + s->off_state[1 - s->cur]);
+    L.scale = c.scale_gla;
+    L.delta = c.gla_delta != 0;
+    L.allow_segments = false;
+    if ((r = launch_lin(L, st))) return r;
+    s->cur = 1 - s->cur;
+  }
+  s->frame += 1;
+  return KTA_OK;
+}
+
+kta_status kta_stream_reset(kta_stream_t s, void* stream) {
+  kta_status r;
+  if ((r = valid_stream(s))) return r;
+  KTA_CUDA(cudaMemsetAsync(s->arena, 0, s->arena_bytes, as_stream(stream)));
+  s->frame = 0;
+  s->cur = 0;
+  return KTA_OK;
+}
+
+int64_t kta_stream_frame(kta_stream_t s) { return valid_stream(s) ? -1 : s->frame; }
+
+size_t kta_stream_state_bytes(kta_stream_t s) { return valid_stream(s) ? 0 : s->arena_bytes; }
+
+kta_status kta_stream_save(kta_stream_t s, void* dev_dst, void* stream) {
+  kta_status r;
+  if ((r = valid_stream(s))) return r;
+  if (!dev_dst) return fail(KTA_ERR_INVALID_ARG, "null destination");
+  cudaStream_t st = as_stream(stream);
+  BlobHeader hd{};
+  hd.magic = s->magic;
+  hd.cur = static_cast<uint32_t>(s->cur);
+  hd.frame = s->frame;
+  const kta_hybrid_cfg& c = s->cfg;
+  hd.B = c.s.B; hd.P = c.s.P; hd.d = c.s.d; hd.n_swa = c.n_swa; hd.n_dswa = c.n_dswa;
+  hd.n_gla = c.n_gla; hd.W_swa = c.W_swa; hd.W_dswa = c.W_dswa; hd.dil = c.dil;
+  hd.dtype = c.s.dtype; hd.gla_delta = c.gla_delta;
+  KTA_CUDA(cudaMemcpyAsync(dev_dst, s->arena + kHeader, s->arena_bytes - kHeader,
+                           cudaMemcpyDeviceToDevice, st));
+  // The header goes last in the blob so that the arena copy above stays one contiguous copy.
+  KTA_CUDA(cudaMemcpyAsync(static_cast<char*>(dev_dst) + (s->arena_bytes - kHeader), &hd, sizeof(hd),
+                           cudaMemcpyHostToDevice, st));
+  KTA_CUDA(cudaStreamSynchronize(st));
+  return KTA_OK;
+}
+
+kta_status kta_stream_load(kta_stream_t s, const void* dev_src, void* stream) {
+  kta_status r;
+  if ((r = valid_stream(s))) return r;
+  if (!dev_src) return fail(KTA_ERR_INVALID_ARG, "null source");
+  cudaStream_t st = as_stream(stream);
+  BlobHeader hd{};
+  KTA_CUDA(cudaMemcpyAsync(&hd, static_cast<const char*>(dev_src) + (s->arena_bytes - kHeader),
+                           sizeof(hd), cudaMemcpyDeviceToHost, st));
+  KTA_CUDA(cudaStreamSynchronize(st));
+  const kta_hybrid_cfg& c = s->cfg;
+  if (hd.magic != s->magic || hd.B != c.s.B || hd.P != c.s.P || hd.d != c.s.d ||
+      hd.n_swa != c.n_swa || hd.n_dswa != c.n_dswa || hd.n_gla != c.n_gla ||
+      hd.W_swa != c.W_swa || hd.W_dswa != c.W_dswa || hd.dil != c.dil || hd.dtype != c.s.dtype ||
+      hd.gla_delta != c.gla_delta || hd.frame < 0 || hd.cur > 1)
+    return fail(KTA_ERR_STATE, "state blob does not match this stream's configuration");
+  KTA_CUDA(cudaMemcpyAsync(s->arena + kHeader, dev_src, s->arena_bytes - kHeader,
+                           cudaMemcpyDeviceToDevice, st));
+  s->frame = hd.frame;
+  s->cur = static_cast<int>(hd.cur);
+  return KTA_OK;
+}
+
+kta_status kta_stream_destroy(kta_stream_t s) {
+  kta_status r;
+  if ((r = valid_stream(s))) return r;
+  {
+    std::lock_guard<std::mutex> lk(g_streams_mu);
+    g_streams.erase(s);
+  }
+  s->magic = 0;
+  cudaError_t e1 = cudaDeviceSynchronize();
+  cudaError_t e2 = cudaFree(s->arena);
+  delete s;
+  if (e1 != cudaSuccess || e2 != cudaSuccess)
+    return fail(KTA_ERR_CUDA, "stream teardown failed: %s",
+                cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
+  return KTA_OK;
+}
+
+// --------------------------------------------------------------------------- diagnostics
+
+kta_status kta_device_status(void* stream) {
+  KTA_CUDA(cudaStreamSynchronize(as_stream(stream)));
+  unsigned int word = 0;
+  KTA_CUDA(cudaMemcpyFromSymbol(&word, kta::g_dev_error, sizeof(word)));
+  if (word) {
+    const unsigned int zero = 0;
+    KTA_CUDA(cudaMemcpyToSymbol(kta::g_dev_error, &zero, sizeof(zero)));
+    if (word & kta::DEVERR_WAIT_TIMEOUT)
+      return fail(KTA_ERR_TIMEOUT, "a bounded device wait expired (code 0x%x)", word);
+    return fail(KTA_ERR_CUDA, "device error word 0x%x", word);
+  }
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+}  // extern "C"
+
+namespace kta {
+__global__ void wait_timeout_probe_kernel(long long budget) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  // Nobody arrives on `bar`: the bounded wait must give up after `budget` cycles.
+  mbar_wait(&bar, 0, budget);
+}
+}  // namespace kta
+
+extern "C" kta_status kta_selftest_wait_timeout(long long budget_cycles, void* stream) {
+  if (budget_cycles < 1 || budget_cycles > (1LL << 31))
+    return fail(KTA_ERR_INVALID_ARG, "budget must be in [1, 2^31] cycles");
+  kta::wait_timeout_probe_kernel<<<1, 1, 0, as_stream(stream)>>>(budget_cycles);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}

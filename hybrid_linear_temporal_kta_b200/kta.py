@@ -1,0 +1,271 @@
+"""ctypes binding of libkta.so (C ABI in include/kta.h).
+
+Argument marshalling only: every step of the operator runs in the library's CUDA kernels. Tensors
+are torch CUDA tensors in the operator's layout [B, N, H, d] (token-major, heads interleaved);
+calls are enqueued on torch's current CUDA stream. Importing this module loads the library and
+raises if it is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from . import build as _build
+
+_LIB_PATH = _build.LIB
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libkta.so not built ({_LIB_PATH}); run hybrid_linear_temporal_kta_b200.build")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+BF16, F32 = 0, 1
+_DT = {torch.bfloat16: BF16, torch.float32: F32}
+_STATUS = {0: "KTA_OK", 1: "KTA_ERR_INVALID_ARG", 2: "KTA_ERR_UNSUPPORTED", 3: "KTA_ERR_ALIGNMENT",
+           4: "KTA_ERR_CUDA", 5: "KTA_ERR_TIMEOUT", 6: "KTA_ERR_STATE"}
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("F", ctypes.c_int), ("P", ctypes.c_int), ("d", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+class HybridCfg(ctypes.Structure):
+    _fields_ = [("s", Shape), ("n_swa", ctypes.c_int), ("n_dswa", ctypes.c_int),
+                ("n_gla", ctypes.c_int), ("W_swa", ctypes.c_int), ("W_dswa", ctypes.c_int),
+                ("dil", ctypes.c_int), ("chunk", ctypes.c_int), ("gla_delta", ctypes.c_int),
+                ("scale_softmax", ctypes.c_float), ("scale_gla", ctypes.c_float)]
+
+
+_vp, _i, _f, _st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int
+_fp = ctypes.c_void_p
+
+_SIGS = {
+    "kta_status_str": ([_st], ctypes.c_char_p),
+    "kta_last_error": ([], ctypes.c_char_p),
+    "kta_version": ([], _i),
+    "kta_swa_fwd": ([_vp, _vp, _vp, _vp, Shape, _i, _i, _i, _f, _vp], _st),
+    "kta_dswa_fwd": ([_vp, _vp, _vp, _vp, Shape, _i, _i, _i, _i, _f, _vp], _st),
+    "kta_gla_chunk_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp], _st),
+    "kta_gla_delta_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
+                          _st),
+    "kta_hybrid_fwd": ([ctypes.POINTER(HybridCfg), _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
+    "kta_stream_create": ([ctypes.POINTER(HybridCfg), ctypes.POINTER(_vp)], _st),
+    "kta_stream_step": ([_vp, _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
+    "kta_stream_reset": ([_vp, _vp], _st),
+    "kta_stream_frame": ([_vp], ctypes.c_int64),
+    "kta_stream_state_bytes": ([_vp], ctypes.c_size_t),
+    "kta_stream_save": ([_vp, _vp, _vp], _st),
+    "kta_stream_load": ([_vp, _vp, _vp], _st),
+    "kta_stream_destroy": ([_vp], _st),
+    "kta_device_status": ([_vp], _st),
+    "kta_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _st),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+class KtaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.kta_last_error().decode()
+        super().__init__(f"{where}: {_STATUS.get(status, status)}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise KtaError(status, where)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t, off_elems: int = 0):
+    return None if t is None else ctypes.c_void_p(t.data_ptr() + off_elems * t.element_size())
+
+
+def _need(t, name, dtype=None):
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+
+
+def _shape(q: torch.Tensor, P: int) -> Shape:
+    B, N, _, d = q.shape
+    if N % P:
+        raise ValueError(f"N = {N} is not a whole number of frames of P = {P}")
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bf16 or fp32")
+    return Shape(B, N // P, P, d, _DT[q.dtype])
+
+
+def version() -> int:
+    return _lib.kta_version()
+
+
+def _softmax(fn, q, k, v, P, W, dil, scale, heads, out, stream):
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.dtype)
+    Htot, d = q.shape[2], q.shape[3]
+    h0, h1 = heads if heads is not None else (0, Htot)
+    o = torch.empty_like(q) if out is None else out
+    _need(o, "out", q.dtype)
+    s = _shape(q, P)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    args = [_ptr(q, h0 * d), _ptr(k, h0 * d), _ptr(v, h0 * d), _ptr(o, h0 * d), s, h1 - h0, Htot, W]
+    if dil is not None:
+        args.append(dil)
+    _check(fn(*args, scale, _stream(stream)), fn.__name__)
+    return o
+
+
+def swa_fwd(q, k, v, *, P: int, W: int, scale: float | None = None, heads=None, out=None,
+            stream=None):
+    """Frame-block-causal sliding-window attention over W frames of P tokens."""
+    return _softmax(_lib.kta_swa_fwd, q, k, v, P, W, None, scale, heads, out, stream)
+
+
+def dswa_fwd(q, k, v, *, P: int, W: int, dil: int, scale: float | None = None, heads=None,
+             out=None, stream=None):
+    """Dilated sliding-window attention: key frames f, f-dil, ..., f-(W-1)*dil."""
+    return _softmax(_lib.kta_dswa_fwd, q, k, v, P, W, dil, scale, heads, out, stream)
+
+
+def _linear(delta, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream):
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.dtype)
+    _need(alpha, "alpha", torch.float32)
+    if delta:
+        _need(beta, "beta", torch.float32)
+    B, N, Htot, d = q.shape
+    h0, h1 = heads if heads is not None else (0, Htot)
+    H = h1 - h0
+    o = torch.empty_like(q) if out is None else out
+    _need(o, "out", q.dtype)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32)
+    S_out = torch.empty((B, H, d, d), device=q.device, dtype=torch.float32) if return_state else None
+    s = Shape(B, 1, N, d, _DT[q.dtype])  # one frame of N tokens: the linear branches ignore frames
+    if delta:
+        st = _lib.kta_gla_delta_fwd(_ptr(q, h0 * d), _ptr(k, h0 * d), _ptr(v, h0 * d), _ptr(alpha),
+                                    _ptr(beta), _ptr(S0), _ptr(S_out), _ptr(o, h0 * d), s, H, Htot,
+                                    chunk, scale, _stream(stream))
+    else:
+        st = _lib.kta_gla_chunk_fwd(_ptr(q, h0 * d), _ptr(k, h0 * d), _ptr(v, h0 * d), _ptr(alpha),
+                                    _ptr(S0), _ptr(S_out), _ptr(o, h0 * d), s, H, Htot, chunk,
+                                    scale, _stream(stream))
+    _check(st, "kta_gla_delta_fwd" if delta else "kta_gla_chunk_fwd")
+    return (o, S_out) if return_state else o
+
+
+def gla_chunk_fwd(q, k, v, alpha, *, chunk: int = 64, scale: float = 1.0, S0=None,
+                  return_state: bool = False, heads=None, out=None, stream=None):
+    """Vector-gated GLA; alpha [B, N, H, d] fp32. Returns o (and the final state)."""
+    return _linear(False, q, k, v, alpha, None, chunk, scale, S0, return_state, heads, out, stream)
+
+
+def gla_delta_fwd(q, k, v, alpha, beta, *, chunk: int = 64, scale: float = 1.0, S0=None,
+                  return_state: bool = False, heads=None, out=None, stream=None):
+    """Gated delta rule; alpha, beta [B, N, H] fp32. Returns o (and the final state)."""
+    return _linear(True, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream)
+
+
+def hybrid_cfg(*, B: int, F: int, P: int, d: int, dtype=torch.bfloat16, n_swa: int, n_dswa: int,
+               n_gla: int, W_swa: int = 3, W_dswa: int = 4, dil: int = 3, chunk: int = 64,
+               gla_delta: bool = False, scale_softmax: float | None = None,
+               scale_gla: float = 1.0) -> HybridCfg:
+    return HybridCfg(Shape(B, F, P, d, _DT[dtype]), n_swa, n_dswa, n_gla, W_swa, W_dswa, dil, chunk,
+                     int(gla_delta), 1.0 / math.sqrt(d) if scale_softmax is None else scale_softmax,
+                     scale_gla)
+
+
+def cfg_from_workload(w, B: int | None = None, F: int | None = None) -> HybridCfg:
+    """HybridCfg of a synth.Workload."""
+    return hybrid_cfg(B=w.B if B is None else B, F=w.F if F is None else F, P=w.P, d=w.d,
+                      dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+                      n_swa=w.n_swa, n_dswa=w.n_dswa, n_gla=w.n_gla, W_swa=w.W_swa,
+                      W_dswa=w.W_dswa, dil=w.dil, chunk=w.chunk, gla_delta=w.gla_delta,
+                      scale_softmax=w.scale_softmax)
+
+
+def hybrid_fwd(cfg: HybridCfg, q, k, v, alpha=None, beta=None, *, out=None, stream=None):
+    """Hybrid layer: SWA heads, DSWA heads, GLA heads (outputs concatenated by head)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.dtype)
+    o = torch.empty_like(q) if out is None else out
+    _check(_lib.kta_hybrid_fwd(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                               _ptr(beta), _ptr(o), _stream(stream)), "kta_hybrid_fwd")
+    return o
+
+
+class Stream:
+    """One-frame-at-a-time rollout with carried GLA state and rolling K/V rings."""
+
+    def __init__(self, cfg: HybridCfg):
+        self.cfg = cfg
+        h = ctypes.c_void_p()
+        _check(_lib.kta_stream_create(ctypes.byref(cfg), ctypes.byref(h)), "kta_stream_create")
+        self._h = h
+
+    def step(self, q_f, k_f, v_f, alpha_f=None, beta_f=None, *, out=None, stream=None):
+        o = torch.empty_like(q_f) if out is None else out
+        _check(_lib.kta_stream_step(self._h, _ptr(q_f), _ptr(k_f), _ptr(v_f), _ptr(alpha_f),
+                                    _ptr(beta_f), _ptr(o), _stream(stream)), "kta_stream_step")
+        return o
+
+    def reset(self, stream=None):
+        _check(_lib.kta_stream_reset(self._h, _stream(stream)), "kta_stream_reset")
+
+    @property
+    def frame(self) -> int:
+        return int(_lib.kta_stream_frame(self._h))
+
+    @property
+    def state_bytes(self) -> int:
+        return int(_lib.kta_stream_state_bytes(self._h))
+
+    def save(self, stream=None) -> torch.Tensor:
+        blob = torch.empty(self.state_bytes, dtype=torch.uint8, device="cuda")
+        _check(_lib.kta_stream_save(self._h, _ptr(blob), _stream(stream)), "kta_stream_save")
+        return blob
+
+    def load(self, blob: torch.Tensor, stream=None):
+        _check(_lib.kta_stream_load(self._h, _ptr(blob), _stream(stream)), "kta_stream_load")
+
+    def close(self):
+        if self._h is not None:
+            _check(_lib.kta_stream_destroy(self._h), "kta_stream_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def device_status(stream=None):
+    """Raise KtaError if a bounded device wait expired since the last check."""
+    _check(_lib.kta_device_status(_stream(stream)), "kta_device_status")
+
+
+def selftest_wait_timeout(budget_cycles: int, stream=None):
+    _check(_lib.kta_selftest_wait_timeout(int(budget_cycles), _stream(stream)),
+           "kta_selftest_wait_timeout")
+
+
+def raw_call(name: str, *args) -> int:
+    """Call an exported entry point with raw ctypes arguments; returns the kta_status code."""
+    return int(getattr(_lib, name)(*args))
+
+
+def last_error() -> str:
+    return _lib.kta_last_error().decode()

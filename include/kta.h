@@ -1,0 +1,191 @@
+/*
+ * kta.h -- C ABI of libkta.so: the Hybrid Linear Temporal Attention operator on B200 (sm_100a).
+ *
+ * Operator source: paper-read "Kairos: A Native World Model Stack for Physical AI"
+ * (yingwang.github.io), section 2 "Method", second pillar: short-range sliding-window attention
+ * (SWA), mid-range dilated sliding-window attention (DSWA), and global gated linear attention
+ * (GLA, "based on GatedDeltaNet") whose state update is given there as four equations. The
+ * ai-papers.net summary ("3-layer hybrid temporal architecture") and the secrett2633 review
+ * ("Method & Key Results", the Delta Update Rule) describe the same three branches.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Tensors are row-major, token-major with heads interleaved: x[b][n][h][c] is at element
+ *  offset ((b*N + n)*ld_heads + h)*d + c, i.e. the pages' (B, F*L, D) layout with D = H*d and
+ *  L = P tokens per frame. N = F*P tokens, frames in time order, tokens of a frame contiguous.
+ *  A call that serves heads [h0, h0+H) of a wider tensor receives pointers already offset by
+ *  h0*d elements and ld_heads = the tensor's total head count; its H heads are computed.
+ *  q, k, v, o use kta_shape.dtype (KTA_BF16: bf16, KTA_F32: fp32). Gates and states are fp32.
+ *  o is written only for the computed heads; nothing else in o is touched.
+ *
+ *  Every pointer is a DEVICE pointer into memory the caller owns (cudaMalloc / torch). The
+ *  library keeps no reference to it after the call's work has run. Work is enqueued on the
+ *  CUDA stream passed as `stream` (a cudaStream_t; NULL = the legacy default stream) and the
+ *  call returns without waiting for it.
+ *
+ *  Errors: every entry point returns kta_status. Argument, size and alignment errors are found
+ *  before anything is enqueued and leave every output untouched. A launch failure returns
+ *  KTA_ERR_CUDA; kta_last_error() gives a one-line description (per host thread). No entry point
+ *  aborts, throws, or exits.
+ *
+ *  Supported sizes: d in {32, 64, 128}; bf16 softmax and chunk kernels need d in {64, 128};
+ *  KTA_F32 runs every branch on fp32 CUDA cores (the fp32 reference mode). B, F, P >= 1;
+ *  N = F*P < 2^31. Alignment: q, k, v, o 16-byte aligned; (ld_heads*d*elem) a multiple of 16.
+ *
+ *  Scales: softmax scores use `scale` (d^-1/2 is standard attention); GLA / delta outputs are
+ *  multiplied by `scale` (1.0 gives the pages' o_t = S_t q_t, which has no scale).
+ */
+#ifndef KTA_H
+#define KTA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KTA_VERSION 1
+
+typedef enum {
+  KTA_OK = 0,
+  KTA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, W < 1, dil < 1, ...          */
+  KTA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement (e.g. d = 96)  */
+  KTA_ERR_ALIGNMENT = 3,    /* pointer or row stride not 16-byte aligned                    */
+  KTA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed                          */
+  KTA_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired                           */
+  KTA_ERR_STATE = 6         /* handle misuse: destroyed handle, frame capacity exceeded      */
+} kta_status;
+
+typedef enum { KTA_BF16 = 0, KTA_F32 = 1 } kta_dtype;
+
+/* Frame grid of one call: B sequences of F frames of P tokens, head dimension d. */
+typedef struct {
+  int B, F, P, d;
+  kta_dtype dtype;
+} kta_shape;
+
+/* Human-readable name of a status code (static string). */
+const char* kta_status_str(kta_status s);
+
+/* Detail of the last failed call on this host thread ("" if none). */
+const char* kta_last_error(void);
+
+/* ABI version (KTA_VERSION of the build). */
+int kta_version(void);
+
+/*
+ * SWA -- paper-read, section 2, second pillar, SWA paragraph: standard softmax attention inside
+ * a window of L x window_size tokens. Query token t of frame f = t/P sees every key s of frames
+ * f-W+1 .. f (the own frame in full, no later frame):
+ *     o_t = sum_s softmax_s(scale * q_t . k_s) v_s.
+ * q, k, v, o: [B][N][ld_heads][d] (H heads computed). W >= 1 frames (W >= F gives full
+ * frame-causal attention).
+ */
+kta_status kta_swa_fwd(const void* q, const void* k, const void* v, void* o, kta_shape s,
+                       int H, int ld_heads, int W, float scale, void* stream);
+
+/*
+ * DSWA -- paper-read, section 2, second pillar, DSWA paragraph: the SWA window size, with
+ * frames taken every dil-th step: query frame f sees key frames f, f-dil, ..., f-(W-1)*dil.
+ * When dil divides F this equals SWA on the page's reshape (B, F*L, D) -> (B*dil, F/dil*L, D)
+ * with frame f in group f mod dil. dil = 1 is SWA.
+ */
+kta_status kta_dswa_fwd(const void* q, const void* k, const void* v, void* o, kta_shape s,
+                        int H, int ld_heads, int W, int dil, float scale, void* stream);
+
+/*
+ * GLA with a vector forget gate -- paper-read, section 2, second pillar, GLA paragraph (a
+ * fixed-size state updated once per token, gated forgetting):
+ *     S_t = diag(alpha_t) S_{t-1} + k_t^T v_t,     o_t = scale * q_t S_t
+ * token-causal over the flattened token order, S is d x d fp32, key-major (S[i][j], i over key
+ * dims). alpha: [B][N][H][d] fp32 in (0,1). S0: [B][H][d][d] initial state or NULL (= 0).
+ * S_out: [B][H][d][d] final state or NULL. chunk in {16, 32, 64} (the token block of the
+ * chunked form; results do not depend on it beyond rounding).
+ */
+kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* S0, float* S_out, void* o, kta_shape s, int H,
+                             int ld_heads, int chunk, float scale, void* stream);
+
+/*
+ * Gated delta rule -- paper-read, section 2, second pillar, the four update equations:
+ *     v_old = M_{t-1} k_t,   v_new = beta_t v_t + (1 - beta_t) v_old,
+ *     M_t = alpha_t M_{t-1} - v_old k_t^T + v_new k_t^T,   o_t = scale * M_t q_t
+ * with scalar alpha_t (forget gate) and beta_t per token and head: alpha, beta [B][N][H] fp32.
+ * The page's M is d_v x d_k; S0 / S_out hold its transpose S = M^T, [B][H][d][d] key-major,
+ * the same layout as kta_gla_chunk_fwd. NULL S0 = zero state.
+ */
+kta_status kta_gla_delta_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, float* S_out, void* o,
+                             kta_shape s, int H, int ld_heads, int chunk, float scale,
+                             void* stream);
+
+/*
+ * Hybrid layer. The pages say only that the three branches' outputs form one mixed temporal
+ * representation; this ABI splits heads: heads [0, n_swa) are SWA (window W_swa), the next
+ * n_dswa heads DSWA (window W_dswa, dilation dil), the last n_gla heads GLA (vector gate) or,
+ * with gla_delta = 1, the gated delta rule. Outputs are concatenated by head in o.
+ * q, k, v, o: [B][N][H][d] with H = n_swa + n_dswa + n_gla. alpha: [B][N][n_gla][d] (vector
+ * GLA) or [B][N][n_gla] (delta); beta: [B][N][n_gla] (delta only, else ignored).
+ * The softmax and GLA branches run concurrently on internal streams forked from `stream` and
+ * joined back into it before the call returns.
+ */
+typedef struct {
+  kta_shape s;
+  int n_swa, n_dswa, n_gla;
+  int W_swa, W_dswa, dil;
+  int chunk;
+  int gla_delta;
+  float scale_softmax, scale_gla;
+} kta_hybrid_cfg;
+
+kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* beta, void* o, void* stream);
+
+/*
+ * Streaming rollout -- paper-read, section 2, third pillar: low-latency rolling prediction, one
+ * frame at a time. A stream holds, per sequence, the GLA state and a ring of the last
+ * W_swa frames (SWA heads) or (W_dswa-1)*dil+1 frames (DSWA heads) of k and v. Each step takes
+ * one frame of P tokens ([B][P][H][d] q, k, v, o; alpha [B][P][n_gla](...)), appends its k, v to
+ * the rings, and produces exactly the rows of that frame that kta_hybrid_fwd would produce for
+ * the whole sequence. cfg->s.F is ignored. kta_stream_create allocates the rings and state on
+ * the current CUDA device; nothing else is allocated by steps.
+ */
+typedef struct kta_stream_s* kta_stream_t;
+
+kta_status kta_stream_create(const kta_hybrid_cfg* cfg, kta_stream_t* out);
+kta_status kta_stream_step(kta_stream_t st, const void* q_f, const void* k_f, const void* v_f,
+                           const float* alpha_f, const float* beta_f, void* o_f, void* stream);
+/* Back to frame 0 with a zero state (enqueued on `stream`). */
+kta_status kta_stream_reset(kta_stream_t st, void* stream);
+/* Frames consumed so far. */
+int64_t kta_stream_frame(kta_stream_t st);
+/* Size of the opaque state blob written by kta_stream_save (rings + GLA state + counter). */
+size_t kta_stream_state_bytes(kta_stream_t st);
+/* Copy the state to / from device memory of kta_stream_state_bytes bytes (on `stream`). A
+ * blob may be loaded into any stream created with an identical cfg. */
+kta_status kta_stream_save(kta_stream_t st, void* dev_dst, void* stream);
+kta_status kta_stream_load(kta_stream_t st, const void* dev_src, void* stream);
+/* Frees the rings and state; synchronises the device first. */
+kta_status kta_stream_destroy(kta_stream_t st);
+
+/*
+ * Device-side health. Every wait inside the library's kernels is bounded; a wait that runs out
+ * records a code in a device error word and lets its kernel finish cleanly instead of hanging.
+ * kta_device_status synchronises `stream`, returns KTA_ERR_TIMEOUT if such a code was recorded
+ * since the last call (and clears it), KTA_ERR_CUDA on a pending CUDA error, else KTA_OK.
+ */
+kta_status kta_device_status(void* stream);
+
+/*
+ * Diagnostic: launches one thread that waits on a barrier nobody arrives at, with a budget of
+ * `budget_cycles` SM clock cycles (1 .. 2^31), so that the bounded-wait path can be exercised
+ * without hanging the GPU. The next kta_device_status(stream) must return KTA_ERR_TIMEOUT.
+ */
+kta_status kta_selftest_wait_timeout(long long budget_cycles, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KTA_H */
