@@ -6,19 +6,23 @@
 //
 // Chunked form used here (exact algebra, C tokens per chunk, chunks aligned to multiples of C
 // from token 0). Let b_t = sum_{r <= t in chunk} log2 alpha_r (a vector over key dims), m the
-// chunk's middle token and S_0 the state at the chunk start:
-//   o_t   = scale * [ (q_t * 2^{b_t}) S_0 + sum_{s <= t} ((q_t * 2^{b_t - b_m}) . (k_s * 2^{b_m - b_s})) v_s ]
-//   S_end = diag(2^{b_C}) S_0 + sum_s (k_s * 2^{b_C - b_s})^T v_s
-// The middle reference point keeps both factors of the intra-chunk product within 2^{|b| over
-// half a chunk}; the state and inter-chunk factors are <= 1.
+// chunk's middle token, S_0 the state at the chunk start, and
+//   Qi_t = q_t * 2^{b_t - b_m},   Ki_s = k_s * 2^{b_m - b_s}   (elementwise over key dims).
+// Then
+//   o_t   = scale * [ Qi_t (diag(2^{b_m}) S_0) + sum_{s <= t} (Qi_t . Ki_s) v_s ]
+//   S_end = diag(2^{b_C - b_m}) [ diag(2^{b_m}) S_0 + Ki^T V ]
+// so one pair of decayed operands (one exp2 each per element) serves the intra-chunk scores, the
+// inter-chunk read-out and the state update. The middle reference point keeps both factors of the
+// intra-chunk product within 2^{|b| over half a chunk}; every other factor is <= 1.
 //
 // Sequence parallelism: the tokens of a sequence are split into segments of whole chunks.
 //   pass 1 (OUTPUT = false): each segment's end state from a zero start, and its total log2 decay;
-//   pass 2 (OUTPUT = true):  each segment folds S0 and the earlier segments' pass-1 results into
-//                            its start state, then runs the chunks and writes o.
+//   carry:                   S_start(0) = S0, S_start(s+1) = diag(2^{L_s}) S_start(s) + S_loc(s),
+//                            one thread per state element, written over S_loc in the workspace;
+//   pass 2 (OUTPUT = true):  each segment runs its chunks from S_start and writes o.
 // The value dimension is split in BV = 64 column slices (columns of S are independent).
-// CTA = 4 warps. Warp w computes output rows [16w, 16w+16) of a chunk and state rows
-// [w*D/4, (w+1)*D/4).
+// CTA = 4 warps, two CTAs per SM. Warp w computes output rows [16w, 16w+16) of a chunk and state
+// rows [w*D/4, (w+1)*D/4).
 #pragma once
 
 #include "mma_sync.cuh"
@@ -49,18 +53,17 @@ struct GlaSmem {
   static constexpr int BV = 64;
   static constexpr int LDK = D + 8;   // padded rows: conflict-free ldmatrix
   static constexpr int LDV = BV + 8;
-  __nv_bfloat16 q[C * LDK];   // raw q, then the intra-chunk query operand
-  __nv_bfloat16 qg[C * LDK];  // query decayed from the chunk start (inter-chunk operand)
-  __nv_bfloat16 k[C * LDK];   // raw k, then the intra-chunk key operand
-  __nv_bfloat16 kc[C * LDK];  // key decayed to the chunk end (state-update operand)
+  __nv_bfloat16 q[C * LDK];   // raw q, then Qi
+  __nv_bfloat16 k[C * LDK];   // raw k, then Ki
   __nv_bfloat16 v[C * LDV];
-  __nv_bfloat16 s[D * LDV];   // bf16 copy of the chunk-start state slice
+  __nv_bfloat16 s[D * LDV];   // bf16 copy of diag(2^{b_m}) S_0 (value slice)
   float g[C * D];             // alpha, then the cumulative log2 gate b_t
-  float gend[D];              // 2^{b_C}
+  float emid[D];              // 2^{b_m}
+  float cend[D];              // 2^{b_C - b_m}
 };
 
 template <int D, int C, bool OUTPUT>
-__global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
+__global__ void __launch_bounds__(128, 2) gla_chunk_kernel(const GlaParams p) {
   using SM = GlaSmem<D, C>;
   constexpr int BV = SM::BV, LDK = SM::LDK, LDV = SM::LDV;
   constexpr int RW = D / 4;           // state rows per warp
@@ -92,44 +95,39 @@ __global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
       for (int r = 0; r < 4; ++r) st[mt][nt][r] = 0.f;
 
   if (OUTPUT) {
-    const long long sb = static_cast<long long>(bh) * D * D;
-    if (p.S0) {
+    // start state: S0 for a single segment, else the carry kernel's S_start of this segment
+    const float* Ss = p.nseg > 1 ? p.ws_S + (static_cast<long long>(bh) * p.nseg + seg) * D * D
+                                 : (p.S0 ? p.S0 + static_cast<long long>(bh) * D * D : nullptr);
+    if (Ss) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
-            st[mt][nt][r] = p.S0[sb + srow(mt, r) * D + j0 + scol(nt, r)];
-    }
-    for (int s2 = 0; s2 < seg; ++s2) {
-      const float* L = p.ws_L + (static_cast<long long>(bh) * p.nseg + s2) * D;
-      const float* Sl = p.ws_S + (static_cast<long long>(bh) * p.nseg + s2) * D * D;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int row = srow(mt, r);
-          const float dec = exp2f(L[row]);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            st[mt][nt][r] = fmaf(dec, st[mt][nt][r], Sl[row * D + j0 + scol(nt, r)]);
-        }
+          for (int r = 0; r < 4; ++r) st[mt][nt][r] = Ss[srow(mt, r) * D + j0 + scol(nt, r)];
     }
   }
   float ltot = 0.f;  // this thread's key dim (tid < D): total log2 decay over the segment
 
-  auto write_state_smem = [&]() {
+  // Scale the state rows by 2^{b_m} (registers) and keep a bf16 copy for the inter-chunk product.
+  auto prescale_and_publish = [&]() {
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int mt = 0; mt < MT; ++mt) {
+      const float ea = sm.emid[srow(mt, 0)], eb = sm.emid[srow(mt, 2)];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int r0 = srow(mt, 0), c0 = scol(nt, 0);
-        *reinterpret_cast<uint32_t*>(&sm.s[r0 * LDV + c0]) = bf16x2(st[mt][nt][0], st[mt][nt][1]);
-        *reinterpret_cast<uint32_t*>(&sm.s[(r0 + 8) * LDV + c0]) = bf16x2(st[mt][nt][2], st[mt][nt][3]);
+        st[mt][nt][0] *= ea;
+        st[mt][nt][1] *= ea;
+        st[mt][nt][2] *= eb;
+        st[mt][nt][3] *= eb;
+        if (OUTPUT) {
+          const int r0 = srow(mt, 0), c0 = scol(nt, 0);
+          *reinterpret_cast<uint32_t*>(&sm.s[r0 * LDV + c0]) = bf16x2(st[mt][nt][0], st[mt][nt][1]);
+          *reinterpret_cast<uint32_t*>(&sm.s[(r0 + 8) * LDV + c0]) = bf16x2(st[mt][nt][2], st[mt][nt][3]);
+        }
       }
+    }
   };
-  if (OUTPUT) write_state_smem();
 
   for (int c0 = t_begin; c0 < t_end; c0 += C) {
     const int n = min(C, t_end - c0);
@@ -164,34 +162,28 @@ __global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
       cp_async_wait_all();
     }
     __syncthreads();
-    // ---- cumulative log2 gate per key dim
+    // ---- cumulative log2 gate per key dim, and the per-dim factors 2^{b_m}, 2^{b_C - b_m}
     if (tid < D) {
-      float acc = 0.f;
+      float acc = 0.f, bm = 0.f;
 #pragma unroll 8
       for (int t = 0; t < C; ++t) {
         acc += __log2f(sm.g[t * D + tid]);
         sm.g[t * D + tid] = acc;
+        if (t == MID) bm = acc;
       }
-      sm.gend[tid] = exp2f(acc);
+      sm.emid[tid] = exp2f(bm);
+      sm.cend[tid] = exp2f(acc - bm);
       ltot += acc;
     }
     __syncthreads();
-    // ---- decayed operands
+    // ---- decayed operands (in place) and the pre-scaled state
     for (int idx = tid; idx < C * D; idx += 128) {
       const int t = idx / D, i = idx % D;
-      const float bt = sm.g[t * D + i];
-      const float bl = sm.g[(C - 1) * D + i];
-      const float kv = __bfloat162float(sm.k[t * LDK + i]);
-      sm.kc[t * LDK + i] = __float2bfloat16_rn(kv * exp2f(bl - bt));
-      if (OUTPUT) {
-        const float bm = sm.g[MID * D + i];
-        const float qv = __bfloat162float(sm.q[t * LDK + i]);
-        const float e = exp2f(bt - bm);
-        sm.q[t * LDK + i] = __float2bfloat16_rn(qv * e);
-        sm.qg[t * LDK + i] = __float2bfloat16_rn(qv * exp2f(bt));
-        sm.k[t * LDK + i] = __float2bfloat16_rn(kv * exp2f(bm - bt));
-      }
+      const float d = sm.g[t * D + i] - sm.g[MID * D + i];
+      sm.k[t * LDK + i] = __float2bfloat16_rn(__bfloat162float(sm.k[t * LDK + i]) * exp2f(-d));
+      if (OUTPUT) sm.q[t * LDK + i] = __float2bfloat16_rn(__bfloat162float(sm.q[t * LDK + i]) * exp2f(d));
     }
+    prescale_and_publish();
     __syncthreads();
 
     if (OUTPUT && warp < RT) {
@@ -246,17 +238,15 @@ __global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
           mma16816(ov[2 * np + 1], pa[kk], bv[2], bv[3]);
         }
       }
-      // O += Qg S_0
+      // O += Qi diag(2^{b_m}) S_0
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t ag[4];
-        ldsm_x4(ag, &sm.qg[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
           uint32_t bs[4];
           ldsm_x4_t(bs, &sm.s[frag_b_kmajor(lane, kk * 16, np * 16, LDV)]);
-          mma16816(ov[2 * np], ag, bs[0], bs[1]);
-          mma16816(ov[2 * np + 1], ag, bs[2], bs[3]);
+          mma16816(ov[2 * np], aq[kk], bs[0], bs[1]);
+          mma16816(ov[2 * np + 1], aq[kk], bs[2], bs[3]);
         }
       }
       // store rows < n
@@ -273,15 +263,7 @@ __global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
       }
     }
 
-    // ---- state update: S = diag(2^{b_C}) S + Kc^T V  (all warps)
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float dec = sm.gend[srow(mt, r)];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) st[mt][nt][r] *= dec;
-      }
+    // ---- state update: S = diag(2^{b_C - b_m}) (diag(2^{b_m}) S + Ki^T V)  (all warps)
 #pragma unroll
     for (int kk = 0; kk < C / 16; ++kk) {
       uint32_t bv[NT / 2][4];
@@ -290,7 +272,7 @@ __global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         uint32_t ak[4];
-        ldsm_x4_t(ak, &sm.kc[frag_a_kmajor(lane, warp * RW + mt * 16, kk * 16, LDK)]);
+        ldsm_x4_t(ak, &sm.k[frag_a_kmajor(lane, warp * RW + mt * 16, kk * 16, LDK)]);
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
           mma16816(st[mt][2 * np], ak, bv[np][0], bv[np][1]);
@@ -298,8 +280,18 @@ __global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
         }
       }
     }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const float ca = sm.cend[srow(mt, 0)], cb = sm.cend[srow(mt, 2)];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        st[mt][nt][0] *= ca;
+        st[mt][nt][1] *= ca;
+        st[mt][nt][2] *= cb;
+        st[mt][nt][3] *= cb;
+      }
+    }
     __syncthreads();
-    if (OUTPUT) write_state_smem();
   }
 
   if (!OUTPUT) {
@@ -319,6 +311,38 @@ __global__ void __launch_bounds__(128) gla_chunk_kernel(const GlaParams p) {
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int r = 0; r < 4; ++r) So[srow(mt, r) * D + j0 + scol(nt, r)] = st[mt][nt][r];
+  }
+}
+
+// Segment carry: for one (sequence, head) and one state element (i, j), walk the segments in
+// order, replacing each segment's local end state by the state at its start:
+//   S_start(0) = S0 (or 0),  S_start(s+1) = 2^{L_s[i]} S_start(s) + S_loc(s).
+// All loads of a group of segments are issued before the dependent chain of FMAs.
+template <int D>
+__global__ void __launch_bounds__(128) gla_carry_kernel(const GlaParams p) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * 128 + threadIdx.x;  // element index i * D + j
+  if (e >= D * D) return;
+  const int i = e / D;
+  float cur = p.S0 ? p.S0[static_cast<long long>(bh) * D * D + e] : 0.f;
+  float* S = p.ws_S + static_cast<long long>(bh) * p.nseg * D * D + e;
+  const float* L = p.ws_L + static_cast<long long>(bh) * p.nseg * D + i;
+  constexpr int G = 8;
+  for (int s0 = 0; s0 < p.nseg; s0 += G) {
+    float sl[G], dl[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+      const bool in = s0 + u < p.nseg;
+      sl[u] = in ? S[static_cast<long long>(s0 + u) * D * D] : 0.f;
+      dl[u] = in ? L[static_cast<long long>(s0 + u) * D] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+      if (s0 + u < p.nseg) {
+        S[static_cast<long long>(s0 + u) * D * D] = cur;
+        cur = fmaf(exp2f(dl[u]), cur, sl[u]);
+      }
+    }
   }
 }
 

@@ -13,6 +13,7 @@
 #include <mutex>
 #include <string>
 #include <utility>
+#include <vector>
 
 #include "kta.h"
 #include "kta_ptx.cuh"
@@ -159,6 +160,41 @@ kta_status set_smem_attr(K kernel, size_t bytes) {
   return KTA_OK;
 }
 
+// ------------------------------------------------------------------------- tracing
+
+struct TraceRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+
+struct TraceState {
+  bool on = false;
+  std::vector<TraceRec> recs;
+};
+
+TraceState& trace_state() {
+  thread_local TraceState t;
+  return t;
+}
+
+// Brackets one kernel launch with events on its stream while tracing is on.
+struct TraceScope {
+  TraceRec rec{nullptr, nullptr, nullptr};
+  cudaStream_t st;
+  TraceScope(const char* name, cudaStream_t s) : st(s) {
+    TraceState& t = trace_state();
+    if (!t.on) return;
+    if (cudaEventCreate(&rec.a) != cudaSuccess || cudaEventCreate(&rec.b) != cudaSuccess) return;
+    rec.name = name;
+    cudaEventRecord(rec.a, st);
+  }
+  ~TraceScope() {
+    if (!rec.name) return;
+    cudaEventRecord(rec.b, st);
+    trace_state().recs.push_back(rec);
+  }
+};
+
 // ------------------------------------------------------------------------- softmax launches
 
 struct WinGroup {
@@ -216,14 +252,26 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   p.scale_log2 = L.scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(L.o);
   p.o_ld = L.o_ld;
-  const long long nblk = static_cast<long long>(L.Fq) * Htot * L.B * p.n_qt;
+  const long long nblk = static_cast<long long>(L.Fq) * Htot * L.B * p.n_qt;  // one CTA per tile
   if (nblk <= 0) return KTA_OK;
-  if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "grid too large (%lld CTAs)", nblk);
+  if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "too many tiles (%lld)", nblk);
   const size_t smem = kta::win_smem_bytes<D>();
   if ((s = set_smem_attr(kta::win_attn_tc_kernel<D>, smem))) return s;
-  kta::win_attn_tc_kernel<D><<<static_cast<unsigned>(nblk), 192, smem, st>>>(tq, tk0, tv0, tk1,
-                                                                             tv1, p);
-  KTA_CUDA(cudaGetLastError());
+  {
+    TraceScope ts("win_attn_tc", st);
+    kta::win_attn_tc_kernel<D><<<static_cast<unsigned>(nblk), 192, smem, st>>>(tq, tk0, tv0, tk1,
+                                                                               tv1, p);
+  }
+  const cudaError_t le = cudaGetLastError();
+  if (le != cudaSuccess) {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, kta::win_attn_tc_kernel<D>);
+    return fail(KTA_ERR_CUDA,
+                "win_attn_tc launch failed: %s (grid %lld x 192, dyn smem %zu, regs %d, max threads "
+                "%d, max dyn smem %d)",
+                cudaGetErrorString(le), nblk, smem, fa.numRegs, fa.maxThreadsPerBlock,
+                fa.maxDynamicSharedSizeBytes);
+  }
   return KTA_OK;
 }
 
@@ -252,10 +300,13 @@ kta_status launch_win_f32(const WinLaunch& L, cudaStream_t st) {
   const WinGroup& g1 = L.g[1].H > 0 ? L.g[1] : L.g[0];
   dim3 grid((L.Fq * L.P + 3) / 4, p.Htot, L.B);
   if (grid.y > 65535 || grid.z > 65535) return fail(KTA_ERR_UNSUPPORTED, "too many heads/batches");
-  kta::win_attn_f32_kernel<<<grid, 128, 0, st>>>(
-      static_cast<const float*>(L.q), static_cast<const float*>(L.g[0].k),
-      static_cast<const float*>(L.g[0].v), static_cast<const float*>(g1.k),
-      static_cast<const float*>(g1.v), static_cast<float*>(L.o), p);
+  {
+    TraceScope ts("win_attn_f32", st);
+    kta::win_attn_f32_kernel<<<grid, 128, 0, st>>>(
+        static_cast<const float*>(L.q), static_cast<const float*>(L.g[0].k),
+        static_cast<const float*>(L.g[0].v), static_cast<const float*>(g1.k),
+        static_cast<const float*>(g1.v), static_cast<float*>(L.o), p);
+  }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
@@ -330,10 +381,21 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
   if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
   dim3 grid(nseg, slices, L.B * L.H);
   if (nseg > 1) {
-    kta::gla_chunk_kernel<D, C, false><<<grid, 128, smem, st>>>(p);
+    {
+      TraceScope ts("gla_chunk_state", st);
+      kta::gla_chunk_kernel<D, C, false><<<grid, 128, smem, st>>>(p);
+    }
     KTA_CUDA(cudaGetLastError());
+    {
+      TraceScope ts("gla_carry", st);
+      kta::gla_carry_kernel<D><<<dim3((D * D + 127) / 128, L.B * L.H), 128, 0, st>>>(p);
+    }
   }
-  kta::gla_chunk_kernel<D, C, true><<<grid, 128, smem, st>>>(p);
+  KTA_CUDA(cudaGetLastError());
+  {
+    TraceScope ts("gla_chunk_out", st);
+    kta::gla_chunk_kernel<D, C, true><<<grid, 128, smem, st>>>(p);
+  }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
@@ -360,7 +422,10 @@ kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
   if ((sa = set_smem_attr(kta::delta_chunk_kernel<D>, smem))) return sa;
   if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
   dim3 grid(D / SM::BV, L.B * L.H);
-  kta::delta_chunk_kernel<D><<<grid, 128, smem, st>>>(p);
+  {
+    TraceScope ts("delta_chunk", st);
+    kta::delta_chunk_kernel<D><<<grid, 128, smem, st>>>(p);
+  }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
@@ -379,6 +444,7 @@ kta_status launch_rec_f32(const LinLaunch& L, cudaStream_t st) {
   p.S_out = L.S_out;
   if (L.B > 65535) return fail(KTA_ERR_UNSUPPORTED, "B > 65535");
   dim3 grid(L.H, L.B);
+  TraceScope ts(L.delta ? "delta_rec_f32" : "gla_rec_f32", st);
   if (L.delta)
     kta::delta_rec_f32_kernel<D><<<grid, D, 0, st>>>(
         static_cast<const float*>(L.q), static_cast<const float*>(L.k),
@@ -653,16 +719,18 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
     if ((r = launch_win(W, st))) return r;
     return launch_lin(L, st);
   }
+  // The persistent softmax kernel is launched first and takes every SM; the GLA kernels, forked
+  // onto a side stream, fill SMs as soon as softmax CTAs retire (the tail of the softmax pass).
   ThreadStreams* ts = nullptr;
   if ((r = thread_streams(&ts))) return r;
   KTA_CUDA(cudaEventRecord(ts->fork, st));
+  kta_status r_win = launch_win(W, st);
   KTA_CUDA(cudaStreamWaitEvent(ts->side, ts->fork, 0));
   kta_status r_lin = launch_lin(L, ts->side);
   KTA_CUDA(cudaEventRecord(ts->join, ts->side));
-  kta_status r_win = launch_win(W, st);
   KTA_CUDA(cudaStreamWaitEvent(st, ts->join, 0));
-  if (r_lin) return r_lin;
-  return r_win;
+  if (r_win) return r_win;
+  return r_lin;
 }
 
 // --------------------------------------------------------------------------- streaming
@@ -952,6 +1020,47 @@ kta_status kta_stream_destroy(kta_stream_t s) {
     return fail(KTA_ERR_CUDA, "stream teardown failed: %s",
                 cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
   return KTA_OK;
+}
+
+// --------------------------------------------------------------------------- tracing
+
+kta_status kta_trace_begin(void) {
+  TraceState& t = trace_state();
+  for (TraceRec& r : t.recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  t.recs.clear();
+  t.on = true;
+  return KTA_OK;
+}
+
+kta_status kta_trace_end(int* n, const char** names, int* launches, double* total_ms, int cap) {
+  TraceState& t = trace_state();
+  t.on = false;
+  std::vector<const char*> keys;
+  std::map<const char*, std::pair<int, double>> agg;
+  kta_status st = KTA_OK;
+  for (TraceRec& r : t.recs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess && st == KTA_OK)
+      st = fail(KTA_ERR_CUDA, "trace event read failed: %s", cudaGetErrorString(e));
+    if (!agg.count(r.name)) keys.push_back(r.name);
+    agg[r.name].first += 1;
+    agg[r.name].second += ms;
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  t.recs.clear();
+  if (n) *n = static_cast<int>(keys.size());
+  for (int i = 0; i < static_cast<int>(keys.size()) && i < cap; ++i) {
+    if (names) names[i] = keys[i];
+    if (launches) launches[i] = agg[keys[i]].first;
+    if (total_ms) total_ms[i] = agg[keys[i]].second;
+  }
+  return st;
 }
 
 // --------------------------------------------------------------------------- diagnostics

@@ -61,6 +61,9 @@ _SIGS = {
     "kta_stream_destroy": ([_vp], _st),
     "kta_device_status": ([_vp], _st),
     "kta_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _st),
+    "kta_trace_begin": ([], _st),
+    "kta_trace_end": ([ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_i),
+                       ctypes.POINTER(ctypes.c_double), _i], _st),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -260,6 +263,27 @@ def device_status(stream=None):
 def selftest_wait_timeout(budget_cycles: int, stream=None):
     _check(_lib.kta_selftest_wait_timeout(int(budget_cycles), _stream(stream)),
            "kta_selftest_wait_timeout")
+
+
+class trace:
+    """Context manager: per-kernel launch counts and device milliseconds of every library kernel
+    launched inside the block (CUDA events on each launch's own stream)."""
+
+    def __enter__(self):
+        _check(_lib.kta_trace_begin(), "kta_trace_begin")
+        self.kernels = {}
+        return self
+
+    def __exit__(self, *exc):
+        cap = 32
+        n = _i()
+        names = (ctypes.c_char_p * cap)()
+        launches = (_i * cap)()
+        ms = (ctypes.c_double * cap)()
+        _check(_lib.kta_trace_end(ctypes.byref(n), names, launches, ms, cap), "kta_trace_end")
+        self.kernels = {names[i].decode(): {"launches": launches[i], "ms": ms[i]}
+                        for i in range(min(n.value, cap))}
+        return False
 
 
 def raw_call(name: str, *args) -> int:

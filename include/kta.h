@@ -184,6 +184,16 @@ kta_status kta_device_status(void* stream);
  */
 kta_status kta_selftest_wait_timeout(long long budget_cycles, void* stream);
 
+/*
+ * Tracing. Between kta_trace_begin() and kta_trace_end(), every kernel the library launches from
+ * this host thread is bracketed by a pair of CUDA events recorded on the stream it is launched
+ * on. kta_trace_end synchronises those events and fills, for up to `cap` distinct kernels, the
+ * kernel name (static string), its launch count and its summed device time in milliseconds;
+ * *n receives the number of distinct kernels. Tracing adds two event records per launch.
+ */
+kta_status kta_trace_begin(void);
+kta_status kta_trace_end(int* n, const char** names, int* launches, double* total_ms, int cap);
+
 #ifdef __cplusplus
 }
 #endif
