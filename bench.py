@@ -71,10 +71,19 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "win_attn_tc": ("win_attn_tc.cuh", "kta_ptx.cuh"),
+    "gla_chunk_state": ("gla_chunk.cuh", "mma_sync.cuh"),
+    "gla_chunk_out": ("gla_chunk.cuh", "mma_sync.cuh"),
+    "delta_chunk": ("delta_chunk.cuh", "mma_sync.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the source files a kernel is built from (its ncu counters go stale when it moves)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hybrid_linear_temporal_kta_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -89,7 +98,7 @@ def recorded_traffic(kernel: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
