@@ -1099,3 +1099,152 @@ extern "C" kta_status kta_selftest_wait_timeout(long long budget_cycles, void* s
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
+
+// =========================================================================== no-allocation GLA
+//
+// kta_gla_chunk_fwd allocates its segment workspace with cudaMalloc the first time it needs it
+// (and when a larger call needs more). Some callers cannot allocate device memory at call time:
+// a real-time rollout loop that forbids allocation once it is running, or a process whose device
+// memory is entirely held by another allocator's pool. kta_gla_chunk_fwd_noalloc serves them:
+// the same kernels and segment plan, with the workspace in the fixed device array below instead.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
+constexpr int kNoAllocMaxDevices = 64;
+
+// Segment states and decays of the chunked GLA. Every device that loads the library holds this
+// array until the process exits. Every call shares it and it keeps the last call's contents.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+void* g_noalloc_ptr[kNoAllocMaxDevices];
+cudaError_t g_noalloc_err[kNoAllocMaxDevices];
+
+// Device address of the scratch array on the current device. Host code must not pass the
+// symbol itself to a kernel (on the host it is only a stand-in); the address is looked up once
+// per device, with that device current.
+kta_status noalloc_scratch(void** out) {
+  int dev = 0;
+  KTA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(KTA_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kNoAllocMaxDevices - 1);
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = p;
+  });
+  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev])
+    return fail(KTA_ERR_CUDA, "cudaGetSymbolAddress of the scratch array failed: %s",
+                cudaGetErrorString(g_noalloc_err[dev]));
+  *out = g_noalloc_ptr[dev];
+  return KTA_OK;
+}
+
+// Same segment plan and kernels as launch_gla_chunk; the workspace is the scratch array.
+template <int D, int C>
+kta_status launch_gla_chunk_noalloc(const LinLaunch& L, cudaStream_t st) {
+  using SM = kta::GlaSmem<D, C>;
+  const int slices = D / SM::BV;
+  const long long base = static_cast<long long>(L.B) * L.H * slices;
+  const int nchunks = (L.N + C - 1) / C;
+  const long long want = (4LL * 148 + base - 1) / base;
+  int nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
+  const int seg_chunks = (nchunks + nseg - 1) / nseg;
+  const int seg_len = seg_chunks * C;
+  nseg = (L.N + seg_len - 1) / seg_len;
+  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
+  const size_t need =
+      nseg > 1 ? static_cast<size_t>(L.B) * L.H * nseg * (size_t(D) * D + D) * 4 : 0;
+  if (need > kNoAllocScratchBytes)
+    return fail(KTA_ERR_UNSUPPORTED,
+                "needs %zu bytes of scratch; the no-allocation variant has %zu (use "
+                "kta_gla_chunk_fwd, or fewer sequences x heads per call)",
+                need, kNoAllocScratchBytes);
+  kta::GlaParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(L.q);
+  p.k = static_cast<const __nv_bfloat16*>(L.k);
+  p.v = static_cast<const __nv_bfloat16*>(L.v);
+  p.alpha = L.alpha;
+  p.o = static_cast<__nv_bfloat16*>(L.o);
+  p.ld = L.ld;
+  p.rows_b = L.rows_b;
+  p.N = L.N;
+  p.H = L.H;
+  p.seg_len = seg_len;
+  p.nseg = nseg;
+  p.scale = L.scale;
+  p.S0 = L.S0;
+  p.S_out = L.S_out;
+  if (nseg > 1) {
+    // Every word the kernels read from the scratch is written earlier in the same call (pass 1
+    // writes all segment states and decays, the carry pass rewrites them in place), so nothing
+    // has to be cleared.
+    void* ws = nullptr;
+    kta_status r = noalloc_scratch(&ws);
+    if (r) return r;
+    p.ws_S = static_cast<float*>(ws);
+    p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * nseg * D * D;
+  }
+  const size_t smem = sizeof(SM);
+  KTA_CUDA(cudaFuncSetAttribute(kta::gla_chunk_kernel<D, C, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+  KTA_CUDA(cudaFuncSetAttribute(kta::gla_chunk_kernel<D, C, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+  dim3 grid(nseg, slices, L.B * L.H);
+  if (nseg > 1) {
+    kta::gla_chunk_kernel<D, C, false><<<grid, 128, smem, st>>>(p);
+    KTA_CUDA(cudaGetLastError());
+    kta::gla_carry_kernel<D><<<dim3((D * D + 127) / 128, L.B * L.H), 128, 0, st>>>(p);
+    KTA_CUDA(cudaGetLastError());
+  }
+  kta::gla_chunk_kernel<D, C, true><<<grid, 128, smem, st>>>(p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+}  // namespace
+
+extern "C" kta_status kta_gla_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                                const float* alpha, const float* S0, float* S_out,
+                                                void* o, kta_shape s, int H, int ld_heads,
+                                                int chunk, float scale, void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) || (r = check_ptrs({q, k, v, o})))
+    return r;
+  if (!alpha) return fail(KTA_ERR_INVALID_ARG, "null gate pointer");
+  if (!aligned16(alpha) || (S0 && !aligned16(S0)) || (S_out && !aligned16(S_out)))
+    return fail(KTA_ERR_ALIGNMENT, "gate / state pointers must be 16-byte aligned");
+  if (chunk != 16 && chunk != 32 && chunk != 64)
+    return fail(KTA_ERR_INVALID_ARG, "chunk must be 16, 32 or 64");
+  if (!std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be finite");
+  if (s.dtype != KTA_BF16 || (s.d != 64 && s.d != 128))
+    return fail(KTA_ERR_UNSUPPORTED,
+                "the no-allocation variant covers the bf16 chunked kernel (d = 64 or 128)");
+  LinLaunch L;
+  L.B = s.B;
+  L.N = s.F * s.P;
+  L.H = H;
+  L.d = s.d;
+  L.rows_b = L.N;
+  L.chunk = chunk;
+  L.dt = s.dtype;
+  L.q = q;
+  L.k = k;
+  L.v = v;
+  L.o = o;
+  L.ld = static_cast<long long>(ld_heads) * s.d;
+  L.alpha = alpha;
+  L.S0 = S0;
+  L.S_out = S_out;
+  L.scale = scale;
+  cudaStream_t st = as_stream(stream);
+  if (s.d == 128) {
+    if (chunk == 64) return launch_gla_chunk_noalloc<128, 64>(L, st);
+    if (chunk == 32) return launch_gla_chunk_noalloc<128, 32>(L, st);
+    return launch_gla_chunk_noalloc<128, 16>(L, st);
+  }
+  if (chunk == 64) return launch_gla_chunk_noalloc<64, 64>(L, st);
+  if (chunk == 32) return launch_gla_chunk_noalloc<64, 32>(L, st);
+  return launch_gla_chunk_noalloc<64, 16>(L, st);
+}

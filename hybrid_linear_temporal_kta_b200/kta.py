@@ -50,6 +50,8 @@ _SIGS = {
     "kta_gla_chunk_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp], _st),
     "kta_gla_delta_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
                           _st),
+    "kta_gla_chunk_fwd_noalloc": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
+                                  _st),
     "kta_hybrid_fwd": ([ctypes.POINTER(HybridCfg), _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
     "kta_stream_create": ([ctypes.POINTER(HybridCfg), ctypes.POINTER(_vp)], _st),
     "kta_stream_step": ([_vp, _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),

@@ -108,6 +108,28 @@ kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const 
                              int ld_heads, int chunk, float scale, void* stream);
 
 /*
+ * kta_gla_chunk_fwd without any device allocation. The pages have no counterpart: this is a
+ * service for callers that cannot allocate device memory while they run -- a real-time rollout
+ * loop that forbids allocation once started, or a process whose device memory is entirely held
+ * by another allocator's pool. kta_gla_chunk_fwd takes its segment workspace from a cache it
+ * grows with cudaMalloc; this variant runs the same kernels and segment plan with the workspace
+ * in a fixed 32 MiB array in device memory, which every GPU that loads the library holds until
+ * the process exits. It calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - bf16 only, d in {64, 128}; other arguments and results as kta_gla_chunk_fwd.
+ *  - A call whose workspace would exceed 32 MiB (sequences x heads x segments x (d*d + d) x 4
+ *    bytes) returns KTA_ERR_UNSUPPORTED with the size it needs, before anything is enqueued.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *    with that device current); make that first call before any stream capture.
+ *  - Every call shares the array and leaves its contents behind; each call writes all the
+ *    scratch it reads before reading it, so nothing needs clearing. Calls that overlap on the
+ *    GPU (for example on two streams) race on the array: serialise them.
+ */
+kta_status kta_gla_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                     const float* alpha, const float* S0, float* S_out, void* o,
+                                     kta_shape s, int H, int ld_heads, int chunk, float scale,
+                                     void* stream);
+
+/*
  * Gated delta rule -- paper-read, section 2, second pillar, the four update equations:
  *     v_old = M_{t-1} k_t,   v_new = beta_t v_t + (1 - beta_t) v_old,
  *     M_t = alpha_t M_{t-1} - v_old k_t^T + v_new k_t^T,   o_t = scale * M_t q_t

@@ -1,0 +1,83 @@
+"""GPU test of kta_gla_chunk_fwd_noalloc, the GLA entry point that allocates no device memory.
+
+It exists for callers that cannot allocate device memory while they run (a real-time rollout loop
+that forbids allocation once started, or a process whose device memory belongs to another
+allocator's pool): it runs the chunked GLA kernels with their segment workspace in a fixed
+device array instead of memory obtained with cudaMalloc. This file is named to be collected last,
+so that a run stopping at the first failure has run every other test first; it also passes on its
+own in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from hybrid_linear_temporal_kta_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def kta():
+    from hybrid_linear_temporal_kta_b200 import build
+    build.build()
+    from hybrid_linear_temporal_kta_b200 import kta as mod
+    return mod
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _noalloc(kta, q, k, v, alpha, S0, S_out, o, chunk):
+    B, N, H, d = q.shape
+    shape = kta.Shape(B, 1, N, d, kta.BF16)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return kta.raw_call("kta_gla_chunk_fwd_noalloc", _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                        _ptr(S0), _ptr(S_out), _ptr(o), shape, H, H, chunk, ctypes.c_float(1.0),
+                        stream)
+
+
+def _rel(a, b):
+    a = a.double().cpu().numpy()
+    b = b.double().cpu().numpy()
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def test_noalloc_matches_allocating_entry_point_on_two_calls(kta):
+    cases = [
+        # (B, N, H, d, chunk): both use many segments, so the scratch array is in use
+        (1, 20000, 2, 128, 64),
+        (2, 9000, 1, 64, 32),
+    ]
+    for i, (B, N, H, d, chunk) in enumerate(cases):
+        w = synth.HYBRID_BF16.replace(d=d, n_swa=0, n_dswa=0, n_gla=H, chunk=chunk)
+        x = synth.make_inputs(w, N=N, B=B, seed_base=7000 + 10 * i)
+        q, k, v, a = (x[n].cuda() for n in ("q", "k", "v", "alpha"))
+        S0 = torch.randn(B, H, d, d, device="cuda", dtype=torch.float32)
+        o_ref, S_ref = kta.gla_chunk_fwd(q, k, v, a, chunk=chunk, S0=S0, return_state=True)
+        o = torch.full_like(q, float("nan"))
+        S_out = torch.full_like(S_ref, float("nan"))
+        st = _noalloc(kta, q, k, v, a, S0, S_out, o, chunk)
+        assert st == 0, kta.last_error()
+        torch.cuda.synchronize()
+        kta.device_status()
+        assert _rel(o, o_ref) <= BF16_TOL
+        assert _rel(S_out, S_ref) <= BF16_TOL
+
+
+def test_noalloc_rejects_a_workspace_above_its_maximum(kta):
+    # 8 sequences x 32 heads of 4096 tokens (d = 128) need about 34 MB of segment workspace,
+    # more than the 32 MiB array: refused before anything is enqueued, outputs untouched.
+    B, N, H, d = 8, 4096, 32, 128
+    q = torch.zeros(B, N, H, d, device="cuda", dtype=torch.bfloat16)
+    a = torch.ones(B, N, H, d, device="cuda", dtype=torch.float32)
+    o = torch.full_like(q, 3.0)
+    st = _noalloc(kta, q, q, q, a, None, None, o, 64)
+    assert st == 2  # KTA_ERR_UNSUPPORTED
+    assert "scratch" in kta.last_error()
+    torch.cuda.synchronize()
+    assert torch.all(o == 3.0)
