@@ -165,6 +165,27 @@ def dist_env():
     return ws, rank, local
 
 
+def reduce_max(val: float, ws: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (the job's time is its slowest rank's)."""
+    if ws == 1:
+        return val
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([val], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(ws: int, tokens_per_rank_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own sequences (weak scaling)."""
+    return ws * tokens_per_rank_step * steps / (ms_max / 1e3)
+
+
+def rank_seed_base(base: int, rank: int) -> int:
+    """Each rank draws its own sequences."""
+    return base + 100 * rank
+
+
 # --------------------------------------------------------------------------- CPU oracle timing
 
 
@@ -184,16 +205,17 @@ def oracle_sample(w, x, target_s: float = 12.0):
     hs, hd = (0, w.n_swa), (w.n_swa, w.n_swa + w.n_dswa)
     hg = (w.n_swa + w.n_dswa, w.H)
 
+    out = np.full(q.shape, np.nan)  # written only at the sampled rows; allocated once
+
     def run(M):
         rows = np.sort(rng.choice(w.N, size=M, replace=False))
         t0 = time.perf_counter()
-        out = np.full(q.shape, np.nan)
         oracle.swa(q, k, v, w.P, w.W_swa, w.scale_softmax, heads=hs, rows=rows, out=out)
         oracle.dswa(q, k, v, w.P, w.W_dswa, w.dil, w.scale_softmax, heads=hd, rows=rows, out=out)
         oracle.gla(q[:, :M], k[:, :M], v[:, :M], a[:, :M], heads=hg)
         return time.perf_counter() - t0
 
-    M = 64
+    M = 256
     t = run(M)
     M = int(min(w.N, max(64, M * target_s / max(t, 1e-3))))
     t = run(M)
@@ -248,7 +270,7 @@ def run_kta(args):
     from hybrid_linear_temporal_kta_b200 import kta, synth
 
     w = synth.HYBRID_BF16
-    x = synth.make_inputs(w, seed_base=w.seed_base + 100 * rank)
+    x = synth.make_inputs(w, seed_base=rank_seed_base(w.seed_base, rank))
     cfg = kta.cfg_from_workload(w)
     host = {n: x[n].pin_memory() for n in ("q", "k", "v", "alpha")}
     devx = {n: host[n].cuda() for n in host}
@@ -264,11 +286,7 @@ def run_kta(args):
             dist.barrier()
 
     def max_over_ranks(val: float) -> float:
-        if ws == 1:
-            return val
-        t = torch.tensor([val], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(val, ws, torch.device("cuda", local))
 
     for _ in range(args.warmup):
         step()
@@ -293,8 +311,7 @@ def run_kta(args):
     clk = clocks.stop()
     kta.device_status()
     ms = max_over_ranks(e0.elapsed_time(e1))
-    tokens = ws * w.B * w.N * args.steps
-    value = tokens / (ms / 1e3)
+    value = whole_job_rate(ws, w.B * w.N, args.steps, ms)
 
     # ---- the same steps with per-kernel tracing (device time of every launch, on its stream)
     with kta.trace() as tr:
@@ -359,7 +376,7 @@ def run_kta(args):
         "gla_roofline": {"bound": "hbm", "achieved": gla_bytes(w) / t_gla / 1e9 if t_gla > 0 else None,
                          "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                          "frac": gla_bytes(w) / t_gla / 1e9 / float(peaks["hbm_gbs"]) if t_gla > 0 else None},
-        "e2e": {"value": ws * w.B * w.N * args.steps / (ms_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(ws, w.B * w.N, args.steps, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "clocks": clk,
