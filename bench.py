@@ -39,6 +39,12 @@ def parse_args():
     ap.add_argument("--impl", choices=("kta", "reference"), default="kta")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing leg (faster profiling runs)")
+    ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep"),
+                    default="hybrid",
+                    help="hybrid: the 21-frame hybrid layer (the headline line); delta: gated "
+                         "delta rule, 2 x 65,536 tokens x 16 heads; stream: 240-frame rollout one "
+                         "frame per call; sweep: hybrid layer vs full frame-causal attention for "
+                         "F = 8..256 frames of 1,024 tokens (one line per F)")
     return ap.parse_args()
 
 
@@ -62,6 +68,21 @@ def gla_bytes(w) -> float:
     return 12.0 * w.d * w.B * w.N * w.n_gla
 
 
+def delta_bytes(w) -> float:
+    """Algorithmic HBM bytes of the delta-rule heads: q, k, v, o bf16 + alpha, beta fp32."""
+    return (8.0 * w.d + 8.0) * w.B * w.N * w.n_gla
+
+
+def delta_flops(w) -> float:
+    """MMA FLOPs of the chunked delta rule: 10 C d + 6 d^2 per token-head."""
+    return (10.0 * w.chunk * w.d + 6.0 * w.d * w.d) * w.B * w.N * w.n_gla
+
+
+def full_causal_flops(w) -> float:
+    """Frame-causal attention over every earlier frame on all heads: 4 d per visible pair."""
+    return 4.0 * w.d * w.B * w.P * w.P * w.F * (w.F + 1) // 2 * w.H
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -75,7 +96,8 @@ KERNEL_SOURCES = {
     "win_attn_tc": ("win_attn_tc.cuh", "kta_ptx.cuh"),
     "gla_chunk_state": ("gla_chunk.cuh", "mma_sync.cuh"),
     "gla_chunk_out": ("gla_chunk.cuh", "mma_sync.cuh"),
-    "delta_chunk": ("delta_chunk.cuh", "mma_sync.cuh"),
+    "delta_prep": ("delta_chunk.cuh", "mma_sync.cuh"),
+    "delta_scan": ("delta_chunk.cuh", "mma_sync.cuh", "kta_ptx.cuh"),
 }
 
 
@@ -391,10 +413,143 @@ def run_kta(args):
     return 0
 
 
+# --------------------------------------------------------------------------- other workloads
+
+
+def _device_ms(fn, steps: int, warmup: int) -> float:
+    """Mean device milliseconds of fn() over `steps` calls after `warmup` calls (CUDA events on
+    the current stream, synchronised on both sides)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _traced(fn, steps: int) -> dict:
+    import torch
+
+    from hybrid_linear_temporal_kta_b200 import kta
+    with kta.trace() as tr:
+        for _ in range(steps):
+            fn()
+    torch.cuda.synchronize()
+    return {k: {"launches": v["launches"] // steps, "ms_per_step": v["ms"] / steps}
+            for k, v in tr.kernels.items()}
+
+
+def run_other(args):
+    """Timing of the workloads other than the headline hybrid layer (one GPU; one JSON line per
+    workload, or per F for the sweep). Inputs are drawn on the device with the same recipe; the
+    inputs of every workload are larger than the 126 MB L2, so no flush is needed."""
+    import torch
+
+    from hybrid_linear_temporal_kta_b200 import kta, synth
+
+    torch.cuda.set_device(0)
+    peaks, peaks_kind = load_peaks()
+    hbm, tc = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    lines = []
+    if args.workload == "delta":
+        w = synth.DELTA_BF16
+        x = synth.make_inputs_device(w, seed=w.seed_base)
+        o = torch.empty_like(x["q"])
+
+        def step():
+            kta.gla_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], chunk=w.chunk,
+                              out=o)
+        ms = _device_ms(step, args.steps, args.warmup)
+        kern = _traced(step, args.steps)
+        t_star = max(delta_bytes(w) / (hbm * 1e9), delta_flops(w) / (tc * 1e12))
+        lines.append({
+            "workload": w.name, "metric": "gated delta rule fwd tokens/s", "unit": "tokens/s",
+            "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
+            "config": {"B": w.B, "N": w.N, "H": w.n_gla, "d": w.d, "chunk": w.chunk},
+            "roofline": {"bound": "hbm", "algorithmic_bytes": delta_bytes(w),
+                         "algorithmic_flops": delta_flops(w),
+                         "achieved_gbs": delta_bytes(w) / (ms / 1e3) / 1e9, "peak_gbs": hbm,
+                         "t_star_ms": t_star * 1e3, "frac": t_star / (ms / 1e3),
+                         "peak_source": peaks_kind},
+            "kernels": kern})
+    elif args.workload == "stream":
+        w = synth.STREAM_BF16
+        x = synth.make_inputs_device(w, seed=w.seed_base)
+        cfg = kta.cfg_from_workload(w)
+        st = kta.Stream(cfg)
+        o = torch.empty_like(x["q"])
+        P = w.P
+        frames = [tuple(x[n][:, f * P:(f + 1) * P] for n in ("q", "k", "v", "alpha")) +
+                  (o[:, f * P:(f + 1) * P],) for f in range(w.F)]
+
+        def rollout():
+            st.reset()
+            for q, k, v, a, of in frames:
+                st.step(q, k, v, a, out=of)
+        ms = _device_ms(rollout, args.steps, args.warmup)
+        kern = _traced(rollout, args.steps)
+        flops = softmax_flops(w)
+        t_star = max(flops / (tc * 1e12), (8.0 * w.d * w.B * w.N * (w.n_swa + w.n_dswa) +
+                                          gla_bytes(w)) / (hbm * 1e9))
+        lines.append({
+            "workload": w.name, "metric": "streaming rollout tokens/s (one frame per call)",
+            "unit": "tokens/s", "value": w.B * w.N / (ms / 1e3), "ms_per_rollout": ms,
+            "us_per_frame": ms * 1e3 / w.F, "steps": args.steps,
+            "config": {"B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d,
+                       "state_bytes": st.state_bytes},
+            "roofline": {"bound": "tensor", "t_star_ms": t_star * 1e3, "frac": t_star / (ms / 1e3),
+                         "peak_source": peaks_kind},
+            "kernels": kern})
+        st.close()
+    else:  # sweep
+        for F in (8, 16, 32, 64, 128, 256):
+            w = synth.sweep_workload(F)
+            x = synth.make_inputs_device(w, seed=w.seed_base + F)
+            cfg = kta.cfg_from_workload(w)
+            o = torch.empty_like(x["q"])
+
+            def hyb():
+                kta.hybrid_fwd(cfg, x["q"], x["k"], x["v"], x["alpha"], out=o)
+
+            def full():
+                kta.swa_fwd(x["q"], x["k"], x["v"], P=w.P, W=w.F, out=o)
+            ms_h = _device_ms(hyb, args.steps, args.warmup)
+            steps_f = max(1, min(args.steps, 3 if F >= 128 else args.steps))
+            ms_f = _device_ms(full, steps_f, min(args.warmup, 1))
+            fl_h = softmax_flops(w)
+            t_star_h = max(fl_h / (tc * 1e12), (8.0 * w.d * w.B * w.N * (w.n_swa + w.n_dswa) +
+                                                gla_bytes(w)) / (hbm * 1e9))
+            fl_f = full_causal_flops(w)
+            lines.append({
+                "workload": w.name, "metric": "tokens/s, hybrid vs full frame-causal attention",
+                "unit": "tokens/s", "F": F, "N": w.N,
+                "hybrid": {"value": w.B * w.N / (ms_h / 1e3), "ms": ms_h,
+                           "softmax_tflops": fl_h / 1e12, "t_star_ms": t_star_h * 1e3,
+                           "frac": t_star_h / (ms_h / 1e3)},
+                "full_causal": {"value": w.B * w.N / (ms_f / 1e3), "ms": ms_f,
+                                "tflops": fl_f / 1e12,
+                                "achieved_tflops": fl_f / (ms_f / 1e3) / 1e12,
+                                "frac": fl_f / (ms_f / 1e3) / 1e12 / tc},
+                "speedup": ms_f / ms_h})
+            del x, o
+            torch.cuda.empty_cache()
+    kta.device_status()
+    for ln in lines:
+        print(json.dumps(ln), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != "hybrid":
+        return run_other(args)
     return run_kta(args)
 
 

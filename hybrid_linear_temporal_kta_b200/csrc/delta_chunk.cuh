@@ -1,5 +1,5 @@
 // delta_chunk.cuh -- chunked gated delta rule (bf16 in / out, fp32 state and gates) on
-// warp-level bf16 tensor-core tiles.
+// warp-level bf16 tensor-core tiles, TMA-fed.
 //
 // Operator: paper-read "Kairos: A Native World Model Stack for Physical AI", section 2, second
 // pillar, the four update lines (v_old = M k, v_new = beta v + (1-beta) v_old,
@@ -8,22 +8,31 @@
 // o_t = scale * q_t S_t.
 //
 // Chunked form (derived by unrolling inside a chunk of C tokens; gamma_t = prod_{r<=t} alpha_r,
-// gamma_{-1} = 1, S_0 the state at the chunk start):
-//   (I + T) U = diag(beta) V - diag(beta_t gamma_{t-1}) K S_0,
-//        T_ts = beta_t (gamma_{t-1} / gamma_s) (k_t . k_s)          for s < t
-//   o_t   = scale * [ gamma_t q_t S_0 + sum_{s<=t} (gamma_t / gamma_s) (q_t . k_s) u_s ]
-//   S_end = gamma_end S_0 + sum_s k_s^T (gamma_end / gamma_s) u_s
-// (I + T) is unit lower triangular. Its four 16 x 16 diagonal blocks are inverted in fp32 by
-// forward substitution; U follows by block forward substitution on the tensor cores:
-//   U_i = X_ii (R_i - sum_{j<i} T_ij U_j).
-// CTA = 4 warps over (sequence, head, value slice of BV = 32 columns); chunks in order, state in
-// registers. Warp w owns value columns [8w, 8w+8) in the substitution, query rows [16w, 16w+16)
-// of the output, and state rows [32w, 32w+32).
+// gamma_{-1} = 1, S_0 the state at the chunk start, A = (I + T)^{-1} with the strictly lower
+// triangular T_ts = beta_t (gamma_{t-1} / gamma_s) (k_t . k_s)):
+//   U     = U' - W S_0,      U' = A diag(beta) V,      W = A diag(beta_t gamma_{t-1}) K
+//   o_t   = scale * [ gamma_t q_t S_0 + sum_{s<=t} Aq_ts u_s ],  Aq_ts = (gamma_t/gamma_s)(q_t . k_s)
+//   S_end = gamma_end S_0 + sum_s (gamma_end / gamma_s) k_s^T u_s
+// Only the three products with S_0 depend on earlier chunks. Two kernels:
+//   delta_prep_kernel (one CTA per chunk, all chunks at once): cumulative log2 gates, T and Aq,
+//     the inverse of I + T (fp32 inverses of the 16 x 16 diagonal blocks, then block forward
+//     substitution on the tensor cores) applied to [diag(beta gamma_prev) K | diag(beta) V].
+//     Writes W [C][D], U'^T [D][C], Aq [C][C] (bf16) and the gates [C] (fp32) to a workspace.
+//   delta_scan_kernel (one CTA per (value block, sequence, head), chunks in order): a producer
+//     warp streams W, q, k, Aq, U'^T and the gates of the coming chunks into a ring of shared-
+//     memory stages with TMA (128-byte swizzle); each consumer warp owns 16 value columns and
+//     keeps its slice S^T (16 x D, fp32) in registers, so the chunk-to-chunk chain is register-
+//     resident with no block-wide barrier:
+//       U^T = U'^T - S^T W^T,   S^T <- gamma_end S^T + (U^T diag(gamma_end / gamma)) K,
+//       o^T = (S_0^T q^T) diag(gamma) + U^T Aq^T   (S_0^T kept as bf16 fragments).
 #pragma once
 
+#include "kta_ptx.cuh"
 #include "mma_sync.cuh"
 
 namespace kta {
+
+constexpr int DELTA_C = 64;
 
 struct DeltaParams {
   const __nv_bfloat16* q;
@@ -39,345 +48,514 @@ struct DeltaParams {
   float scale;
   const float* S0;        // [B][H][D][D] key-major, or null
   float* S_out;           // or null
+  int nch;                // chunks per sequence
+  __nv_bfloat16* ws_W;    // [B*H][nch][C][D]
+  __nv_bfloat16* ws_U;    // [B*H][nch][D][C]   (U'^T)
+  __nv_bfloat16* ws_A;    // [B*H][nch][C][C]
+  float* ws_g;            // [B*H][nch][C]      cumulative log2 gates
 };
 
+// ------------------------------------------------------------------------------ prep kernel
+
 template <int D>
-struct DeltaSmem {
-  static constexpr int C = 64;
-  static constexpr int BV = 32;
-  static constexpr int LDK = D + 8;
-  static constexpr int LDV = BV + 8;
+struct DeltaPrepSmem {
+  static constexpr int C = DELTA_C;
+  static constexpr int LDK = D + 8;   // padded rows: conflict-free ldmatrix
   static constexpr int LDC = C + 8;
-  __nv_bfloat16 q[C * LDK];
-  __nv_bfloat16 k[C * LDK];
-  __nv_bfloat16 v[C * LDV];
-  __nv_bfloat16 s[D * LDV];     // bf16 chunk-start state slice
-  __nv_bfloat16 u[C * LDV];     // U (and the block right-hand sides while solving)
-  __nv_bfloat16 ur[C * LDV];    // diag(gamma_end / gamma_s) U
-  __nv_bfloat16 tb[C * LDC];    // T in bf16 (off-diagonal blocks are used)
-  __nv_bfloat16 aq[C * LDC];    // (gamma_t / gamma_s) (q_t . k_s), s <= t
+  union {
+    __nv_bfloat16 q[C * LDK];   // raw q (until Q K^T is in registers)
+    float tf[C * (C + 1)];      // then T in fp32
+  };
+  __nv_bfloat16 k[C * LDK];     // raw k, then W (in place)
+  __nv_bfloat16 v[C * LDK];     // raw v, then U' (in place)
+  __nv_bfloat16 tn[C * LDC];    // -T in bf16
+  __nv_bfloat16 aq[C * LDC];    // Aq in bf16
   __nv_bfloat16 xd[4][16 * 24]; // inverses of the 16 x 16 diagonal blocks of I + T
-  float tf[C * (C + 1)];        // T in fp32 (diagonal blocks are inverted from it)
   float lg[C];                  // cumulative log2 alpha
   float beta[C];
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) delta_chunk_kernel(const DeltaParams p) {
-  using SM = DeltaSmem<D>;
-  constexpr int C = SM::C, BV = SM::BV, LDK = SM::LDK, LDV = SM::LDV, LDC = SM::LDC;
-  constexpr int LDT = C + 1;
-  constexpr int RW = D / 4, MT = RW / 16;
+__global__ void __launch_bounds__(128, 3) delta_prep_kernel(const DeltaParams p) {
+  using SM = DeltaPrepSmem<D>;
+  constexpr int C = SM::C, LDK = SM::LDK, LDC = SM::LDC, LDT = C + 1;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SM& sm = *reinterpret_cast<SM*>(smem_raw);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g4 = lane >> 2, t4 = lane & 3;
-  const int slice = blockIdx.x, bh = blockIdx.y;
+  const int cidx = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
-  const int j0 = slice * BV;
+  const int c0 = cidx * C;
+  const int n = min(C, p.N - c0);
   const long long row_b = static_cast<long long>(b) * p.rows_b;
 
-  // state rows [warp*RW, +RW) x BV columns: st[mt][nt][r]
-  float st[MT][BV / 8][4];
-  auto srow = [&](int mt, int r) { return warp * RW + mt * 16 + g4 + (r >= 2 ? 8 : 0); };
-  auto scol = [&](int nt, int r) { return nt * 8 + 2 * t4 + (r & 1); };
-  const long long sb = static_cast<long long>(bh) * D * D;
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < BV / 8; ++nt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-        st[mt][nt][r] = p.S0 ? p.S0[sb + srow(mt, r) * D + j0 + scol(nt, r)] : 0.f;
-
-  auto write_state_smem = [&]() {
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < BV / 8; ++nt) {
-        const int r0 = srow(mt, 0), c0 = scol(nt, 0);
-        *reinterpret_cast<uint32_t*>(&sm.s[r0 * LDV + c0]) = bf16x2(st[mt][nt][0], st[mt][nt][1]);
-        *reinterpret_cast<uint32_t*>(&sm.s[(r0 + 8) * LDV + c0]) = bf16x2(st[mt][nt][2], st[mt][nt][3]);
-      }
-  };
-  write_state_smem();
-
-  for (int c0 = 0; c0 < p.N; c0 += C) {
-    const int n = min(C, p.N - c0);
-    // ---- load q, k (full head dim), v slice; gates
-    {
-      constexpr int QCH = D / 8;
-      for (int idx = tid; idx < C * QCH; idx += 128) {
-        const int t = idx / QCH, c = (idx % QCH) * 8;
-        const long long grow = row_b + c0 + min(t, n - 1);
-        const long long off = grow * p.ld + static_cast<long long>(h) * D + c;
-        const int bytes = t < n ? 16 : 0;
-        cp_async16(&sm.q[t * LDK + c], p.q + off, bytes);
-        cp_async16(&sm.k[t * LDK + c], p.k + off, bytes);
-      }
-      constexpr int VCH = BV / 8;
-      for (int idx = tid; idx < C * VCH; idx += 128) {
-        const int t = idx / VCH, c = (idx % VCH) * 8;
-        const long long grow = row_b + c0 + min(t, n - 1);
-        cp_async16(&sm.v[t * LDV + c], p.v + grow * p.ld + static_cast<long long>(h) * D + j0 + c,
-                   t < n ? 16 : 0);
-      }
-      if (warp == 0) {
-        // cumulative log2 alpha over the chunk (two tokens per lane, warp scan); padding rows
-        // have alpha = 1 and beta = 0.
-        float a0 = 0.f, a1 = 0.f;
-        const int t0 = 2 * lane, t1 = 2 * lane + 1;
-        const long long r0 = (row_b + c0 + t0) * p.H + h, r1 = (row_b + c0 + t1) * p.H + h;
-        if (t0 < n) { a0 = __log2f(p.alpha[r0]); sm.beta[t0] = p.beta[r0]; } else sm.beta[t0] = 0.f;
-        if (t1 < n) { a1 = __log2f(p.alpha[r1]); sm.beta[t1] = p.beta[r1]; } else sm.beta[t1] = 0.f;
-        float pair = a0 + a1;
-        float incl = pair;
-#pragma unroll
-        for (int o2 = 1; o2 < 32; o2 <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, incl, o2);
-          if (lane >= o2) incl += y;
-        }
-        const float excl = incl - pair;
-        sm.lg[t0] = excl + a0;
-        sm.lg[t1] = excl + a0 + a1;
-      }
-      cp_async_wait_all();
+  // ---- q, k, v rows of the chunk (rows >= n zero-filled); gates
+  {
+    constexpr int QCH = D / 8;
+    for (int idx = tid; idx < C * QCH; idx += 128) {
+      const int t = idx / QCH, c = (idx % QCH) * 8;
+      const long long grow = row_b + c0 + min(t, n - 1);
+      const long long off = grow * p.ld + static_cast<long long>(h) * D + c;
+      const int bytes = t < n ? 16 : 0;
+      cp_async16(&sm.q[t * LDK + c], p.q + off, bytes);
+      cp_async16(&sm.k[t * LDK + c], p.k + off, bytes);
+      cp_async16(&sm.v[t * LDK + c], p.v + off, bytes);
     }
-    __syncthreads();
+    if (warp == 0) {
+      // cumulative log2 alpha over the chunk (two tokens per lane, warp scan); padding rows have
+      // alpha = 1 and beta = 0.
+      float a0 = 0.f, a1 = 0.f;
+      const int t0 = 2 * lane, t1 = 2 * lane + 1;
+      const long long r0 = (row_b + c0 + t0) * p.H + h, r1 = (row_b + c0 + t1) * p.H + h;
+      if (t0 < n) { a0 = __log2f(p.alpha[r0]); sm.beta[t0] = p.beta[r0]; } else sm.beta[t0] = 0.f;
+      if (t1 < n) { a1 = __log2f(p.alpha[r1]); sm.beta[t1] = p.beta[r1]; } else sm.beta[t1] = 0.f;
+      const float pair = a0 + a1;
+      float incl = pair;
+#pragma unroll
+      for (int o2 = 1; o2 < 32; o2 <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, o2);
+        if (lane >= o2) incl += y;
+      }
+      const float excl = incl - pair;
+      sm.lg[t0] = excl + a0;
+      sm.lg[t1] = excl + a0 + a1;
+    }
+    cp_async_wait_all();
+  }
+  __syncthreads();
 
-    // ---- K K^T and Q K^T for query rows [16w, 16w+16): T (s < t) and decayed QK (s <= t)
-    {
-      const int r0 = warp * 16;
-      uint32_t ak[D / 16][4], aqf[D / 16][4];
+  // ---- K K^T and Q K^T for rows [16w, 16w+16): T (s < t) and Aq (s <= t)
+  {
+    const int r0 = warp * 16;
+    uint32_t ak[D / 16][4], aqf[D / 16][4];
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      ldsm_x4(ak[kk], &sm.k[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
+      ldsm_x4(aqf[kk], &sm.q[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
+    }
+    float kk_acc[C / 8][4], qk_acc[C / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < C / 8; ++nt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) kk_acc[nt][r] = qk_acc[nt][r] = 0.f;
+#pragma unroll
+    for (int np = 0; np < C / 16; ++np) {
+      if (np > warp) break;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        ldsm_x4(ak[kk], &sm.k[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
-        ldsm_x4(aqf[kk], &sm.q[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
+        uint32_t bk[4];
+        ldsm_x4(bk, &sm.k[frag_b_nmajor(lane, np * 16, kk * 16, LDK)]);
+        mma16816(kk_acc[2 * np], ak[kk], bk[0], bk[1]);
+        mma16816(kk_acc[2 * np + 1], ak[kk], bk[2], bk[3]);
+        mma16816(qk_acc[2 * np], aqf[kk], bk[0], bk[1]);
+        mma16816(qk_acc[2 * np + 1], aqf[kk], bk[2], bk[3]);
       }
-      float kk_acc[C / 8][4], qk_acc[C / 8][4];
+    }
+    __syncthreads();  // every warp's q fragments are in registers: T may overwrite q
+#pragma unroll
+    for (int nt = 0; nt < C / 8; ++nt) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int t = r0 + g4 + (r >= 2 ? 8 : 0);
+        const int s = nt * 8 + 2 * t4 + (r & 1);
+        const float lgt = sm.lg[t], lgs = sm.lg[s];
+        const float lgp = t > 0 ? sm.lg[t - 1] : 0.f;
+        const float tv = s < t ? sm.beta[t] * exp2f(lgp - lgs) * kk_acc[nt][r] : 0.f;
+        const float av = s <= t ? exp2f(lgt - lgs) * qk_acc[nt][r] : 0.f;
+        sm.tf[t * LDT + s] = tv;
+        kk_acc[nt][r] = -tv;
+        qk_acc[nt][r] = av;
+      }
+      const int t = r0 + g4, s = nt * 8 + 2 * t4;
+      *reinterpret_cast<uint32_t*>(&sm.tn[t * LDC + s]) = bf16x2(kk_acc[nt][0], kk_acc[nt][1]);
+      *reinterpret_cast<uint32_t*>(&sm.tn[(t + 8) * LDC + s]) = bf16x2(kk_acc[nt][2], kk_acc[nt][3]);
+      *reinterpret_cast<uint32_t*>(&sm.aq[t * LDC + s]) = bf16x2(qk_acc[nt][0], qk_acc[nt][1]);
+      *reinterpret_cast<uint32_t*>(&sm.aq[(t + 8) * LDC + s]) = bf16x2(qk_acc[nt][2], qk_acc[nt][3]);
+    }
+  }
+  __syncthreads();
+
+  // ---- invert diagonal block `warp` of I + T (lane c < 16 owns column c), fp32
+  {
+    const int base = warp * 16;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) x[r] = (r == lane) ? 1.f : 0.f;
+#pragma unroll
+    for (int r = 1; r < 16; ++r) {
+      float acc = x[r];
+#pragma unroll
+      for (int s = 0; s < r; ++s) acc = fmaf(-sm.tf[(base + r) * LDT + base + s], x[s], acc);
+      x[r] = acc;
+    }
+    if (lane < 16) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) sm.xd[warp][r * 24 + lane] = __float2bfloat16_rn(x[r]);
+    }
+  }
+  __syncthreads();
+
+  // ---- block forward substitution: Z_i = X_ii (R_i - sum_{j<i} T_ij Z_j) on the right-hand
+  // sides R = [diag(beta_t gamma_{t-1}) K | diag(beta) V]; warp w owns D/2 of the 2D columns
+  // (warps 0, 1: the K side -> W; warps 2, 3: the V side -> U'), in place over k / v.
+  {
+    constexpr int CW = D / 2, NTW = CW / 8;
+    const bool kside = warp < 2;
+    const int col0 = (warp & 1) * CW;
+    __nv_bfloat16* buf = kside ? sm.k : sm.v;
+#pragma unroll 1
+    for (int i = 0; i < C / 16; ++i) {
+      const int ta = i * 16 + g4, tb = ta + 8;
+      const float fa = kside ? sm.beta[ta] * (ta > 0 ? exp2f(sm.lg[ta - 1]) : 1.f) : sm.beta[ta];
+      const float fb = kside ? sm.beta[tb] * exp2f(sm.lg[tb - 1]) : sm.beta[tb];
+      float acc[NTW][4];
+#pragma unroll
+      for (int nt = 0; nt < NTW; ++nt) {
+        const int col = col0 + nt * 8 + 2 * t4;
+        const float2 ra = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&buf[ta * LDK + col]));
+        const float2 rb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&buf[tb * LDK + col]));
+        acc[nt][0] = fa * ra.x;
+        acc[nt][1] = fa * ra.y;
+        acc[nt][2] = fb * rb.x;
+        acc[nt][3] = fb * rb.y;
+      }
+      for (int j = 0; j < i; ++j) {
+        uint32_t a[4];
+        ldsm_x4(a, &sm.tn[frag_a_rowmajor(lane, i * 16, j * 16, LDC)]);
+#pragma unroll
+        for (int np = 0; np < NTW / 2; ++np) {
+          uint32_t bz[4];
+          ldsm_x4_t(bz, &buf[frag_b_kmajor(lane, j * 16, col0 + np * 16, LDK)]);
+          mma16816(acc[2 * np], a, bz[0], bz[1]);
+          mma16816(acc[2 * np + 1], a, bz[2], bz[3]);
+        }
+      }
+      // stage Y_i (bf16) over rows of block i (each lane rewrites the elements it read)
+#pragma unroll
+      for (int nt = 0; nt < NTW; ++nt) {
+        const int col = col0 + nt * 8 + 2 * t4;
+        *reinterpret_cast<uint32_t*>(&buf[ta * LDK + col]) = bf16x2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t*>(&buf[tb * LDK + col]) = bf16x2(acc[nt][2], acc[nt][3]);
+      }
+      __syncwarp();
+      uint32_t ax[4];
+      ldsm_x4(ax, &sm.xd[i][frag_a_rowmajor(lane, 0, 0, 24)]);
+      float z[NTW][4];
+#pragma unroll
+      for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) z[nt][r] = 0.f;
+#pragma unroll
+      for (int np = 0; np < NTW / 2; ++np) {
+        uint32_t by[4];
+        ldsm_x4_t(by, &buf[frag_b_kmajor(lane, i * 16, col0 + np * 16, LDK)]);
+        mma16816(z[2 * np], ax, by[0], by[1]);
+        mma16816(z[2 * np + 1], ax, by[2], by[3]);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int nt = 0; nt < NTW; ++nt) {
+        const int col = col0 + nt * 8 + 2 * t4;
+        *reinterpret_cast<uint32_t*>(&buf[ta * LDK + col]) = bf16x2(z[nt][0], z[nt][1]);
+        *reinterpret_cast<uint32_t*>(&buf[tb * LDK + col]) = bf16x2(z[nt][2], z[nt][3]);
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+
+  // ---- workspace: W, U'^T, Aq, gates
+  {
+    const long long wsi = static_cast<long long>(bh) * p.nch + cidx;
+    __nv_bfloat16* W = p.ws_W + wsi * C * D;
+    constexpr int QCH = D / 8;
+    for (int idx = tid; idx < C * QCH; idx += 128) {
+      const int t = idx / QCH, c = (idx % QCH) * 8;
+      *reinterpret_cast<uint4*>(&W[t * D + c]) = *reinterpret_cast<const uint4*>(&sm.k[t * LDK + c]);
+    }
+    __nv_bfloat16* A = p.ws_A + wsi * C * C;
+    for (int idx = tid; idx < C * (C / 8); idx += 128) {
+      const int t = idx / (C / 8), c = (idx % (C / 8)) * 8;
+      *reinterpret_cast<uint4*>(&A[t * C + c]) = *reinterpret_cast<const uint4*>(&sm.aq[t * LDC + c]);
+    }
+    __nv_bfloat16* U = p.ws_U + wsi * D * C;
+    for (int idx = tid; idx < D * (C / 2); idx += 128) {
+      const int j = idx / (C / 2), t = (idx % (C / 2)) * 2;
+      __nv_bfloat162 pr;
+      pr.x = sm.v[t * LDK + j];
+      pr.y = sm.v[(t + 1) * LDK + j];
+      *reinterpret_cast<__nv_bfloat162*>(&U[j * C + t]) = pr;
+    }
+    if (tid < C) p.ws_g[wsi * C + tid] = sm.lg[tid];
+  }
+}
+
+// ------------------------------------------------------------------------------ scan kernel
+
+// Byte offset of element (row, col) in a tile of ROWS rows x (64 * boxes) bf16 columns stored as
+// boxes of [ROWS][64] with the TMA 128-byte swizzle (16-byte group index XOR row % 8).
+template <int ROWS>
+__device__ __forceinline__ uint32_t swz(int row, int col) {
+  return static_cast<uint32_t>((col >> 6) * (ROWS * 128) + row * 128 +
+                               ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
+}
+
+template <int D, int WARPS, int NST>
+struct DeltaScanSmem {
+  static constexpr int C = DELTA_C;
+  static constexpr int VB = 16 * WARPS;   // value columns per CTA
+  static constexpr int NBOX = D / 64;
+  static constexpr int LDO = VB + 8;
+  struct alignas(1024) Stage {
+    __nv_bfloat16 w[NBOX * C * 64];
+    __nv_bfloat16 q[NBOX * C * 64];
+    __nv_bfloat16 k[NBOX * C * 64];
+    __nv_bfloat16 aq[C * 64];
+    __nv_bfloat16 ut[VB * 64];
+    float lg[C];
+  };
+  static constexpr uint32_t STAGE_TX =
+      (3 * NBOX * C * 64 + C * 64 + VB * 64) * 2 + C * 4;  // bytes the TMA unit writes per stage
+  Stage stage[NST];
+  __nv_bfloat16 o[2][C * LDO];
+  uint64_t full[NST];
+  uint64_t empty[NST];
+  int abort_flag;
+};
+
+template <int D, int WARPS, int NST>
+constexpr size_t delta_scan_smem_bytes() {
+  return sizeof(DeltaScanSmem<D, WARPS, NST>) + 1024;  // + manual 1024-byte alignment
+}
+
+template <int D, int WARPS, int NST>
+__global__ void __launch_bounds__((WARPS + 1) * 32, 1)
+    delta_scan_kernel(const __grid_constant__ CUtensorMap tW, const __grid_constant__ CUtensorMap tQ,
+                      const __grid_constant__ CUtensorMap tK, const __grid_constant__ CUtensorMap tA,
+                      const __grid_constant__ CUtensorMap tU, const DeltaParams p) {
+  using SM = DeltaScanSmem<D, WARPS, NST>;
+  constexpr int C = SM::C, VB = SM::VB, NBOX = SM::NBOX, LDO = SM::LDO;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SM& sm = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g4 = lane >> 2, t4 = lane & 3;
+  const int j0 = blockIdx.x * VB, bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const long long row_b = static_cast<long long>(b) * p.rows_b;
+
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], WARPS);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == WARPS) {
+    // ---- producer: one lane streams the stages
+    if (lane == 0) {
+      prefetch_tmap(&tW);
+      prefetch_tmap(&tQ);
+      prefetch_tmap(&tK);
+      prefetch_tmap(&tA);
+      prefetch_tmap(&tU);
+      for (int c = 0; c < p.nch; ++c) {
+        const int s = c % NST;
+        if (c >= NST && !mbar_wait(&sm.empty[s], ((c / NST) - 1) & 1)) break;
+        typename SM::Stage& S = sm.stage[s];
+        uint64_t* bar = &sm.full[s];
+        mbar_arrive_expect_tx(bar, SM::STAGE_TX);
+        const long long wsi = static_cast<long long>(bh) * p.nch + c;
+        const int wrow = static_cast<int>(wsi * C);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx) {
+          tma_load_2d(S.w + bx * C * 64, &tW, bar, bx * 64, wrow);
+          tma_load_4d(S.q + bx * C * 64, &tQ, bar, bx * 64, h, c * C, b);
+          tma_load_4d(S.k + bx * C * 64, &tK, bar, bx * 64, h, c * C, b);
+        }
+        tma_load_2d(S.aq, &tA, bar, 0, wrow);
+        tma_load_2d(S.ut, &tU, bar, 0, static_cast<int>(wsi * D + j0));
+        bulk_load(S.lg, p.ws_g + wsi * C, C * 4, bar);
+      }
+    }
+    return;
+  }
+
+  // ---- consumers: warp w owns value columns jv = j0 + 16w + g4 and jv + 8
+  const int jv = j0 + 16 * warp + g4;
+  const long long sb = static_cast<long long>(bh) * D * D;
+  // st[nt][r] = S^T[jv (+8 for r >= 2)][8 nt + 2 t4 + (r & 1)] = S[8 nt + 2 t4 + (r & 1)][jv (+8)]
+  float st[D / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      st[nt][r] = p.S0 ? p.S0[sb + (nt * 8 + 2 * t4 + (r & 1)) * D + jv + (r >= 2 ? 8 : 0)] : 0.f;
+
+  bool aborted = false;
+  for (int c = 0; c < p.nch; ++c) {
+    const int s = c % NST;
+    const bool ok = mbar_wait(&sm.full[s], (c / NST) & 1);
+    if (!ok) sm.abort_flag = 1;
+    __nv_bfloat16* ob = sm.o[c & 1];
+    if (ok) {
+      const typename SM::Stage& S = sm.stage[s];
+      const uint8_t* Wb = reinterpret_cast<const uint8_t*>(S.w);
+      const uint8_t* Qb = reinterpret_cast<const uint8_t*>(S.q);
+      const uint8_t* Kb = reinterpret_cast<const uint8_t*>(S.k);
+      const uint8_t* Ab = reinterpret_cast<const uint8_t*>(S.aq);
+      const uint8_t* Ub = reinterpret_cast<const uint8_t*>(S.ut);
+      // lane row / column offsets of the ldmatrix address patterns
+      const int nm_r = (lane & 7) + (lane >> 4) * 8, nm_c = ((lane >> 3) & 1) * 8;  // B stored [n][k]
+      const int km_r = (lane & 7) + ((lane >> 3) & 1) * 8, km_c = (lane >> 4) * 8;  // B stored [k][n]
+
+      // (a) S^T as bf16 A fragments (k = key dim)
+      uint32_t sa[D / 16][4];
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        sa[kk][0] = bf16x2(st[2 * kk][0], st[2 * kk][1]);
+        sa[kk][1] = bf16x2(st[2 * kk][2], st[2 * kk][3]);
+        sa[kk][2] = bf16x2(st[2 * kk + 1][0], st[2 * kk + 1][1]);
+        sa[kk][3] = bf16x2(st[2 * kk + 1][2], st[2 * kk + 1][3]);
+      }
+      // (b) X = S^T W^T  (n = token)
+      float xw[C / 8][4];
 #pragma unroll
       for (int nt = 0; nt < C / 8; ++nt)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) kk_acc[nt][r] = qk_acc[nt][r] = 0.f;
-#pragma unroll
-      for (int np = 0; np < C / 16; ++np) {
-        if (np > warp) break;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          uint32_t bk[4];
-          ldsm_x4(bk, &sm.k[frag_b_nmajor(lane, np * 16, kk * 16, LDK)]);
-          mma16816(kk_acc[2 * np], ak[kk], bk[0], bk[1]);
-          mma16816(kk_acc[2 * np + 1], ak[kk], bk[2], bk[3]);
-          mma16816(qk_acc[2 * np], aqf[kk], bk[0], bk[1]);
-          mma16816(qk_acc[2 * np + 1], aqf[kk], bk[2], bk[3]);
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < C / 8; ++nt) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int t = r0 + g4 + (r >= 2 ? 8 : 0);
-          const int s = nt * 8 + 2 * t4 + (r & 1);
-          const float lgt = sm.lg[t], lgs = sm.lg[s];
-          const float lgp = t > 0 ? sm.lg[t - 1] : 0.f;
-          const float tv = s < t ? sm.beta[t] * exp2f(lgp - lgs) * kk_acc[nt][r] : 0.f;
-          const float av = s <= t ? exp2f(lgt - lgs) * qk_acc[nt][r] : 0.f;
-          sm.tf[t * LDT + s] = tv;
-          kk_acc[nt][r] = tv;
-          qk_acc[nt][r] = av;
-        }
-        const int t = r0 + g4, s = nt * 8 + 2 * t4;
-        *reinterpret_cast<uint32_t*>(&sm.tb[t * LDC + s]) = bf16x2(kk_acc[nt][0], kk_acc[nt][1]);
-        *reinterpret_cast<uint32_t*>(&sm.tb[(t + 8) * LDC + s]) = bf16x2(kk_acc[nt][2], kk_acc[nt][3]);
-        *reinterpret_cast<uint32_t*>(&sm.aq[t * LDC + s]) = bf16x2(qk_acc[nt][0], qk_acc[nt][1]);
-        *reinterpret_cast<uint32_t*>(&sm.aq[(t + 8) * LDC + s]) = bf16x2(qk_acc[nt][2], qk_acc[nt][3]);
-      }
-    }
-    __syncthreads();
-
-    // ---- invert diagonal block `warp` of I + T (lane c < 16 owns column c), fp32
-    {
-      const int base = warp * 16;
-      float x[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) x[r] = (r == lane) ? 1.f : 0.f;
-#pragma unroll
-      for (int r = 1; r < 16; ++r) {
-        float acc = x[r];
-#pragma unroll
-        for (int s = 0; s < r; ++s) acc = fmaf(-sm.tf[(base + r) * LDT + base + s], x[s], acc);
-        x[r] = acc;
-      }
-      if (lane < 16) {
-#pragma unroll
-        for (int r = 0; r < 16; ++r) sm.xd[warp][r * 24 + lane] = __float2bfloat16_rn(x[r]);
-      }
-    }
-
-    // ---- R = diag(beta) V - diag(beta_t gamma_{t-1}) K S_0 for value columns [8w, 8w+8)
-    float racc[C / 16][4];
-    {
-#pragma unroll
-      for (int mt = 0; mt < C / 16; ++mt)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) racc[mt][r] = 0.f;
+        for (int r = 0; r < 4; ++r) xw[nt][r] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        // B = S_0 rows [16kk, 16kk+16) x this warp's 8 value columns
-        uint32_t bs[2];
-        ldsm_x2_t(bs, &sm.s[frag_b_kmajor(lane, kk * 16, warp * 8, LDV)]);
 #pragma unroll
-        for (int mt = 0; mt < C / 16; ++mt) {
-          uint32_t a[4];
-          ldsm_x4(a, &sm.k[frag_a_rowmajor(lane, mt * 16, kk * 16, LDK)]);
-          mma16816(racc[mt], a, bs[0], bs[1]);
+        for (int np = 0; np < C / 16; ++np) {
+          uint32_t bw[4];
+          ldsm_x4(bw, Wb + swz<C>(np * 16 + nm_r, kk * 16 + nm_c));
+          mma16816(xw[2 * np], sa[kk], bw[0], bw[1]);
+          mma16816(xw[2 * np + 1], sa[kk], bw[2], bw[3]);
         }
       }
+      // (c) U^T = U'^T - X  (value rows 16w + g4 (+8), token columns)
 #pragma unroll
-      for (int mt = 0; mt < C / 16; ++mt)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int t = mt * 16 + g4 + (r >= 2 ? 8 : 0);
-          const int col = warp * 8 + 2 * t4 + (r & 1);
-          const float gp = t > 0 ? exp2f(sm.lg[t - 1]) : 1.f;
-          const float bt = sm.beta[t];
-          racc[mt][r] = bt * __bfloat162float(sm.v[t * LDV + col]) - bt * gp * racc[mt][r];
-        }
-    }
-    __syncthreads();  // diagonal inverses visible to every warp
-
-    // ---- block forward substitution for this warp's 8 value columns
-#pragma unroll
-    for (int i = 0; i < C / 16; ++i) {
-      float y[4] = {racc[i][0], racc[i][1], racc[i][2], racc[i][3]};
-#pragma unroll
-      for (int j = 0; j < C / 16; ++j) {
-        if (j >= i) break;
-        uint32_t a[4], bu[2];
-        ldsm_x4(a, &sm.tb[frag_a_rowmajor(lane, i * 16, j * 16, LDC)]);
-        ldsm_x2_t(bu, &sm.u[frag_b_kmajor(lane, j * 16, warp * 8, LDV)]);
-        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-        mma16816(tmp, a, bu[0], bu[1]);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) y[r] -= tmp[r];
+      for (int nt = 0; nt < C / 8; ++nt) {
+        const int tc = nt * 8 + 2 * t4;
+        const float2 ua = __bfloat1622float2(
+            *reinterpret_cast<const __nv_bfloat162*>(Ub + swz<VB>(16 * warp + g4, tc)));
+        const float2 ub = __bfloat1622float2(
+            *reinterpret_cast<const __nv_bfloat162*>(Ub + swz<VB>(16 * warp + g4 + 8, tc)));
+        xw[nt][0] = ua.x - xw[nt][0];
+        xw[nt][1] = ua.y - xw[nt][1];
+        xw[nt][2] = ub.x - xw[nt][2];
+        xw[nt][3] = ub.y - xw[nt][3];
       }
-      // stage Y_i (bf16) in the U rows of block i, then U_i = X_ii Y_i
-      const int t = i * 16 + g4, col = warp * 8 + 2 * t4;
-      *reinterpret_cast<uint32_t*>(&sm.u[t * LDV + col]) = bf16x2(y[0], y[1]);
-      *reinterpret_cast<uint32_t*>(&sm.u[(t + 8) * LDV + col]) = bf16x2(y[2], y[3]);
-      __syncwarp();
-      uint32_t a[4], by[2];
-      ldsm_x4(a, &sm.xd[i][frag_a_rowmajor(lane, 0, 0, 24)]);
-      ldsm_x2_t(by, &sm.u[frag_b_kmajor(lane, i * 16, warp * 8, LDV)]);
-      float uo[4] = {0.f, 0.f, 0.f, 0.f};
-      mma16816(uo, a, by[0], by[1]);
-      __syncwarp();
-      *reinterpret_cast<uint32_t*>(&sm.u[t * LDV + col]) = bf16x2(uo[0], uo[1]);
-      *reinterpret_cast<uint32_t*>(&sm.u[(t + 8) * LDV + col]) = bf16x2(uo[2], uo[3]);
-      __syncwarp();
-    }
-    __syncthreads();  // U complete
-
-    // ---- scaled U for the state update: ur_s = (gamma_end / gamma_s) u_s
-    for (int idx = tid; idx < C * BV; idx += 128) {
-      const int t = idx / BV, c = idx % BV;
-      const float r = exp2f(sm.lg[C - 1] - sm.lg[t]);
-      sm.ur[t * LDV + c] = __float2bfloat16_rn(r * __bfloat162float(sm.u[t * LDV + c]));
-    }
-
-    // ---- outputs for rows [16w, 16w+16): gamma_t q_t S_0 + Aq U
-    {
-      const int r0 = warp * 16;
-      float ov[BV / 8][4];
+      // (d) U^T as A fragments (k = token): plain, and scaled by gamma_end / gamma_s
+      const float lgC = S.lg[C - 1];
+      uint32_t ua[C / 16][4], ur[C / 16][4];
 #pragma unroll
-      for (int nt = 0; nt < BV / 8; ++nt)
+      for (int kk = 0; kk < C / 16; ++kk) {
+        const int ta = 16 * kk + 2 * t4, tb = ta + 8;
+        const float da0 = exp2f(lgC - S.lg[ta]), da1 = exp2f(lgC - S.lg[ta + 1]);
+        const float db0 = exp2f(lgC - S.lg[tb]), db1 = exp2f(lgC - S.lg[tb + 1]);
+        ua[kk][0] = bf16x2(xw[2 * kk][0], xw[2 * kk][1]);
+        ua[kk][1] = bf16x2(xw[2 * kk][2], xw[2 * kk][3]);
+        ua[kk][2] = bf16x2(xw[2 * kk + 1][0], xw[2 * kk + 1][1]);
+        ua[kk][3] = bf16x2(xw[2 * kk + 1][2], xw[2 * kk + 1][3]);
+        ur[kk][0] = bf16x2(xw[2 * kk][0] * da0, xw[2 * kk][1] * da1);
+        ur[kk][1] = bf16x2(xw[2 * kk][2] * da0, xw[2 * kk][3] * da1);
+        ur[kk][2] = bf16x2(xw[2 * kk + 1][0] * db0, xw[2 * kk + 1][1] * db1);
+        ur[kk][3] = bf16x2(xw[2 * kk + 1][2] * db0, xw[2 * kk + 1][3] * db1);
+      }
+      // (e) S^T = gamma_end S^T + Ur^T K  (n = key dim)
+      const float gC = exp2f(lgC);
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) st[nt][r] *= gC;
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+#pragma unroll
+        for (int np = 0; np < D / 16; ++np) {
+          uint32_t bk[4];
+          ldsm_x4_t(bk, Kb + swz<C>(kk * 16 + km_r, np * 16 + km_c));
+          mma16816(st[2 * np], ur[kk], bk[0], bk[1]);
+          mma16816(st[2 * np + 1], ur[kk], bk[2], bk[3]);
+        }
+      }
+      // (f) O = (S_0^T q^T) diag(gamma) + U^T Aq^T  (n = token; Aq is zero above its diagonal)
+      float ov[C / 8][4];
+#pragma unroll
+      for (int nt = 0; nt < C / 8; ++nt)
 #pragma unroll
         for (int r = 0; r < 4; ++r) ov[nt][r] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t a[4];
-        ldsm_x4(a, &sm.q[frag_a_rowmajor(lane, r0, kk * 16, LDK)]);
 #pragma unroll
-        for (int np = 0; np < BV / 16; ++np) {
-          uint32_t bs[4];
-          ldsm_x4_t(bs, &sm.s[frag_b_kmajor(lane, kk * 16, np * 16, LDV)]);
-          mma16816(ov[2 * np], a, bs[0], bs[1]);
-          mma16816(ov[2 * np + 1], a, bs[2], bs[3]);
-        }
-      }
-      const float ga = exp2f(sm.lg[r0 + g4]), gb = exp2f(sm.lg[r0 + g4 + 8]);
-#pragma unroll
-      for (int nt = 0; nt < BV / 8; ++nt) {
-        ov[nt][0] *= ga;
-        ov[nt][1] *= ga;
-        ov[nt][2] *= gb;
-        ov[nt][3] *= gb;
-      }
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk) {
-        if (kk > warp) break;
-        uint32_t a[4];
-        ldsm_x4(a, &sm.aq[frag_a_rowmajor(lane, r0, kk * 16, LDC)]);
-#pragma unroll
-        for (int np = 0; np < BV / 16; ++np) {
-          uint32_t bu[4];
-          ldsm_x4_t(bu, &sm.u[frag_b_kmajor(lane, kk * 16, np * 16, LDV)]);
-          mma16816(ov[2 * np], a, bu[0], bu[1]);
-          mma16816(ov[2 * np + 1], a, bu[2], bu[3]);
+        for (int np = 0; np < C / 16; ++np) {
+          uint32_t bq[4];
+          ldsm_x4(bq, Qb + swz<C>(np * 16 + nm_r, kk * 16 + nm_c));
+          mma16816(ov[2 * np], sa[kk], bq[0], bq[1]);
+          mma16816(ov[2 * np + 1], sa[kk], bq[2], bq[3]);
         }
       }
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int t = r0 + g4 + hr * 8;
-        if (t < n) {
-          __nv_bfloat16* orow = p.o + (row_b + c0 + t) * p.ld + static_cast<long long>(h) * D + j0;
+      for (int nt = 0; nt < C / 8; ++nt) {
+        const int tc = nt * 8 + 2 * t4;
+        const float g0 = exp2f(S.lg[tc]), g1 = exp2f(S.lg[tc + 1]);
+        ov[nt][0] *= g0;
+        ov[nt][1] *= g1;
+        ov[nt][2] *= g0;
+        ov[nt][3] *= g1;
+      }
 #pragma unroll
-          for (int nt = 0; nt < BV / 8; ++nt)
-            *reinterpret_cast<uint32_t*>(orow + nt * 8 + 2 * t4) =
-                bf16x2(ov[nt][2 * hr] * p.scale, ov[nt][2 * hr + 1] * p.scale);
+      for (int np = 0; np < C / 16; ++np) {
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          if (kk > np) break;
+          uint32_t ba[4];
+          ldsm_x4(ba, Ab + swz<C>(np * 16 + nm_r, kk * 16 + nm_c));
+          mma16816(ov[2 * np], ua[kk], ba[0], ba[1]);
+          mma16816(ov[2 * np + 1], ua[kk], ba[2], ba[3]);
         }
+      }
+      // every read of the stage is done: hand it back to the producer
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+      // (g) stage O (bf16, [token][value column]) for coalesced stores
+      const int vr = 16 * warp + g4;
+#pragma unroll
+      for (int nt = 0; nt < C / 8; ++nt) {
+        const int tc = nt * 8 + 2 * t4;
+        ob[tc * LDO + vr] = __float2bfloat16_rn(ov[nt][0] * p.scale);
+        ob[(tc + 1) * LDO + vr] = __float2bfloat16_rn(ov[nt][1] * p.scale);
+        ob[tc * LDO + vr + 8] = __float2bfloat16_rn(ov[nt][2] * p.scale);
+        ob[(tc + 1) * LDO + vr + 8] = __float2bfloat16_rn(ov[nt][3] * p.scale);
       }
     }
-    __syncthreads();  // ur complete; every read of s done
-
-    // ---- state: S = gamma_end S + K^T Ur
+    named_bar_sync(1, WARPS * 32);
+    if (sm.abort_flag) {
+      aborted = true;
+      break;
+    }
     {
-      const float gend = exp2f(sm.lg[C - 1]);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < BV / 8; ++nt)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) st[mt][nt][r] *= gend;
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk) {
-        uint32_t bu[BV / 16][4];
-#pragma unroll
-        for (int np = 0; np < BV / 16; ++np) ldsm_x4_t(bu[np], &sm.ur[frag_b_kmajor(lane, kk * 16, np * 16, LDV)]);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          uint32_t a[4];
-          ldsm_x4_t(a, &sm.k[frag_a_kmajor(lane, warp * RW + mt * 16, kk * 16, LDK)]);
-#pragma unroll
-          for (int np = 0; np < BV / 16; ++np) {
-            mma16816(st[mt][2 * np], a, bu[np][0], bu[np][1]);
-            mma16816(st[mt][2 * np + 1], a, bu[np][2], bu[np][3]);
-          }
-        }
+      const int n = min(C, p.N - c * C);
+      constexpr int PCS = VB / 8;
+      for (int idx = tid; idx < n * PCS; idx += WARPS * 32) {
+        const int t = idx / PCS, pc = (idx % PCS) * 8;
+        *reinterpret_cast<uint4*>(p.o + (row_b + static_cast<long long>(c) * C + t) * p.ld +
+                                  static_cast<long long>(h) * D + j0 + pc) =
+            *reinterpret_cast<const uint4*>(&ob[t * LDO + pc]);
       }
     }
-    __syncthreads();
-    write_state_smem();
   }
-  if (p.S_out) {
-    float* So = p.S_out + sb;
+  if (p.S_out && !aborted) {
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int nt = 0; nt < D / 8; ++nt)
 #pragma unroll
-      for (int nt = 0; nt < BV / 8; ++nt)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) So[srow(mt, r) * D + j0 + scol(nt, r)] = st[mt][nt][r];
+      for (int r = 0; r < 4; ++r)
+        p.S_out[sb + (nt * 8 + 2 * t4 + (r & 1)) * D + jv + (r >= 2 ? 8 : 0)] = st[nt][r];
   }
 }
 

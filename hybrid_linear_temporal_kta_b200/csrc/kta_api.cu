@@ -89,6 +89,19 @@ kta_status make_map(CUtensorMap* m, const void* base, int d, int heads, long lon
   return KTA_OK;
 }
 
+// Tiled bf16 map of rank r (dims innermost first, byte strides of dims 1..r-1), 128-byte swizzle.
+kta_status make_map_nd(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return KTA_OK;
+}
+
 // ------------------------------------------------------------------------- per-device state
 
 struct DeviceRes {
@@ -402,7 +415,14 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
 
 template <int D>
 kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
-  using SM = kta::DeltaSmem<D>;
+  constexpr int C = kta::DELTA_C, WARPS = 2, NST = 3;
+  using PS = kta::DeltaPrepSmem<D>;
+  using SS = kta::DeltaScanSmem<D, WARPS, NST>;
+  const long long BH = static_cast<long long>(L.B) * L.H;
+  if (BH > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
+  const long long nch = (L.N + C - 1) / C;
+  // workspace rows are addressed with 32-bit TMA coordinates
+  if (BH * nch * D >= (1LL << 31)) return fail(KTA_ERR_UNSUPPORTED, "B*H*N too large for the delta workspace");
   kta::DeltaParams p{};
   p.q = static_cast<const __nv_bfloat16*>(L.q);
   p.k = static_cast<const __nv_bfloat16*>(L.k);
@@ -417,14 +437,52 @@ kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
   p.scale = L.scale;
   p.S0 = L.S0;
   p.S_out = L.S_out;
-  const size_t smem = sizeof(SM);
-  kta_status sa;
-  if ((sa = set_smem_attr(kta::delta_chunk_kernel<D>, smem))) return sa;
-  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
-  dim3 grid(D / SM::BV, L.B * L.H);
+  p.nch = static_cast<int>(nch);
+  const size_t units = static_cast<size_t>(BH) * nch;
+  const size_t bytes = units * (static_cast<size_t>(C) * D * 2 * 2 + C * C * 2 + C * 4);
+  void* ws = nullptr;
+  kta_status s = workspace(bytes, &ws);
+  if (s) return s;
+  p.ws_W = static_cast<__nv_bfloat16*>(ws);
+  p.ws_U = p.ws_W + units * C * D;
+  p.ws_A = p.ws_U + units * D * C;
+  p.ws_g = reinterpret_cast<float*>(p.ws_A + units * C * C);
+
+  CUtensorMap tW, tQ, tK, tA, tU;
   {
-    TraceScope ts("delta_chunk", st);
-    kta::delta_chunk_kernel<D><<<grid, 128, smem, st>>>(p);
+    const cuuint64_t dW[2] = {static_cast<cuuint64_t>(D), units * C};
+    const cuuint64_t sW[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t bW[2] = {64, static_cast<cuuint32_t>(C)};
+    if ((s = make_map_nd(&tW, p.ws_W, 2, dW, sW, bW))) return s;
+    const cuuint64_t dA[2] = {static_cast<cuuint64_t>(C), units * C};
+    const cuuint64_t sA[1] = {static_cast<cuuint64_t>(C) * 2};
+    if ((s = make_map_nd(&tA, p.ws_A, 2, dA, sA, bW))) return s;
+    const cuuint64_t dU[2] = {static_cast<cuuint64_t>(C), units * D};
+    const cuuint32_t bU[2] = {64, static_cast<cuuint32_t>(SS::VB)};
+    if ((s = make_map_nd(&tU, p.ws_U, 2, dU, sA, bU))) return s;
+    // q, k: (key dim, head, row, sequence); rows past N read as zeros
+    const cuuint64_t dQ[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L.H),
+                              static_cast<cuuint64_t>(L.N), static_cast<cuuint64_t>(L.B)};
+    const cuuint64_t sQ[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L.ld) * 2,
+                              static_cast<cuuint64_t>(L.rows_b) * L.ld * 2};
+    const cuuint32_t bQ[4] = {64, 1, static_cast<cuuint32_t>(C), 1};
+    if ((s = make_map_nd(&tQ, L.q, 4, dQ, sQ, bQ))) return s;
+    if ((s = make_map_nd(&tK, L.k, 4, dQ, sQ, bQ))) return s;
+  }
+  const size_t smem_p = sizeof(PS), smem_s = kta::delta_scan_smem_bytes<D, WARPS, NST>();
+  if ((s = set_smem_attr(kta::delta_prep_kernel<D>, smem_p))) return s;
+  if ((s = set_smem_attr(kta::delta_scan_kernel<D, WARPS, NST>, smem_s))) return s;
+  {
+    TraceScope ts("delta_prep", st);
+    kta::delta_prep_kernel<D><<<dim3(static_cast<unsigned>(nch), static_cast<unsigned>(BH)), 128,
+                                smem_p, st>>>(p);
+  }
+  KTA_CUDA(cudaGetLastError());
+  {
+    TraceScope ts("delta_scan", st);
+    kta::delta_scan_kernel<D, WARPS, NST>
+        <<<dim3(D / SS::VB, static_cast<unsigned>(BH)), (WARPS + 1) * 32, smem_s, st>>>(
+            tW, tQ, tK, tA, tU, p);
   }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;

@@ -138,6 +138,34 @@ def make_inputs(w: Workload, *, seed_base: int | None = None, B: int | None = No
     return out
 
 
+def make_inputs_device(w: Workload, *, seed: int, device="cuda", B: int | None = None,
+                       N: int | None = None) -> dict:
+    """The make_inputs recipe drawn on the device with torch's seeded generator (for timing-only
+    workloads whose inputs are too large to draw on the host): same shapes, distributions and
+    dtypes, different random numbers."""
+    B = w.B if B is None else B
+    N = w.N if N is None else N
+    H, d = w.H, w.d
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    dt = torch_dtype(w.dtype)
+    out = {}
+    for name in ("q", "k", "v"):
+        x = torch.randn((B, N, H, d), generator=g, device=device, dtype=torch.float32)
+        if name == "k" and w.gla_delta and w.n_gla:
+            kg = x[:, :, w.n_swa + w.n_dswa:, :]
+            kg /= kg.norm(dim=-1, keepdim=True)
+        out[name] = x.to(dt)
+        del x
+    out["alpha"] = out["beta"] = None
+    if w.n_gla:
+        shp = (B, N, w.n_gla) if w.gla_delta else (B, N, w.n_gla, d)
+        out["alpha"] = torch.sigmoid(torch.randn(shp, generator=g, device=device) + w.alpha_mu)
+        if w.gla_delta:
+            out["beta"] = torch.sigmoid(torch.randn(shp, generator=g, device=device))
+    return out
+
+
 def sample_rows(N: int, P: int, frac: float, seed: int) -> np.ndarray:
     """Query rows for sampled parity at full size: every frame's first and last row, the rows
     at multiples of 128 around them (tile edges), plus a seeded random fraction."""

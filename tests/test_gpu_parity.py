@@ -190,7 +190,8 @@ def test_bf16_gla_matches_oracle(kta, d, chunk, N, B, H):
 
 
 @pytest.mark.parametrize("d,N,B,H,with_s0", [(128, 300, 2, 2, True), (64, 1000, 1, 3, False),
-                                             (128, 4096, 1, 1, True)])
+                                             (128, 4096, 1, 1, True), (128, 50, 3, 1, True),
+                                             (64, 640, 2, 5, True)])
 def test_bf16_delta_matches_oracle(kta, d, N, B, H, with_s0):
     w = synth.DELTA_BF16.replace(d=d, n_gla=H)
     x = synth.make_inputs(w, N=N, B=B)
