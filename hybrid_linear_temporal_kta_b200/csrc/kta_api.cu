@@ -91,12 +91,13 @@ kta_status make_map(CUtensorMap* m, const void* base, int d, int heads, long lon
 
 // Tiled bf16 map of rank r (dims innermost first, byte strides of dims 1..r-1), 128-byte swizzle.
 kta_status make_map_nd(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                       const cuuint64_t* strides, const cuuint32_t* box) {
+                       const cuuint64_t* strides, const cuuint32_t* box,
+                       CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return KTA_OK;
@@ -105,8 +106,11 @@ kta_status make_map_nd(CUtensorMap* m, const void* base, int rank, const cuuint6
 // ------------------------------------------------------------------------- per-device state
 
 struct DeviceRes {
-  void* ws = nullptr;        // GLA segment workspace (grown on demand)
-  size_t ws_bytes = 0;
+  struct Buf {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+  };
+  std::map<cudaStream_t, Buf> ws;  // linear-attention workspace per stream (grown on demand)
   std::mutex mu;
 };
 
@@ -138,22 +142,26 @@ kta_status thread_streams(ThreadStreams** out) {
   return KTA_OK;
 }
 
-kta_status workspace(size_t bytes, void** out) {
+// Scratch for the chunked linear-attention kernels, one buffer per (device, CUDA stream): work on
+// one stream runs in order, so a buffer is never in use by two calls at once, and calls on
+// different streams never share one. It only grows (after that stream's earlier work is done).
+kta_status workspace(size_t bytes, cudaStream_t st, void** out) {
   int dev = 0;
   KTA_CUDA(cudaGetDevice(&dev));
   DeviceRes& r = device_res(dev);
   std::lock_guard<std::mutex> lk(r.mu);
-  if (r.ws_bytes < bytes) {
-    if (r.ws) {
-      KTA_CUDA(cudaDeviceSynchronize());
-      KTA_CUDA(cudaFree(r.ws));
-      r.ws = nullptr;
-      r.ws_bytes = 0;
+  DeviceRes::Buf& b = r.ws[st];
+  if (b.bytes < bytes) {
+    if (b.ptr) {
+      KTA_CUDA(cudaStreamSynchronize(st));
+      KTA_CUDA(cudaFree(b.ptr));
+      b.ptr = nullptr;
+      b.bytes = 0;
     }
-    KTA_CUDA(cudaMalloc(&r.ws, bytes));
-    r.ws_bytes = bytes;
+    KTA_CUDA(cudaMalloc(&b.ptr, bytes));
+    b.bytes = bytes;
   }
-  *out = r.ws;
+  *out = b.ptr;
   return KTA_OK;
 }
 
@@ -381,7 +389,7 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
   if (nseg > 1) {
     void* ws = nullptr;
     const size_t bytes = static_cast<size_t>(L.B) * L.H * nseg * (size_t(D) * D + D) * 4;
-    kta_status s = workspace(bytes, &ws);
+    kta_status s = workspace(bytes, st, &ws);
     if (s) return s;
     p.ws_S = static_cast<float*>(ws);
     p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * nseg * D * D;
@@ -415,9 +423,9 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
 
 template <int D>
 kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
-  constexpr int C = kta::DELTA_C, WARPS = 2, NST = 3;
+  constexpr int C = kta::DELTA_C, VG = 2, NST = 2;
   using PS = kta::DeltaPrepSmem<D>;
-  using SS = kta::DeltaScanSmem<D, WARPS, NST>;
+  using SS = kta::DeltaScanSmem<D, VG, NST>;
   const long long BH = static_cast<long long>(L.B) * L.H;
   if (BH > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
   const long long nch = (L.N + C - 1) / C;
@@ -441,14 +449,14 @@ kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
   const size_t units = static_cast<size_t>(BH) * nch;
   const size_t bytes = units * (static_cast<size_t>(C) * D * 2 * 2 + C * C * 2 + C * 4);
   void* ws = nullptr;
-  kta_status s = workspace(bytes, &ws);
+  kta_status s = workspace(bytes, st, &ws);
   if (s) return s;
   p.ws_W = static_cast<__nv_bfloat16*>(ws);
   p.ws_U = p.ws_W + units * C * D;
   p.ws_A = p.ws_U + units * D * C;
   p.ws_g = reinterpret_cast<float*>(p.ws_A + units * C * C);
 
-  CUtensorMap tW, tQ, tK, tA, tU;
+  CUtensorMap tW, tQ, tK, tA, tU, tO;
   {
     const cuuint64_t dW[2] = {static_cast<cuuint64_t>(D), units * C};
     const cuuint64_t sW[1] = {static_cast<cuuint64_t>(D) * 2};
@@ -468,10 +476,13 @@ kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
     const cuuint32_t bQ[4] = {64, 1, static_cast<cuuint32_t>(C), 1};
     if ((s = make_map_nd(&tQ, L.q, 4, dQ, sQ, bQ))) return s;
     if ((s = make_map_nd(&tK, L.k, 4, dQ, sQ, bQ))) return s;
+    // o: stores of [C tokens][VB value columns] tiles, unswizzled
+    const cuuint32_t bO[4] = {static_cast<cuuint32_t>(SS::VB), 1, static_cast<cuuint32_t>(C), 1};
+    if ((s = make_map_nd(&tO, L.o, 4, dQ, sQ, bO, CU_TENSOR_MAP_SWIZZLE_NONE))) return s;
   }
-  const size_t smem_p = sizeof(PS), smem_s = kta::delta_scan_smem_bytes<D, WARPS, NST>();
+  const size_t smem_p = sizeof(PS), smem_s = kta::delta_scan_smem_bytes<D, VG, NST>();
   if ((s = set_smem_attr(kta::delta_prep_kernel<D>, smem_p))) return s;
-  if ((s = set_smem_attr(kta::delta_scan_kernel<D, WARPS, NST>, smem_s))) return s;
+  if ((s = set_smem_attr(kta::delta_scan_kernel<D, VG, NST>, smem_s))) return s;
   {
     TraceScope ts("delta_prep", st);
     kta::delta_prep_kernel<D><<<dim3(static_cast<unsigned>(nch), static_cast<unsigned>(BH)), 128,
@@ -480,9 +491,9 @@ kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
   KTA_CUDA(cudaGetLastError());
   {
     TraceScope ts("delta_scan", st);
-    kta::delta_scan_kernel<D, WARPS, NST>
-        <<<dim3(D / SS::VB, static_cast<unsigned>(BH)), (WARPS + 1) * 32, smem_s, st>>>(
-            tW, tQ, tK, tA, tU, p);
+    kta::delta_scan_kernel<D, VG, NST>
+        <<<dim3(D / SS::VB, static_cast<unsigned>(BH)), (SS::NCW + 1) * 32, smem_s, st>>>(
+            tW, tQ, tK, tA, tU, tO, p);
   }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
@@ -998,7 +1009,6 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
     L.S_out = reinterpret_cast<float*>(s->arena + s->off_state[1 - s->cur]);
     L.scale = c.scale_gla;
     L.delta = c.gla_delta != 0;
-    L.allow_segments = false;
     if ((r = launch_lin(L, st))) return r;
     s->cur = 1 - s->cur;
   }

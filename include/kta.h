@@ -34,6 +34,12 @@
  *
  *  Scales: softmax scores use `scale` (d^-1/2 is standard attention); GLA / delta outputs are
  *  multiplied by `scale` (1.0 gives the pages' o_t = S_t q_t, which has no scale).
+ *
+ *  Library scratch: the chunked GLA and delta-rule calls keep one device workspace per (device,
+ *  CUDA stream) they run on, grown with cudaMalloc when a call needs more (after a
+ *  cudaStreamSynchronize of that stream) and kept until the process exits. Calls on the same
+ *  stream run in order; calls on different streams never share scratch. The gated delta rule
+ *  needs about 40 KB per 64-token chunk and head.
  */
 #ifndef KTA_H
 #define KTA_H
