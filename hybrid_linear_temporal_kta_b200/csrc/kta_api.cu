@@ -273,14 +273,15 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   p.scale_log2 = L.scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(L.o);
   p.o_ld = L.o_ld;
-  const long long nblk = static_cast<long long>(L.Fq) * Htot * L.B * p.n_qt;  // one CTA per tile
+  // one CTA per pair of query tiles of a (frame, head, sequence)
+  const long long nblk = static_cast<long long>(L.Fq) * Htot * L.B * ((p.n_qt + 1) / 2);
   if (nblk <= 0) return KTA_OK;
   if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "too many tiles (%lld)", nblk);
   const size_t smem = kta::win_smem_bytes<D>();
   if ((s = set_smem_attr(kta::win_attn_tc_kernel<D>, smem))) return s;
   {
     TraceScope ts("win_attn_tc", st);
-    kta::win_attn_tc_kernel<D><<<static_cast<unsigned>(nblk), 192, smem, st>>>(tq, tk0, tv0, tk1,
+    kta::win_attn_tc_kernel<D><<<static_cast<unsigned>(nblk), 384, smem, st>>>(tq, tk0, tv0, tk1,
                                                                                tv1, p);
   }
   const cudaError_t le = cudaGetLastError();
@@ -288,7 +289,7 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, kta::win_attn_tc_kernel<D>);
     return fail(KTA_ERR_CUDA,
-                "win_attn_tc launch failed: %s (grid %lld x 192, dyn smem %zu, regs %d, max threads "
+                "win_attn_tc launch failed: %s (grid %lld x 384, dyn smem %zu, regs %d, max threads "
                 "%d, max dyn smem %d)",
                 cudaGetErrorString(le), nblk, smem, fa.numRegs, fa.maxThreadsPerBlock,
                 fa.maxDynamicSharedSizeBytes);

@@ -4,19 +4,28 @@
 // pillar. SWA: standard attention over a window of W whole frames ending at the query's frame.
 // DSWA: the same window size with frames taken every dil-th step back (f, f-dil, ...).
 //
-// One CTA computes one tile of up to 128 query rows that lie in ONE frame (tiles restart at
-// every frame start), so every row of the tile sees the same key frames and the only mask is a
-// column bound on the last key tile of each key span. Key spans: for dil == 1 the W visible
-// frames are adjacent and form one span; for dil > 1 each visible frame is its own span.
+// Query tiles of up to 128 rows lie in ONE frame (tiles restart at every frame start), so every
+// row of a tile sees the same key frames and the only mask is a column bound on the last key tile
+// of each key span. Key spans: for dil == 1 the W visible frames are adjacent and form one span;
+// for dil > 1 each visible frame is its own span.
 //
-// Warp roles (192 threads, two CTAs per SM so one CTA's softmax overlaps the other's MMAs):
-//   warp 0      TMA producer: Q once, then K_i and V_i tiles (128 keys x D, 128-byte swizzle).
-//   warp 1      allocates 256 TMEM columns; one thread issues tcgen05.mma:
-//               S = Q K_i^T (SS form, fp32 in TMEM cols [0,128)), then O += P_i V_i (TS form,
-//               P_i read from TMEM where the softmax warps wrote it over S, V MN-major).
-//   warps 2..5  softmax: thread <-> query row (TMEM lane). Row max, lazy rescale of O in TMEM
-//               when the max grows by more than 2^8, P = exp2(S*scale*log2e - m) as bf16 into
-//               TMEM, running row sum; epilogue O / l -> bf16 -> global.
+// One CTA (one per SM: it holds all 512 TMEM columns) computes a PAIR of query tiles A and B of
+// the same sequence, head and frame; both use every K / V tile, which is loaded once for the pair
+// into a four-slot ring (K_0, V_0, K_1, V_1, ...; 128 keys x D, 128-byte swizzle), so the loads
+// run a full key tile ahead of the tensor core. Warp roles (384 threads):
+//   warp 0       TMA producer: Q_A and Q_B once, then the K / V ring.
+//   warp 1       allocates TMEM (S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)); one
+//                thread issues tcgen05.mma in the order S_A(0) S_B(0) | PV_A(i) S_A(i+1) PV_B(i)
+//                S_B(i+1) | ...: S = Q K^T (SS form), O += P V (TS form, P read from TMEM where
+//                the softmax wrote it over S, V MN-major). MMAs of one thread run in issue order,
+//                so S_X(i+1) overwrites P_X(i) only after PV_X(i) has read it, and the softmax of
+//                S_X(i+1) finds O_X stable.
+//   warps 2, 3   idle after set-up.
+//   warps 4..7   softmax of tile A; warps 8..11 softmax of tile B: thread <-> query row (TMEM
+//                lane). Row max (three-input max), lazy rescale of O when the max grows by more
+//                than 2^8, P = exp2(S*scale*log2e - m) as bf16 into TMEM (scaling and row sums on
+//                packed fp32 pairs), running row sum; epilogue O / l -> bf16 -> global.
+// While the softmax of one tile runs, the tensor core works on the other tile's products.
 // Every wait is bounded; on a timeout the CTA records it and unwinds to free its TMEM.
 #pragma once
 
@@ -76,23 +85,21 @@ template <int D>
 struct WinSmem {
   static constexpr int BOX = 128 * 64 * 2;  // one 128-row x 64-column bf16 box, 16 KB
   static constexpr int NBOX = D / 64;
-  alignas(1024) uint8_t q[NBOX * BOX];
-  alignas(1024) uint8_t k[NBOX * BOX];
-  alignas(1024) uint8_t v[NBOX * BOX];
-  uint64_t bar_q, bar_kfull, bar_kempty, bar_vfull, bar_vempty, bar_s, bar_p, bar_pv, bar_fin;
+  static constexpr int NSLOT = 4;           // K / V ring slots
+  alignas(1024) uint8_t q[2][NBOX * BOX];
+  alignas(1024) uint8_t kv[NSLOT][NBOX * BOX];
+  uint64_t bar_q, full[NSLOT], empty[NSLOT], bar_s[2], bar_p[2], bar_o[2], bar_fin;
   uint32_t tmem_base;
   int abort_flag;
 };
 
 template <int D>
 constexpr size_t win_smem_bytes() {
-  // +1024 for manual alignment of the dynamic shared memory base; at least 80 KB so that no
-  // more than two CTAs (2 x 256 TMEM columns) share an SM.
-  return sizeof(WinSmem<D>) + 1024 > 80 * 1024 ? sizeof(WinSmem<D>) + 1024 : 80 * 1024;
+  return sizeof(WinSmem<D>) + 1024;  // + manual 1024-byte alignment of the dynamic base
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(384, 1)
     win_attn_tc_kernel(const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk0,
                        const __grid_constant__ CUtensorMap tv0,
@@ -104,14 +111,16 @@ __global__ void __launch_bounds__(192, 2)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   constexpr int BOX = WinSmem<D>::BOX;
   constexpr int NBOX = WinSmem<D>::NBOX;
+  constexpr int NSLOT = WinSmem<D>::NSLOT;
   constexpr uint32_t TILE_BYTES = 128 * D * 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item: frames latest first (full windows first), then head, sequence, tile
+  // ---- work item: frames latest first (full windows first), then head, sequence, tile pair
+  const int n_pairs = (p.n_qt + 1) >> 1;
   int item = blockIdx.x;
-  const int qt = item % p.n_qt;
-  item /= p.n_qt;
+  const int pr = item % n_pairs;
+  item /= n_pairs;
   const int b = item % p.B;
   item /= p.B;
   const int h = item % p.Htot;
@@ -127,32 +136,32 @@ __global__ void __launch_bounds__(192, 2)
   const CUtensorMap* tk = g ? &tk1 : &tk0;
   const CUtensorMap* tv = g ? &tv1 : &tv0;
   const int ntiles = win_num_tiles(f, p.P, W, dil);
-  const int q_row0 = b * p.q_rows_b + f_local * p.P + qt * 128;
-  const int nq = min(128, p.P - qt * 128);
+  const bool has_b = 2 * pr + 1 < p.n_qt;
+  const int q_row0 = b * p.q_rows_b + f_local * p.P + pr * 256;  // tile A; tile B = +128
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
-    mbar_init(&sm.bar_kfull, 1);
-    mbar_init(&sm.bar_kempty, 1);
-    mbar_init(&sm.bar_vfull, 1);
-    mbar_init(&sm.bar_vempty, 1);
-    mbar_init(&sm.bar_s, 1);
-    mbar_init(&sm.bar_p, 128);
-    mbar_init(&sm.bar_pv, 1);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.bar_s[x], 1);
+      mbar_init(&sm.bar_p[x], 128);
+      mbar_init(&sm.bar_o[x], 1);
+    }
     mbar_init(&sm.bar_fin, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
     __syncwarp();
-    tmem_alloc(&sm.tmem_base, 256);
+    tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tS = sm.tmem_base;        // S / P: columns [0, 128)
-  const uint32_t tO = sm.tmem_base + 128;  // O: columns [128, 128 + D)
   volatile int* abort_flag = &sm.abort_flag;
 
   if (warp == 0) {
@@ -161,169 +170,222 @@ __global__ void __launch_bounds__(192, 2)
       prefetch_tmap(&tq);
       prefetch_tmap(tk);
       prefetch_tmap(tv);
-      mbar_arrive_expect_tx(&sm.bar_q, TILE_BYTES);
-      for (int c = 0; c < NBOX; ++c) tma_load_3d(sm.q + c * BOX, &tq, &sm.bar_q, c * 64, h, q_row0);
-      int k_issued = 0, v_issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
+      mbar_arrive_expect_tx(&sm.bar_q, has_b ? 2 * TILE_BYTES : TILE_BYTES);
+      for (int x = 0; x < (has_b ? 2 : 1); ++x)
+        for (int c = 0; c < NBOX; ++c)
+          tma_load_3d(sm.q[x] + c * BOX, &tq, &sm.bar_q, c * 64, h, q_row0 + 128 * x);
+      int issued = 0;
+      for (int n = 0; n < 2 * ntiles; ++n) {  // load n: K_{n/2} (n even) or V_{n/2} (n odd)
         if (*abort_flag) break;
+        const int slot = n % NSLOT, use = n / NSLOT;
         int fr0, off, nv;
-        win_tile(i, f, p.P, W, dil, fr0, off, nv);
+        win_tile(n >> 1, f, p.P, W, dil, fr0, off, nv);
         const int krow = (b * kbf + fr0 % kmod) * p.P + off;
-        if (i > 0 && !mbar_wait(&sm.bar_kempty, (i - 1) & 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&sm.bar_kfull, TILE_BYTES);
-        for (int c = 0; c < NBOX; ++c) tma_load_3d(sm.k + c * BOX, tk, &sm.bar_kfull, c * 64, hk, krow);
-        ++k_issued;
-        if (i > 0 && !mbar_wait(&sm.bar_vempty, (i - 1) & 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&sm.bar_vfull, TILE_BYTES);
-        for (int c = 0; c < NBOX; ++c) tma_load_3d(sm.v + c * BOX, tv, &sm.bar_vfull, c * 64, hk, krow);
-        ++v_issued;
+        if (use > 0 && !mbar_wait(&sm.empty[slot], (use - 1) & 1)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(&sm.full[slot], TILE_BYTES);
+        const CUtensorMap* tm = (n & 1) ? tv : tk;
+        for (int c = 0; c < NBOX; ++c)
+          tma_load_3d(sm.kv[slot] + c * BOX, tm, &sm.full[slot], c * 64, hk, krow);
+        ++issued;
       }
       // Let the copies this thread started land before the CTA can exit (bounded waits).
       mbar_wait(&sm.bar_q, 0);
-      if (k_issued > 0) mbar_wait(&sm.bar_kfull, (k_issued - 1) & 1);
-      if (v_issued > 0) mbar_wait(&sm.bar_vfull, (v_issued - 1) & 1);
+      for (int n = issued - NSLOT > 0 ? issued - NSLOT : 0; n < issued; ++n)
+        mbar_wait(&sm.full[n % NSLOT], (n / NSLOT) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t ID_O = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_base = smem_u32(sm.q), k_base = smem_u32(sm.k), v_base = smem_u32(sm.v);
-      bool ok = mbar_wait(&sm.bar_q, 0);
-      if (!ok) *abort_flag = 1;
-      for (int i = 0; ok && i < ntiles; ++i) {
-        if (*abort_flag) break;
-        if (!mbar_wait(&sm.bar_kfull, i & 1)) { *abort_flag = 1; break; }
-        // P_{i-1} lives in the S columns: S_i may only be written once PV_{i-1} has finished.
-        if (i > 0 && !mbar_wait(&sm.bar_pv, (i - 1) & 1)) { *abort_flag = 1; break; }
-        tc_fence_after();
+      const uint32_t tbase = sm.tmem_base;
+      const uint32_t q_base[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      auto issue_s = [&](int x, int slot) {
+        const uint32_t k_base = smem_u32(sm.kv[slot]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
-          mma_ss(tS, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(k_base + off, 16, 1024),
-                 ID_S, kk > 0 ? 1u : 0u);
+          mma_ss(tbase + 128 * x, smem_desc_sw128(q_base[x] + off, 16, 1024),
+                 smem_desc_sw128(k_base + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.bar_s);
-        mma_commit(&sm.bar_kempty);
-        if (!mbar_wait(&sm.bar_p, i & 1)) { *abort_flag = 1; break; }
-        if (!mbar_wait(&sm.bar_vfull, i & 1)) { *abort_flag = 1; break; }
-        tc_fence_after();
+        mma_commit(&sm.bar_s[x]);
+      };
+      auto issue_pv = [&](int x, int slot, bool first) {
+        const uint32_t v_base = smem_u32(sm.kv[slot]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(tO, tS + kk * 8, smem_desc_sw128(v_base + kk * 16 * 128, BOX, 1024), ID_O,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&sm.bar_pv);
-        mma_commit(&sm.bar_vempty);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tbase + 256 + 128 * x, tbase + 128 * x + kk * 8,
+                 smem_desc_sw128(v_base + kk * 16 * 128, BOX, 1024), ID_O,
+                 (!first || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_o[x]);
+      };
+      bool ok = mbar_wait(&sm.bar_q, 0) && ntiles > 0;
+      if (ok && !mbar_wait(&sm.full[0], 0)) ok = false;
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (has_b) issue_s(1, 0);
+        mma_commit(&sm.empty[0]);
       }
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int vs = (2 * i + 1) % NSLOT;
+        const uint32_t ph = (i >> 1) & 1;  // phase of both slots of tile i
+        const bool more = i + 1 < ntiles;
+        const int ks1 = (2 * i + 2) % NSLOT;
+        const uint32_t ph1 = ((i + 1) >> 1) & 1;
+        if (*abort_flag) { ok = false; break; }
+        // tile A: PV_A(i), then S_A(i+1)
+        if (!mbar_wait(&sm.bar_p[0], i & 1) || !mbar_wait(&sm.full[vs], ph)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, vs, i == 0);
+        if (more) {
+          if (!mbar_wait(&sm.full[ks1], ph1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(0, ks1);
+        }
+        // tile B: PV_B(i), then S_B(i+1)
+        if (has_b) {
+          if (!mbar_wait(&sm.bar_p[1], i & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, vs, i == 0);
+        }
+        mma_commit(&sm.empty[vs]);
+        if (more) {
+          if (has_b) issue_s(1, ks1);
+          mma_commit(&sm.empty[ks1]);
+        }
+      }
+      if (!ok) *abort_flag = 1;
       // All MMAs issued by this thread are complete once bar_fin flips.
       mma_commit(&sm.bar_fin);
       mbar_wait(&sm.bar_fin, 0);
     }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue (tile x)
+    const int x = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
+    const int nq = min(128, p.P - (2 * pr + x) * 128);  // rows of this tile inside the frame
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = sm.tmem_base + 128 * x;
+    const uint32_t tO = sm.tmem_base + 256 + 128 * x;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
+    bool ok = x == 0 || has_b;
+    for (int i = 0; ok && i < ntiles; ++i) {
       int fr0, off, nv;
       win_tile(i, f, p.P, W, dil, fr0, off, nv);
-      const bool got = !*abort_flag && mbar_wait(&sm.bar_s, i & 1);
+      const bool got = !*abort_flag && mbar_wait(&sm.bar_s[x], i & 1);
       if (!__all_sync(0xffffffffu, got)) { *abort_flag = 1; ok = false; break; }
       tc_fence_after();
-      // pass 1: row maximum of the valid columns
-      float mx = -INFINITY;
+      // the whole S row in registers: four loads, one wait
+      uint32_t r[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + lane_off + 32 * c, r);
-        tmem_wait_ld();
-        if (nv == 128) {
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+      tmem_wait_ld();
+      tmem_ld_fence(r);
+      // row maximum of the valid columns (three-input max, four independent partial maxima)
+      float mp[4];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(r[j]));
-        } else {
+      for (int u = 0; u < 4; ++u) mp[u] = -INFINITY;
+      if (nv == 128) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (32 * c + j < nv) mx = fmaxf(mx, __uint_as_float(r[j]));
-        }
+        for (int j = 0; j < 64; ++j)
+          mp[j & 3] = max3f(mp[j & 3], __uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          if (j < nv) mp[j & 3] = fmaxf(mp[j & 3], __uint_as_float(r[j]));
       }
+      const float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
       const float mnew = fmaxf(m, mx * sl2);
+      // lazy rescale: the reference m moves only when the row maximum grows by more than 2^8
+      bool rescale = false;
+      float fac = 1.0f;
       if (i == 0) {
         m = mnew;
       } else {
         const bool need = mnew > m + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          // O is stable here: S_i was issued only after PV_{i-1} completed.
-          const float fac = need ? ex2_approx(m - mnew) : 1.0f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + lane_off + 32 * c, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * fac);
-            tmem_st32(tO + lane_off + 32 * c, r);
-          }
-          tmem_wait_st();
-          if (need) {
-            l *= fac;
-            m = mnew;
-          }
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          fac = ex2_approx(m - mnew);
+          m = mnew;
         }
       }
-      // pass 2: P = exp2(S * scale * log2e - m) as bf16 pairs, written over S
-      float ls = 0.f;
+      // P = exp2(S * scale * log2e - m) as bf16 pairs, written over S (the scaling and the row
+      // sum on packed fp32 pairs)
+      const uint64_t sc2 = f32x2_pack(sl2, sl2), nm2 = f32x2_pack(-m, -m);
+      uint64_t lp2[2] = {f32x2_pack(0.f, 0.f), f32x2_pack(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + lane_off + 32 * c, r);
-        tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int col = 32 * c + 2 * j;
-          float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * j]), sl2, -m));
-          float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * j + 1]), sl2, -m));
+          float x0, x1;
+          f32x2_unpack(ffma2(f32x2_pack(__uint_as_float(r[col]), __uint_as_float(r[col + 1])), sc2, nm2),
+                       x0, x1);
+          float p0 = ex2_approx(x0);
+          float p1 = ex2_approx(x1);
           if (nv < 128) {
             p0 = col < nv ? p0 : 0.f;
             p1 = col + 1 < nv ? p1 : 0.f;
           }
-          ls += p0 + p1;
+          lp2[j & 1] = fadd2(lp2[j & 1], f32x2_pack(p0, p1));
           pk[j] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + lane_off + 16 * c, pk);
       }
-      l += ls;
+      float la, lb, lc, ld;
+      f32x2_unpack(lp2[0], la, lb);
+      f32x2_unpack(lp2[1], lc, ld);
+      if (rescale) {
+        // O is stable here: S_x(i) completed, and it runs after PV_x(i-1) on the tensor pipe.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ro[32];
+          tmem_ld32(tO + lane_off + 32 * c, ro);
+          tmem_wait_ld();
+          tmem_ld_fence(ro);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * fac);
+          tmem_st32(tO + lane_off + 32 * c, ro);
+        }
+        l *= fac;
+      }
+      l += (la + lb) + (lc + ld);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.bar_p);
+      mbar_arrive(&sm.bar_p[x]);
     }
     // epilogue: O / l -> bf16 -> global (rows of this frame only)
-    const bool fin = ok && ntiles > 0 && mbar_wait(&sm.bar_pv, (ntiles - 1) & 1);
-    if (__all_sync(0xffffffffu, fin)) {
-      tc_fence_after();
-      const float inv = 1.0f / l;
-      __nv_bfloat16* orow = p.o + static_cast<long long>(q_row0 + row) * p.o_ld + h * D;
+    const bool active = x == 0 || has_b;
+    if (active) {
+      const bool fin = ok && ntiles > 0 && mbar_wait(&sm.bar_o[x], (ntiles - 1) & 1);
+      if (__all_sync(0xffffffffu, fin)) {
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        __nv_bfloat16* orow =
+            p.o + static_cast<long long>(q_row0 + 128 * x + row) * p.o_ld + h * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + lane_off + 32 * c, r);
-        tmem_wait_ld();
-        if (row < nq) {
-          uint32_t w[16];
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tO + lane_off + 32 * c, rr);
+          tmem_wait_ld();
+          tmem_ld_fence(rr);
+          if (row < nq) {
+            uint32_t w[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            w[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * inv, __uint_as_float(r[2 * j + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+            for (int j = 0; j < 16; ++j)
+              w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * inv, __uint_as_float(rr[2 * j + 1]) * inv);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          }
         }
+      } else {
+        *abort_flag = 1;
       }
-    } else {
-      *abort_flag = 1;
     }
     tc_fence_before();
   }
@@ -331,7 +393,7 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(sm.tmem_base, 256);
+    tmem_dealloc(sm.tmem_base, 512);
   }
 }
 
