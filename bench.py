@@ -211,7 +211,7 @@ def rank_seed_base(base: int, rank: int) -> int:
 # --------------------------------------------------------------------------- CPU oracle timing
 
 
-def oracle_sample(w, x, target_s: float = 12.0):
+def oracle_sample(w, x, target_s: float = 20.0):
     """Time the fp64 CPU oracle on a bounded sample of the workload: M query rows (seeded) of the
     16 softmax heads plus the first M tokens of the 8 GLA heads. Returns tokens/s and details."""
     import numpy as np

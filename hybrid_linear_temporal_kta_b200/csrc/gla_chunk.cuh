@@ -21,10 +21,11 @@
 //                            one thread per state element, written over S_loc in the workspace;
 //   pass 2 (OUTPUT = true):  each segment runs its chunks from S_start and writes o.
 // The value dimension is split in BV = 64 column slices (columns of S are independent).
-// CTA = 4 warps, two CTAs per SM. Warp w computes output rows [16w, 16w+16) of a chunk and state
+// CTA = 4 warps, three CTAs per SM. Warp w computes output rows [16w, 16w+16) of a chunk and state
 // rows [w*D/4, (w+1)*D/4).
 #pragma once
 
+#include "kta_ptx.cuh"
 #include "mma_sync.cuh"
 
 namespace kta {
@@ -57,13 +58,12 @@ struct GlaSmem {
   __nv_bfloat16 k[C * LDK];   // raw k, then Ki
   __nv_bfloat16 v[C * LDV];
   __nv_bfloat16 s[D * LDV];   // bf16 copy of diag(2^{b_m}) S_0 (value slice)
-  float g[C * D];             // alpha, then the cumulative log2 gate b_t
   float emid[D];              // 2^{b_m}
   float cend[D];              // 2^{b_C - b_m}
 };
 
 template <int D, int C, bool OUTPUT>
-__global__ void __launch_bounds__(128, 2) gla_chunk_kernel(const GlaParams p) {
+__global__ void __launch_bounds__(128, 3) gla_chunk_kernel(const GlaParams p) {
   using SM = GlaSmem<D, C>;
   constexpr int BV = SM::BV, LDK = SM::LDK, LDV = SM::LDV;
   constexpr int RW = D / 4;           // state rows per warp
@@ -149,40 +149,41 @@ __global__ void __launch_bounds__(128, 2) gla_chunk_kernel(const GlaParams p) {
         cp_async16(&sm.v[t * LDV + c], p.v + grow * p.ld + static_cast<long long>(h) * D + j0 + c,
                    t < n ? 16 : 0);
       }
-      constexpr int ACH = D / 4;  // 16-byte pieces per fp32 row
-      for (int idx = tid; idx < C * ACH; idx += 128) {
-        const int t = idx / ACH, c = (idx % ACH) * 4;
-        if (t < n) {
-          const long long grow = row_b + c0 + t;
-          cp_async16(&sm.g[t * D + c], p.alpha + (grow * p.H + h) * D + c, 16);
-        } else {
-          *reinterpret_cast<float4*>(&sm.g[t * D + c]) = make_float4(1.f, 1.f, 1.f, 1.f);
-        }
-      }
-      cp_async_wait_all();
+      cp_async_commit();
     }
-    __syncthreads();
-    // ---- cumulative log2 gate per key dim, and the per-dim factors 2^{b_m}, 2^{b_C - b_m}
+    // gates of this thread's key column (rows >= n: alpha = 1), loaded straight into registers
+    // while the copies above are in flight; bt[t] becomes the cumulative log2 gate below
+    float bt[C];
     if (tid < D) {
-      float acc = 0.f, bm = 0.f;
-#pragma unroll 8
+      const float* ap = p.alpha + ((row_b + c0) * p.H + h) * D + tid;
+#pragma unroll
+      for (int t = 0; t < C; ++t) bt[t] = t < n ? __ldg(ap + static_cast<long long>(t) * p.H * D) : 1.f;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // ---- per key dim (thread tid < D owns column tid): the cumulative log2 gate b_t in
+    // registers, the factors 2^{b_m}, 2^{b_C - b_m}, and the decayed operands of its column,
+    // Ki_t = k_t 2^{b_m - b_t} and Qi_t = q_t 2^{b_t - b_m}, written in place
+    if (tid < D) {
+      float acc = 0.f;
+#pragma unroll
       for (int t = 0; t < C; ++t) {
-        acc += __log2f(sm.g[t * D + tid]);
-        sm.g[t * D + tid] = acc;
-        if (t == MID) bm = acc;
+        acc += __log2f(bt[t]);
+        bt[t] = acc;
       }
-      sm.emid[tid] = exp2f(bm);
-      sm.cend[tid] = exp2f(acc - bm);
+      const float bm = bt[MID];
+      sm.emid[tid] = ex2_approx(bm);
+      sm.cend[tid] = ex2_approx(acc - bm);
       ltot += acc;
+#pragma unroll
+      for (int t = 0; t < C; ++t) {
+        const float dd = bt[t] - bm;
+        sm.k[t * LDK + tid] = __float2bfloat16_rn(__bfloat162float(sm.k[t * LDK + tid]) * ex2_approx(-dd));
+        if (OUTPUT)
+          sm.q[t * LDK + tid] = __float2bfloat16_rn(__bfloat162float(sm.q[t * LDK + tid]) * ex2_approx(dd));
+      }
     }
     __syncthreads();
-    // ---- decayed operands (in place) and the pre-scaled state
-    for (int idx = tid; idx < C * D; idx += 128) {
-      const int t = idx / D, i = idx % D;
-      const float d = sm.g[t * D + i] - sm.g[MID * D + i];
-      sm.k[t * LDK + i] = __float2bfloat16_rn(__bfloat162float(sm.k[t * LDK + i]) * exp2f(-d));
-      if (OUTPUT) sm.q[t * LDK + i] = __float2bfloat16_rn(__bfloat162float(sm.q[t * LDK + i]) * exp2f(d));
-    }
     prescale_and_publish();
     __syncthreads();
 

@@ -366,7 +366,7 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
   const int nchunks = (L.N + C - 1) / C;
   int nseg = 1;
   if (L.allow_segments) {
-    const long long want = (4LL * 148 + base - 1) / base;
+    const long long want = (3LL * 148 + base - 1) / base;  // one wave of 3 CTAs per SM
     nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
   }
   const int seg_chunks = (nchunks + nseg - 1) / nseg;
@@ -1217,7 +1217,7 @@ kta_status launch_gla_chunk_noalloc(const LinLaunch& L, cudaStream_t st) {
   const int slices = D / SM::BV;
   const long long base = static_cast<long long>(L.B) * L.H * slices;
   const int nchunks = (L.N + C - 1) / C;
-  const long long want = (4LL * 148 + base - 1) / base;
+  const long long want = (3LL * 148 + base - 1) / base;  // one wave of 3 CTAs per SM
   int nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
   const int seg_chunks = (nchunks + nseg - 1) / nseg;
   const int seg_len = seg_chunks * C;
