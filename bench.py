@@ -39,6 +39,11 @@ def parse_args():
     ap.add_argument("--impl", choices=("kta", "reference"), default="kta")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing leg (faster profiling runs)")
+    ap.add_argument("--frames", type=int, default=None,
+                    help="profiling only: override the hybrid workload's frame count (the "
+                         "headline line is the default, 21 frames)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="profiling only: override the delta workload's tokens per sequence")
     ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep"),
                     default="hybrid",
                     help="hybrid: the 21-frame hybrid layer (the headline line); delta: gated "
@@ -291,7 +296,8 @@ def run_kta(args):
 
     from hybrid_linear_temporal_kta_b200 import kta, synth
 
-    w = synth.HYBRID_BF16
+    w = synth.HYBRID_BF16 if args.frames is None else synth.HYBRID_BF16.replace(
+        name=f"hybrid_bf16_F{args.frames}_P1560", F=args.frames)
     x = synth.make_inputs(w, seed_base=rank_seed_base(w.seed_base, rank))
     cfg = kta.cfg_from_workload(w)
     host = {n: x[n].pin_memory() for n in ("q", "k", "v", "alpha")}
@@ -386,7 +392,8 @@ def run_kta(args):
                    "d": w.d, "heads": f"{w.n_swa} SWA W={w.W_swa} | {w.n_dswa} DSWA W={w.W_dswa} "
                                       f"dil={w.dil} | {w.n_gla} GLA chunk={w.chunk}",
                    "parallelism": f"dp{ws} (independent sequences per GPU, no collective)",
-                   "l2": "inputs 738 MB per step > 126 MB L2; no flush"},
+                   "l2": f"inputs {h2d / 1e6:.0f} MB per step"
+                         f"{' > 126 MB L2; no flush' if h2d > 126e6 else ' (fits L2)'}"},
         "roofline": {"kernel": "win_attn_tc (SWA+DSWA heads, tcgen05)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
@@ -458,6 +465,8 @@ def run_other(args):
     lines = []
     if args.workload == "delta":
         w = synth.DELTA_BF16
+        if args.tokens is not None:
+            w = w.replace(name=f"gated_delta_bf16_B2_L{args.tokens}", F=1, P=args.tokens)
         x = synth.make_inputs_device(w, seed=w.seed_base)
         o = torch.empty_like(x["q"])
 
