@@ -306,19 +306,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 64 (inputs below -126 return ~0). Cody-Waite split x = n + f with
-// n = rint(x) (the 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2]; 2^f from a cubic fitted by
-// least squares at 2000 Chebyshev nodes on [-1/2, 1/2] (max relative error 7.8e-5, far below
-// bf16 resolution); 2^n is added to the exponent field. Used to take part of the softmax
-// exponentials off the MUFU pipe.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.05508868f, f, 0.24260405f), f, 0.69327623f), f, 0.99992895f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Three-input maximum (one instruction on sm_100).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
