@@ -273,8 +273,11 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   p.scale_log2 = L.scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(L.o);
   p.o_ld = L.o_ld;
-  // one CTA per pair of query tiles of a (frame, head, sequence)
-  const long long nblk = static_cast<long long>(L.Fq) * Htot * L.B * ((p.n_qt + 1) / 2);
+  // one CTA per pair of query tiles of a (frame, head, sequence); one per tile when pairs would
+  // leave SMs idle (a streaming step's single frame)
+  const long long units = static_cast<long long>(L.Fq) * Htot * L.B;
+  p.pair = units * ((p.n_qt + 1) / 2) >= 2 * 148 ? 2 : 1;
+  const long long nblk = units * (p.pair == 2 ? (p.n_qt + 1) / 2 : p.n_qt);
   if (nblk <= 0) return KTA_OK;
   if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "too many tiles (%lld)", nblk);
   const size_t smem = kta::win_smem_bytes<D>();

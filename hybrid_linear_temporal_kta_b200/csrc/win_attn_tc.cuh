@@ -10,7 +10,8 @@
 // for dil > 1 each visible frame is its own span.
 //
 // One CTA (one per SM: it holds all 512 TMEM columns) computes a PAIR of query tiles A and B of
-// the same sequence, head and frame; both use every K / V tile, which is loaded once for the pair
+// the same sequence, head and frame (launches too small to fill the GPU with pairs give each CTA
+// one tile); both use every K / V tile, which is loaded once for the pair
 // into a four-slot ring (K_0, V_0, K_1, V_1, ...; 128 keys x D, 128-byte swizzle), so the loads
 // run a full key tile ahead of the tensor core. Warp roles (384 threads):
 //   warp 0       TMA producer: Q_A and Q_B once, then the K / V ring.
@@ -39,6 +40,7 @@ struct WinParams {
   int Fq;           // query frames in this launch (sequence: F; streaming step: 1)
   int f_base;       // absolute frame index of query frame 0
   int n_qt;         // query tiles per frame = ceil(P / 128)
+  int pair;         // query tiles per CTA: 2 (tiles 2u, 2u+1) or 1 (small launches)
   int Htot;         // heads in this launch (group 0 then group 1)
   int H0;           // heads of group 0
   int W[2];         // window (frames) per group
@@ -117,10 +119,10 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work item: frames latest first (full windows first), then head, sequence, tile pair
-  const int n_pairs = (p.n_qt + 1) >> 1;
+  const int n_units = p.pair == 2 ? (p.n_qt + 1) >> 1 : p.n_qt;
   int item = blockIdx.x;
-  const int pr = item % n_pairs;
-  item /= n_pairs;
+  const int pr = item % n_units;  // first query tile of this CTA: pr * p.pair
+  item /= n_units;
   const int b = item % p.B;
   item /= p.B;
   const int h = item % p.Htot;
@@ -136,8 +138,8 @@ __global__ void __launch_bounds__(384, 1)
   const CUtensorMap* tk = g ? &tk1 : &tk0;
   const CUtensorMap* tv = g ? &tv1 : &tv0;
   const int ntiles = win_num_tiles(f, p.P, W, dil);
-  const bool has_b = 2 * pr + 1 < p.n_qt;
-  const int q_row0 = b * p.q_rows_b + f_local * p.P + pr * 256;  // tile A; tile B = +128
+  const bool has_b = p.pair == 2 && 2 * pr + 1 < p.n_qt;
+  const int q_row0 = b * p.q_rows_b + f_local * p.P + pr * p.pair * 128;  // tile A; B = +128
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(384, 1)
     const int x = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int nq = min(128, p.P - (2 * pr + x) * 128);  // rows of this tile inside the frame
+    const int nq = min(128, p.P - (p.pair * pr + x) * 128);  // rows of this tile in the frame
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = sm.tmem_base + 128 * x;
     const uint32_t tO = sm.tmem_base + 256 + 128 * x;
