@@ -66,7 +66,7 @@ def _load():
             lib.oracle_gla.argtypes = [_f32p, _f32p, _f32p, _f32p, _f64p, _f64p, _f64p] + [
                 _int] * 6 + [ctypes.c_double]
             lib.oracle_delta.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p,
-                                         _f64p] + [_int] * 6 + [ctypes.c_double]
+                                         _f64p] + [_int] * 6 + [ctypes.c_double, _int]
             lib.oracle_visible.argtypes = [_i64p, _i64p, ctypes.c_int64, _int, _int, _int, _int,
                                            _u8p]
             lib.oracle_set_threads.argtypes = [_int]
@@ -166,8 +166,11 @@ def gla(q, k, v, alpha, scale: float = 1.0, S0=None, heads=None, out=None):
     return o, S_out
 
 
-def delta(q, k, v, alpha, beta, scale: float = 1.0, S0=None, heads=None, out=None):
-    """Gated delta rule in the page's form; alpha, beta: [B, N, h1-h0] scalars.
+def delta(q, k, v, alpha, beta, scale: float = 1.0, S0=None, heads=None, out=None,
+          erase_decayed: bool = False):
+    """Gated delta rule in the page's form; alpha, beta: [B, N, h1-h0] scalars. With
+    erase_decayed the erase term is decayed too (the GatedDeltaNet form
+    M_t = alpha_t M_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T).
 
     Returns (o [B, N, H, d] float64, S_out [B, h1-h0, d, d] float64, key-major, i.e. the
     transpose of the page's d_v x d_k state).
@@ -180,13 +183,14 @@ def delta(q, k, v, alpha, beta, scale: float = 1.0, S0=None, heads=None, out=Non
     s0 = None if S0 is None else _f64(S0)
     rc = _load().oracle_delta(_p(q, _f32p), _p(k, _f32p), _p(v, _f32p), _p(a, _f32p),
                               _p(be, _f32p), None if s0 is None else _p(s0, _f64p),
-                              _p(o, _f64p), _p(S_out, _f64p), B, N, H, d, h0, h1, float(scale))
+                              _p(o, _f64p), _p(S_out, _f64p), B, N, H, d, h0, h1, float(scale),
+                              int(bool(erase_decayed)))
     _check(rc, "delta")
     return o, S_out
 
 
 def hybrid(q, k, v, alpha, beta, *, P: int, n_swa: int, n_dswa: int, n_gla: int,
-           W_swa: int, W_dswa: int, dil: int, gla_delta: bool = False,
+           W_swa: int, W_dswa: int, dil: int, gla_delta: int = 0,
            scale_softmax: float, scale_gla: float = 1.0, rows=None):
     """Per-head split (SWA heads, then DSWA heads, then GLA heads), outputs concatenated by
     head. The pages only say that the three branches are mixed; the head split is the
@@ -204,8 +208,9 @@ def hybrid(q, k, v, alpha, beta, *, P: int, n_swa: int, n_dswa: int, n_gla: int,
     S = None
     if n_gla:
         hg = (n_swa + n_dswa, H)
-        if gla_delta:
-            _, S = delta(q32, k32, v32, alpha, beta, scale_gla, heads=hg, out=o)
+        if gla_delta:  # 1: the page's delta rule; 2: its decayed-erase form
+            _, S = delta(q32, k32, v32, alpha, beta, scale_gla, heads=hg, out=o,
+                         erase_decayed=int(gla_delta) == 2)
         else:
             _, S = gla(q32, k32, v32, alpha, scale_gla, heads=hg, out=o)
     return o, S

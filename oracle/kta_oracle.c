@@ -179,11 +179,15 @@ int oracle_gla(const float* q, const float* k, const float* v, const float* alph
  *   v_new = beta_t v_t + (1 - beta_t) v_old
  *   M_t   = alpha_t M_{t-1} - v_old k_t^T + v_new k_t^T
  *   o_t   = scale * M_t q_t
- * alpha_t and beta_t are scalars per token and head. */
+ * alpha_t and beta_t are scalars per token and head. erase_decayed selects the other reading of
+ * the same paragraph, which says the branch is based on GatedDeltaNet: GatedDeltaNet's own update
+ * decays the erase term too,
+ *   M_t   = alpha_t M_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ * i.e. alpha_t (M_{t-1} - beta_t v_old k_t^T) + beta_t v_t k_t^T. */
 int oracle_delta(const float* q, const float* k, const float* v,
                  const float* alpha, const float* beta, const double* S0,
                  double* o, double* S_out,
-                 int B, int N, int H, int d, int h0, int h1, double scale) {
+                 int B, int N, int H, int d, int h0, int h1, double scale, int erase_decayed) {
     if (B < 1 || N < 0 || H < 1 || d < 1 || h0 < 0 || h1 > H || h0 >= h1) return 1;
     int64_t nh = h1 - h0;
     int nt = oracle_get_threads();
@@ -206,10 +210,21 @@ int oracle_delta(const float* q, const float* k, const float* v,
                 for (int64_t i = 0; i < d; ++i) acc += S[i * d + j] * (double)kt[i];
                 vold[j] = acc;
             }
-            for (int64_t j = 0; j < d; ++j) vnew[j] = be * (double)vt[j] + (1.0 - be) * vold[j];
-            for (int64_t i = 0; i < d; ++i)
-                for (int64_t j = 0; j < d; ++j)
-                    S[i * d + j] = a * S[i * d + j] - vold[j] * (double)kt[i] + vnew[j] * (double)kt[i];
+            if (!erase_decayed) {
+                /* the page's four lines: v_new = beta v + (1 - beta) v_old,
+                   M = alpha M - v_old k^T + v_new k^T */
+                for (int64_t j = 0; j < d; ++j) vnew[j] = be * (double)vt[j] + (1.0 - be) * vold[j];
+                for (int64_t i = 0; i < d; ++i)
+                    for (int64_t j = 0; j < d; ++j)
+                        S[i * d + j] = a * S[i * d + j] - vold[j] * (double)kt[i] + vnew[j] * (double)kt[i];
+            } else {
+                /* decayed erase (the GatedDeltaNet form): M = alpha M (I - beta k k^T) + beta v k^T,
+                   where M k = v_old is read from the undecayed state */
+                for (int64_t i = 0; i < d; ++i)
+                    for (int64_t j = 0; j < d; ++j)
+                        S[i * d + j] = a * (S[i * d + j] - be * vold[j] * (double)kt[i])
+                                       + be * (double)vt[j] * (double)kt[i];
+            }
             double* ot = o + IDX4(b, t, h, 0, N, H, d);
             for (int64_t j = 0; j < d; ++j) {
                 double acc = 0.0;

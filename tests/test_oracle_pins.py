@@ -104,12 +104,14 @@ def delta_standard_form(q, k, v, a, be, scale, M0=None):
     return o, M
 
 
-def delta_chunked(q, k, v, a, be, scale, C, M0=None):
+def delta_chunked(q, k, v, a, be, scale, C, M0=None, decayed=False):
     """Chunked (UT / triangular-solve) form of the page's delta rule, derived by unrolling the
     recurrence inside a chunk:  gamma_t = prod_{r<=t} a_r,
        (I + T) U = diag(be) V - diag(be * gamma_{t-1}) K M0^T,  T_ts = be_t g_{t-1}/g_s (k_t.k_s)
        o_t = gamma_t M0 q_t + sum_{s<=t} gamma_t/gamma_s (q_t.k_s) u_s
-       M_C = gamma_C M0 + sum_s gamma_C/gamma_s u_s k_s^T."""
+       M_C = gamma_C M0 + sum_s gamma_C/gamma_s u_s k_s^T.
+    With the decayed erase (u_t = be_t (v_t - a_t M_{t-1} k_t)) every gamma_{t-1} above becomes
+    gamma_t."""
     q, k, v, a, be = (x.astype(np.float64) for x in (q, k, v, a, be))
     N, d = q.shape
     M = np.zeros((d, d)) if M0 is None else M0.copy()
@@ -119,7 +121,7 @@ def delta_chunked(q, k, v, a, be, scale, C, M0=None):
         Q, K, V, A, Bt = q[sl], k[sl], v[sl], a[sl], be[sl]
         n = Q.shape[0]
         g = np.cumprod(A)
-        gprev = np.concatenate([[1.0], g[:-1]])
+        gprev = g.copy() if decayed else np.concatenate([[1.0], g[:-1]])
         T = np.zeros((n, n))
         for t in range(n):
             for s in range(t):
@@ -193,6 +195,71 @@ def test_delta_exact_associative_recall():
     assert relerr(M @ kk.T, v[0, :, 0].astype(np.float64).T) < 1e-5
     # o_t = M_t q_t with q_t = k_t reads back the value just written
     assert relerr(o[0, :, 0], v[0, :, 0].astype(np.float64)) < 1e-5
+
+
+# ----------------------------------------------------------------------------- delta, decayed erase
+
+
+def pow2_gates(*shape):
+    """Forget gates that are powers of two, so that v / alpha and alpha * beta are exact."""
+    return RNG.choice(np.array([1.0, 0.5, 0.25], np.float32), size=shape)
+
+
+def test_decayed_erase_equals_page_form_with_rescaled_inputs():
+    # alpha M (I - b k k^T) + b v k^T = alpha M + (alpha b) ((v / alpha) - M k) k^T
+    B, N, H, d = 2, 29, 2, 5
+    q, v = rnd(B, N, H, d), rnd(B, N, H, d)
+    k = rnd(B, N, H, d)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    a, be = pow2_gates(B, N, H), gates(B, N, H, lo=0.05, hi=0.95)
+    M0 = RNG.standard_normal((B, H, d, d))
+    o, S = oracle.delta(q, k, v, a, be, scale=0.7, S0=M0, erase_decayed=True)
+    o2, S2 = oracle.delta(q, k, v / a[..., None], a, a * be, scale=0.7, S0=M0)
+    assert relerr(o, o2) < 1e-12
+    assert relerr(S, S2) < 1e-12
+
+
+def test_decayed_erase_equals_gated_deltanet_standard_form():
+    B, N, H, d = 1, 31, 1, 6
+    q, v = rnd(B, N, H, d), rnd(B, N, H, d)
+    k = rnd(B, N, H, d)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    a, be = pow2_gates(B, N, H), gates(B, N, H, lo=0.05, hi=0.95)
+    M0 = RNG.standard_normal((B, H, d, d))
+    o, S = oracle.delta(q, k, v, a, be, scale=1.0, S0=M0, erase_decayed=True)
+    # delta_standard_form(a, b', v') runs M = a M (I - (b'/a) k k^T) + (b'/a)(a v') k^T
+    ref, Mref = delta_standard_form(q[0, :, 0], k[0, :, 0], v[0, :, 0] / a[0, :, 0, None],
+                                    a[0, :, 0], a[0, :, 0] * be[0, :, 0], 1.0, M0[0, 0].T)
+    assert relerr(o[0, :, 0], ref) < 1e-11
+    assert relerr(S[0, 0].T, Mref) < 1e-11
+
+
+def test_decayed_erase_with_unit_gate_is_the_page_form():
+    B, N, H, d = 1, 25, 1, 6
+    q, k, v = rnd(B, N, H, d), rnd(B, N, H, d), rnd(B, N, H, d)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    ones, be = np.ones((B, N, H), np.float32), gates(B, N, H, lo=0.05, hi=0.95)
+    o1, S1 = oracle.delta(q, k, v, ones, be, erase_decayed=True)
+    o2, S2 = oracle.delta(q, k, v, ones, be)
+    assert relerr(o1, o2) < 1e-13 and relerr(S1, S2) < 1e-13
+
+
+@pytest.mark.parametrize("C", [1, 8, 64])
+def test_decayed_erase_equals_its_chunked_ut_form(C):
+    B, N, H, d = 1, 70, 1, 8
+    q, v = rnd(B, N, H, d), rnd(B, N, H, d)
+    k = rnd(B, N, H, d)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    a, be = gates(B, N, H, lo=0.6), gates(B, N, H, lo=0.05, hi=0.95)
+    M0 = RNG.standard_normal((B, H, d, d))
+    o, S = oracle.delta(q, k, v, a, be, scale=1.0, S0=M0, erase_decayed=True)
+    ref, Mref = delta_chunked(q[0, :, 0], k[0, :, 0], v[0, :, 0], a[0, :, 0], be[0, :, 0], 1.0,
+                              C, M0[0, 0].T, decayed=True)
+    assert relerr(o[0, :, 0], ref) < 1e-10
+    assert relerr(S[0, 0].T, Mref) < 1e-10
+    # and the two forms really differ when alpha < 1
+    o_page, _ = oracle.delta(q, k, v, a, be, scale=1.0, S0=M0)
+    assert relerr(o_page, o) > 1e-3
 
 
 # ----------------------------------------------------------------------------- softmax branches
