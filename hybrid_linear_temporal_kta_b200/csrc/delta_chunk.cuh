@@ -7,6 +7,10 @@
 // and row vectors this is  u_t = beta_t (v_t - k_t S_{t-1}),  S_t = alpha_t S_{t-1} + k_t^T u_t,
 // o_t = scale * q_t S_t.
 //
+// The decayed-erase reading (GatedDeltaNet's own update, the branch the page says it is based on)
+// is u_t = beta_t (v_t - alpha_t k_t S_{t-1}); it changes only gamma_{t-1} -> gamma_t in T and W
+// below (erase_decayed).
+//
 // Chunked form (derived by unrolling inside a chunk of C tokens; gamma_t = prod_{r<=t} alpha_r,
 // gamma_{-1} = 1, S_0 the state at the chunk start, A = (I + T)^{-1} with the strictly lower
 // triangular T_ts = beta_t (gamma_{t-1} / gamma_s) (k_t . k_s)):
@@ -50,6 +54,7 @@ struct DeltaParams {
   const float* S0;        // [B][H][D][D] key-major, or null
   float* S_out;           // or null
   int nch;                // chunks per sequence
+  int erase_decayed;      // 1: decayed erase (GatedDeltaNet form): gamma_{t-1} -> gamma_t in T, W
   __nv_bfloat16* ws_W;    // [B*H][nch][C][D]
   __nv_bfloat16* ws_U;    // [B*H][nch][D][C]   (U'^T)
   __nv_bfloat16* ws_A;    // [B*H][nch][C][C]
@@ -161,7 +166,8 @@ __global__ void __launch_bounds__(128, 3) delta_prep_kernel(const DeltaParams p)
         const int t = r0 + g4 + (r >= 2 ? 8 : 0);
         const int s = nt * 8 + 2 * t4 + (r & 1);
         const float lgt = sm.lg[t], lgs = sm.lg[s];
-        const float lgp = t > 0 ? sm.lg[t - 1] : 0.f;
+        // the erase term sees gamma_{t-1} (page form) or gamma_t (decayed erase)
+        const float lgp = p.erase_decayed ? lgt : (t > 0 ? sm.lg[t - 1] : 0.f);
         const float tv = s < t ? sm.beta[t] * exp2f(lgp - lgs) * kk_acc[nt][r] : 0.f;
         const float av = s <= t ? exp2f(lgt - lgs) * qk_acc[nt][r] : 0.f;
         sm.tf[t * LDT + s] = tv;
@@ -208,8 +214,9 @@ __global__ void __launch_bounds__(128, 3) delta_prep_kernel(const DeltaParams p)
 #pragma unroll 1
     for (int i = 0; i < C / 16; ++i) {
       const int ta = i * 16 + g4, tb = ta + 8;
-      const float fa = kside ? sm.beta[ta] * (ta > 0 ? exp2f(sm.lg[ta - 1]) : 1.f) : sm.beta[ta];
-      const float fb = kside ? sm.beta[tb] * exp2f(sm.lg[tb - 1]) : sm.beta[tb];
+      const int pa = p.erase_decayed ? ta : ta - 1, pb = p.erase_decayed ? tb : tb - 1;
+      const float fa = kside ? sm.beta[ta] * (pa >= 0 ? exp2f(sm.lg[pa]) : 1.f) : sm.beta[ta];
+      const float fb = kside ? sm.beta[tb] * exp2f(sm.lg[pb]) : sm.beta[tb];
       float acc[NTW][4];
 #pragma unroll
       for (int nt = 0; nt < NTW; ++nt) {

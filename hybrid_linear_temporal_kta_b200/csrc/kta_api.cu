@@ -358,6 +358,7 @@ struct LinLaunch {
   float* S_out = nullptr;
   float scale = 1.f;
   bool delta = false;
+  bool erase_decayed = false;  // delta rule: decayed erase (GatedDeltaNet form)
   bool allow_segments = true;
 };
 
@@ -450,6 +451,7 @@ kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
   p.S0 = L.S0;
   p.S_out = L.S_out;
   p.nch = static_cast<int>(nch);
+  p.erase_decayed = L.erase_decayed ? 1 : 0;
   const size_t units = static_cast<size_t>(BH) * nch;
   const size_t bytes = units * (static_cast<size_t>(C) * D * 2 * 2 + C * C * 2 + C * 4);
   void* ws = nullptr;
@@ -515,6 +517,7 @@ kta_status launch_rec_f32(const LinLaunch& L, cudaStream_t st) {
   p.scale = L.scale;
   p.S0 = L.S0;
   p.S_out = L.S_out;
+  p.erase_decayed = L.erase_decayed ? 1 : 0;
   if (L.B > 65535) return fail(KTA_ERR_UNSUPPORTED, "B > 65535");
   dim3 grid(L.H, L.B);
   TraceScope ts(L.delta ? "delta_rec_f32" : "gla_rec_f32", st);
@@ -678,7 +681,7 @@ kta_status kta_dswa_fwd(const void* q, const void* k, const void* v, void* o, kt
 static kta_status lin_common(const void* q, const void* k, const void* v, const float* alpha,
                              const float* beta, const float* S0, float* S_out, void* o,
                              kta_shape s, int H, int ld_heads, int chunk, float scale, bool delta,
-                             void* stream) {
+                             bool erase_decayed, void* stream) {
   kta_status r;
   if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) || (r = check_ptrs({q, k, v, o})))
     return r;
@@ -707,6 +710,7 @@ static kta_status lin_common(const void* q, const void* k, const void* v, const 
   L.S_out = S_out;
   L.scale = scale;
   L.delta = delta;
+  L.erase_decayed = erase_decayed;
   return launch_lin(L, as_stream(stream));
 }
 
@@ -714,14 +718,23 @@ kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const 
                              const float* S0, float* S_out, void* o, kta_shape s, int H,
                              int ld_heads, int chunk, float scale, void* stream) {
   return lin_common(q, k, v, alpha, nullptr, S0, S_out, o, s, H, ld_heads, chunk, scale, false,
-                    stream);
+                    false, stream);
 }
 
 kta_status kta_gla_delta_fwd(const void* q, const void* k, const void* v, const float* alpha,
                              const float* beta, const float* S0, float* S_out, void* o,
                              kta_shape s, int H, int ld_heads, int chunk, float scale,
                              void* stream) {
-  return lin_common(q, k, v, alpha, beta, S0, S_out, o, s, H, ld_heads, chunk, scale, true, stream);
+  return lin_common(q, k, v, alpha, beta, S0, S_out, o, s, H, ld_heads, chunk, scale, true, false,
+                    stream);
+}
+
+kta_status kta_gla_gdn_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                           const float* beta, const float* S0, float* S_out, void* o,
+                           kta_shape s, int H, int ld_heads, int chunk, float scale,
+                           void* stream) {
+  return lin_common(q, k, v, alpha, beta, S0, S_out, o, s, H, ld_heads, chunk, scale, true, true,
+                    stream);
 }
 
 static kta_status check_cfg(const kta_hybrid_cfg* c) {
@@ -738,6 +751,8 @@ static kta_status check_cfg(const kta_hybrid_cfg* c) {
       return fail(KTA_ERR_INVALID_ARG, "scale_softmax must be > 0");
   }
   if (c->n_gla > 0) {
+    if (c->gla_delta < 0 || c->gla_delta > 2)
+      return fail(KTA_ERR_INVALID_ARG, "gla_delta must be 0, 1 or 2");
     if (c->chunk != 16 && c->chunk != 32 && c->chunk != 64)
       return fail(KTA_ERR_INVALID_ARG, "chunk must be 16, 32 or 64");
     if (!std::isfinite(c->scale_gla)) return fail(KTA_ERR_INVALID_ARG, "scale_gla must be finite");
@@ -786,6 +801,7 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
   L.beta = beta;
   L.scale = cfg->scale_gla;
   L.delta = cfg->gla_delta != 0;
+  L.erase_decayed = cfg->gla_delta == 2;
 
   const bool both = (cfg->n_swa + cfg->n_dswa) > 0 && cfg->n_gla > 0;
   if (!both) {
@@ -1013,6 +1029,7 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
     L.S_out = reinterpret_cast<float*>(s->arena + s->off_state[1 - s->cur]);
     L.scale = c.scale_gla;
     L.delta = c.gla_delta != 0;
+    L.erase_decayed = c.gla_delta == 2;
     if ((r = launch_lin(L, st))) return r;
     s->cur = 1 - s->cur;
   }

@@ -95,6 +95,7 @@ struct RecF32Params {
   float scale;
   const float* S0;       // [B][H][d][d] key-major or null
   float* S_out;          // [B][H][d][d] or null
+  int erase_decayed;     // delta rule: 1 = decayed erase (GatedDeltaNet form)
 };
 
 // Vector-gated GLA, token by token. One CTA per (b, h); thread j owns column j of S (all key
@@ -165,10 +166,19 @@ __global__ void __launch_bounds__(D) delta_rec_f32_kernel(const float* __restric
     for (int i = 0; i < D; ++i) vold = fmaf(S[i], ks[i], vold);
     const float vnew = be * vj + (1.f - be) * vold;
     float acc = 0.f;
+    if (p.erase_decayed) {
+      // S = alpha (S - beta v_old k^T) + beta v k^T
 #pragma unroll
-    for (int i = 0; i < D; ++i) {
-      S[i] = a * S[i] - vold * ks[i] + vnew * ks[i];
-      acc = fmaf(S[i], qs[i], acc);
+      for (int i = 0; i < D; ++i) {
+        S[i] = a * (S[i] - be * vold * ks[i]) + be * vj * ks[i];
+        acc = fmaf(S[i], qs[i], acc);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < D; ++i) {
+        S[i] = a * S[i] - vold * ks[i] + vnew * ks[i];
+        acc = fmaf(S[i], qs[i], acc);
+      }
     }
     o[row * p.ld + h * D + j] = acc * p.scale;
     __syncthreads();

@@ -50,6 +50,8 @@ _SIGS = {
     "kta_gla_chunk_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp], _st),
     "kta_gla_delta_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
                           _st),
+    "kta_gla_gdn_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
+                        _st),
     "kta_gla_chunk_fwd_noalloc": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
                                   _st),
     "kta_hybrid_fwd": ([ctypes.POINTER(HybridCfg), _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
@@ -144,7 +146,8 @@ def dswa_fwd(q, k, v, *, P: int, W: int, dil: int, scale: float | None = None, h
     return _softmax(_lib.kta_dswa_fwd, q, k, v, P, W, dil, scale, heads, out, stream)
 
 
-def _linear(delta, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream):
+def _linear(delta, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream,
+            erase_decayed=False):
     for n, t in (("q", q), ("k", k), ("v", v)):
         _need(t, n, q.dtype)
     _need(alpha, "alpha", torch.float32)
@@ -160,9 +163,9 @@ def _linear(delta, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, 
     S_out = torch.empty((B, H, d, d), device=q.device, dtype=torch.float32) if return_state else None
     s = Shape(B, 1, N, d, _DT[q.dtype])  # one frame of N tokens: the linear branches ignore frames
     if delta:
-        st = _lib.kta_gla_delta_fwd(_ptr(q, h0 * d), _ptr(k, h0 * d), _ptr(v, h0 * d), _ptr(alpha),
-                                    _ptr(beta), _ptr(S0), _ptr(S_out), _ptr(o, h0 * d), s, H, Htot,
-                                    chunk, scale, _stream(stream))
+        fn = _lib.kta_gla_gdn_fwd if erase_decayed else _lib.kta_gla_delta_fwd
+        st = fn(_ptr(q, h0 * d), _ptr(k, h0 * d), _ptr(v, h0 * d), _ptr(alpha), _ptr(beta),
+                _ptr(S0), _ptr(S_out), _ptr(o, h0 * d), s, H, Htot, chunk, scale, _stream(stream))
     else:
         st = _lib.kta_gla_chunk_fwd(_ptr(q, h0 * d), _ptr(k, h0 * d), _ptr(v, h0 * d), _ptr(alpha),
                                     _ptr(S0), _ptr(S_out), _ptr(o, h0 * d), s, H, Htot, chunk,
@@ -178,14 +181,17 @@ def gla_chunk_fwd(q, k, v, alpha, *, chunk: int = 64, scale: float = 1.0, S0=Non
 
 
 def gla_delta_fwd(q, k, v, alpha, beta, *, chunk: int = 64, scale: float = 1.0, S0=None,
-                  return_state: bool = False, heads=None, out=None, stream=None):
-    """Gated delta rule; alpha, beta [B, N, H] fp32. Returns o (and the final state)."""
-    return _linear(True, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream)
+                  return_state: bool = False, heads=None, out=None, stream=None,
+                  erase_decayed: bool = False):
+    """Gated delta rule; alpha, beta [B, N, H] fp32. Returns o (and the final state).
+    erase_decayed: the GatedDeltaNet form M = alpha M (I - beta k k^T) + beta v k^T."""
+    return _linear(True, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream,
+                   erase_decayed)
 
 
 def hybrid_cfg(*, B: int, F: int, P: int, d: int, dtype=torch.bfloat16, n_swa: int, n_dswa: int,
                n_gla: int, W_swa: int = 3, W_dswa: int = 4, dil: int = 3, chunk: int = 64,
-               gla_delta: bool = False, scale_softmax: float | None = None,
+               gla_delta: int = 0, scale_softmax: float | None = None,
                scale_gla: float = 1.0) -> HybridCfg:
     return HybridCfg(Shape(B, F, P, d, _DT[dtype]), n_swa, n_dswa, n_gla, W_swa, W_dswa, dil, chunk,
                      int(gla_delta), 1.0 / math.sqrt(d) if scale_softmax is None else scale_softmax,

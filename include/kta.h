@@ -149,10 +149,24 @@ kta_status kta_gla_delta_fwd(const void* q, const void* k, const void* v, const 
                              void* stream);
 
 /*
+ * Gated delta rule with the erase term decayed too -- the GatedDeltaNet update, which the
+ * paper-read's GLA paragraph names as the branch's basis:
+ *     M_t = alpha_t M_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = scale * M_t q_t
+ * (the page's four lines keep v_old k^T undecayed). It equals kta_gla_delta_fwd with beta
+ * replaced by alpha * beta and v by v / alpha. Same arguments, layouts and errors as
+ * kta_gla_delta_fwd.
+ */
+kta_status kta_gla_gdn_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                           const float* beta, const float* S0, float* S_out, void* o,
+                           kta_shape s, int H, int ld_heads, int chunk, float scale,
+                           void* stream);
+
+/*
  * Hybrid layer. The pages say only that the three branches' outputs form one mixed temporal
  * representation; this ABI splits heads: heads [0, n_swa) are SWA (window W_swa), the next
  * n_dswa heads DSWA (window W_dswa, dilation dil), the last n_gla heads GLA (vector gate) or,
- * with gla_delta = 1, the gated delta rule. Outputs are concatenated by head in o.
+ * with gla_delta = 1, the gated delta rule (the page's form), with gla_delta = 2 its decayed-erase
+ * form (kta_gla_gdn_fwd). Outputs are concatenated by head in o.
  * q, k, v, o: [B][N][H][d] with H = n_swa + n_dswa + n_gla. alpha: [B][N][n_gla][d] (vector
  * GLA) or [B][N][n_gla] (delta); beta: [B][N][n_gla] (delta only, else ignored).
  * The softmax and GLA branches run concurrently on internal streams forked from `stream` and
@@ -163,7 +177,7 @@ typedef struct {
   int n_swa, n_dswa, n_gla;
   int W_swa, W_dswa, dil;
   int chunk;
-  int gla_delta;
+  int gla_delta;            /* 0: vector-gated GLA, 1: delta rule, 2: decayed-erase delta rule */
   float scale_softmax, scale_gla;
 } kta_hybrid_cfg;
 

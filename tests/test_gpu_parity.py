@@ -78,6 +78,12 @@ def test_f32_linear_branches_with_state(kta, d):
     ref, Sref = oracle.delta(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], S0=S0)
     assert_heads_close(o, ref, range(H), F32_TOL, what="f32 delta")
     assert rel(S.cpu().numpy(), Sref) < F32_TOL
+    o, S = kta.gla_delta_fwd(dev(xd["q"]), dev(xd["k"]), dev(xd["v"]), dev(xd["alpha"]),
+                             dev(xd["beta"]), S0=dev(S0), return_state=True, erase_decayed=True)
+    ref, Sref = oracle.delta(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], S0=S0,
+                             erase_decayed=True)
+    assert_heads_close(o, ref, range(H), F32_TOL, what="f32 decayed-erase delta")
+    assert rel(S.cpu().numpy(), Sref) < F32_TOL
 
 
 @pytest.mark.parametrize("W,dil", [(1, 1), (2, 1), (3, 2), (9, 1)])
@@ -205,6 +211,22 @@ def test_bf16_delta_matches_oracle(kta, d, N, B, H, with_s0):
     assert rel(S.cpu().numpy(), Sref) < BF16_TOL
 
 
+@pytest.mark.parametrize("d,N,B,H,with_s0", [(128, 300, 2, 2, True), (64, 1000, 1, 3, False),
+                                             (128, 50, 1, 1, True), (128, 4096, 1, 1, False)])
+def test_bf16_decayed_erase_delta_matches_oracle(kta, d, N, B, H, with_s0):
+    w = synth.DELTA_BF16.replace(d=d, n_gla=H)
+    x = synth.make_inputs(w, N=N, B=B)
+    S0 = (torch.from_numpy(np.random.default_rng(6).standard_normal((B, H, d, d)).astype(np.float32))
+          * 0.1 if with_s0 else None)
+    o, S = kta.gla_delta_fwd(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["alpha"]),
+                             dev(x["beta"]), S0=dev(S0), return_state=True, erase_decayed=True)
+    kta.device_status()
+    ref, Sref = oracle.delta(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S0=S0,
+                             erase_decayed=True)
+    assert_heads_close(o, ref, range(H), BF16_TOL, what=f"decayed-erase delta d={d} N={N}")
+    assert rel(S.cpu().numpy(), Sref) < BF16_TOL
+
+
 # --------------------------------------------------------------------------- hybrid
 
 
@@ -228,6 +250,17 @@ def test_bf16_hybrid_delta_heads(kta):
                            n_dswa=1, n_gla=2, W_swa=w.W_swa, W_dswa=w.W_dswa, dil=w.dil,
                            gla_delta=True, scale_softmax=w.scale_softmax)
     assert_heads_close(o, ref, range(w.H), BF16_TOL, what="hybrid delta")
+
+
+def test_bf16_hybrid_decayed_erase_delta_heads(kta):
+    w = synth.HYBRID_BF16.replace(F=5, P=180, n_swa=1, n_dswa=1, n_gla=2, gla_delta=2)
+    x = synth.make_inputs(w)
+    o = kta.hybrid_fwd(kta.cfg_from_workload(w), dev(x["q"]), dev(x["k"]), dev(x["v"]),
+                       dev(x["alpha"]), dev(x["beta"]))
+    ref, _ = oracle.hybrid(x["q"], x["k"], x["v"], x["alpha"], x["beta"], P=w.P, n_swa=1,
+                           n_dswa=1, n_gla=2, W_swa=w.W_swa, W_dswa=w.W_dswa, dil=w.dil,
+                           gla_delta=2, scale_softmax=w.scale_softmax)
+    assert_heads_close(o, ref, range(w.H), BF16_TOL, what="hybrid decayed-erase delta")
 
 
 @pytest.mark.slow
@@ -270,6 +303,30 @@ def _stream_case(dtype="bf16"):
     w = synth.STREAM_BF16.replace(F=9, P=200, n_swa=2, n_dswa=2, n_gla=2, dtype=dtype,
                                   d=128 if dtype == "bf16" else 64)
     return w, synth.make_inputs(w, B=2)
+
+
+@pytest.mark.parametrize("gla_delta", [1, 2])
+def test_stream_rollout_with_delta_heads(kta, gla_delta):
+    w = synth.STREAM_BF16.replace(F=7, P=150, n_swa=1, n_dswa=1, n_gla=2, gla_delta=gla_delta)
+    x = synth.make_inputs(w, B=2)
+    cfg = kta.cfg_from_workload(w, B=2)
+    q, k, v, a, be = (dev(x[n]) for n in ("q", "k", "v", "alpha", "beta"))
+    full = kta.hybrid_fwd(cfg, q, k, v, a, be)
+    st = kta.Stream(cfg)
+    outs = []
+    for f in range(w.F):
+        sl = slice(f * w.P, (f + 1) * w.P)
+        outs.append(st.step(q[:, sl].contiguous(), k[:, sl].contiguous(), v[:, sl].contiguous(),
+                            a[:, sl].contiguous(), be[:, sl].contiguous()))
+    kta.device_status()
+    roll = torch.cat(outs, dim=1)
+    assert_heads_close(roll, full.float().cpu().numpy().astype(np.float64), range(w.H), BF16_TOL,
+                       what="delta stream vs full")
+    ref, _ = oracle.hybrid(x["q"], x["k"], x["v"], x["alpha"], x["beta"], P=w.P, n_swa=1,
+                           n_dswa=1, n_gla=2, W_swa=w.W_swa, W_dswa=w.W_dswa, dil=w.dil,
+                           gla_delta=gla_delta, scale_softmax=w.scale_softmax)
+    assert_heads_close(roll, ref, range(w.H), BF16_TOL, what="delta stream vs oracle")
+    st.close()
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
