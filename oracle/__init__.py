@@ -69,9 +69,17 @@ def _load():
                                          _f64p] + [_int] * 6 + [ctypes.c_double, _int]
             lib.oracle_visible.argtypes = [_i64p, _i64p, ctypes.c_int64, _int, _int, _int, _int,
                                            _u8p]
+            lib.oracle_softmax_bwd.argtypes = [_f32p, _f32p, _f32p, _f64p, _f64p, _f64p, _f64p] + [
+                _int] * 10 + [ctypes.c_double]
+            lib.oracle_gla_bwd.argtypes = [_f32p, _f32p, _f32p, _f32p, _f64p, _f64p, _f64p, _f64p,
+                                           _f64p, _f64p, _f64p] + [_int] * 6 + [ctypes.c_double]
+            lib.oracle_delta_bwd.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p,
+                                             _f64p, _f64p, _f64p, _f64p, _f64p, _f64p] + [
+                _int] * 6 + [ctypes.c_double, _int]
             lib.oracle_set_threads.argtypes = [_int]
             lib.oracle_get_threads.restype = _int
-            for name in ("oracle_swa", "oracle_dswa", "oracle_gla", "oracle_delta"):
+            for name in ("oracle_swa", "oracle_dswa", "oracle_gla", "oracle_delta",
+                         "oracle_softmax_bwd", "oracle_gla_bwd", "oracle_delta_bwd"):
                 getattr(lib, name).restype = _int
             _lib = lib
     return _lib
@@ -214,6 +222,57 @@ def hybrid(q, k, v, alpha, beta, *, P: int, n_swa: int, n_dswa: int, n_gla: int,
         else:
             _, S = gla(q32, k32, v32, alpha, scale_gla, heads=hg, out=o)
     return o, S
+
+
+def softmax_bwd(q, k, v, dout, P: int, W: int, scale: float, dil: int = 1,
+                dilated: bool = False, heads=None):
+    """Reverse mode of swa (dilated=False) / dswa: the gradients (dq, dk, dv) of
+    L = sum(dout * o) for the heads (h0, h1); other heads are zero. float64 [B, N, H, d]."""
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f64(dout)
+    B, N, H, d = q.shape
+    h0, h1 = heads if heads is not None else (0, H)
+    dq, dk, dv = (np.zeros((B, N, H, d)) for _ in range(3))
+    rc = _load().oracle_softmax_bwd(_p(q, _f32p), _p(k, _f32p), _p(v, _f32p), _p(do, _f64p),
+                                    _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p), B, N, H, d, h0,
+                                    h1, P, W, dil, int(bool(dilated)), float(scale))
+    _check(rc, "softmax_bwd")
+    return dq, dk, dv
+
+
+def gla_bwd(q, k, v, alpha, dout, scale: float = 1.0, S0=None, heads=None):
+    """Reverse mode of gla: (dq, dk, dv, dalpha, dS0) of L = sum(dout * o)."""
+    q, k, v, a, do = _f32(q), _f32(k), _f32(v), _f32(alpha), _f64(dout)
+    B, N, H, d = q.shape
+    h0, h1 = heads if heads is not None else (0, H)
+    dq, dk, dv = (np.zeros((B, N, H, d)) for _ in range(3))
+    da = np.zeros((B, N, h1 - h0, d))
+    dS0 = np.zeros((B, h1 - h0, d, d))
+    s0 = None if S0 is None else _f64(S0)
+    rc = _load().oracle_gla_bwd(_p(q, _f32p), _p(k, _f32p), _p(v, _f32p), _p(a, _f32p),
+                                None if s0 is None else _p(s0, _f64p), _p(do, _f64p),
+                                _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p), _p(da, _f64p),
+                                _p(dS0, _f64p), B, N, H, d, h0, h1, float(scale))
+    _check(rc, "gla_bwd")
+    return dq, dk, dv, da, dS0
+
+
+def delta_bwd(q, k, v, alpha, beta, dout, scale: float = 1.0, S0=None, heads=None,
+              erase_decayed: bool = False):
+    """Reverse mode of delta: (dq, dk, dv, dalpha, dbeta, dS0) of L = sum(dout * o)."""
+    q, k, v, a, be, do = _f32(q), _f32(k), _f32(v), _f32(alpha), _f32(beta), _f64(dout)
+    B, N, H, d = q.shape
+    h0, h1 = heads if heads is not None else (0, H)
+    dq, dk, dv = (np.zeros((B, N, H, d)) for _ in range(3))
+    da, db = np.zeros((B, N, h1 - h0)), np.zeros((B, N, h1 - h0))
+    dS0 = np.zeros((B, h1 - h0, d, d))
+    s0 = None if S0 is None else _f64(S0)
+    rc = _load().oracle_delta_bwd(_p(q, _f32p), _p(k, _f32p), _p(v, _f32p), _p(a, _f32p),
+                                  _p(be, _f32p), None if s0 is None else _p(s0, _f64p),
+                                  _p(do, _f64p), _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p),
+                                  _p(da, _f64p), _p(db, _f64p), _p(dS0, _f64p), B, N, H, d, h0,
+                                  h1, float(scale), int(bool(erase_decayed)))
+    _check(rc, "delta_bwd")
+    return dq, dk, dv, da, db, dS0
 
 
 def visible(t, s, P: int, W: int, dil: int = 1, dilated: bool = False) -> np.ndarray:

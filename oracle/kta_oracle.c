@@ -239,3 +239,253 @@ int oracle_delta(const float* q, const float* k, const float* v,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------------ backward
+ * Reverse mode of the operators above: given dO, the gradients of L = sum(dO * O) with respect
+ * to q, k, v and the gates, written out from the chain rule of each forward definition. Only the
+ * head range [h0, h1) of the gradient arrays is written (zeroed first). */
+
+static void zero_heads(double* x, int B, int N, int H, int d, int h0, int h1) {
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t t = 0; t < N; ++t)
+            memset(x + IDX4(b, t, h0, 0, N, H, d), 0, sizeof(double) * (size_t)(h1 - h0) * (size_t)d);
+}
+
+/* Softmax branches: with p_ts = softmax_s(scale q_t . k_s) over the visible keys and
+ * o_t = sum_s p_ts v_s: dp_ts = dO_t . v_s, ds_ts = p_ts (dp_ts - dO_t . o_t),
+ * dq_t = scale sum_s ds_ts k_s, dk_s = scale sum_t ds_ts q_t, dv_s = sum_t p_ts dO_t. */
+int oracle_softmax_bwd(const float* q, const float* k, const float* v, const double* dout,
+                       double* dq, double* dk, double* dv,
+                       int B, int N, int H, int d, int h0, int h1, int P, int W, int dil,
+                       int dilated, double scale) {
+    if (B < 1 || N < 0 || H < 1 || d < 1 || h0 < 0 || h1 > H || h0 >= h1 || P < 1 || W < 1 ||
+        dil < 1)
+        return 1;
+    zero_heads(dq, B, N, H, d, h0, h1);
+    zero_heads(dk, B, N, H, d, h0, h1);
+    zero_heads(dv, B, N, H, d, h0, h1);
+    int64_t nh = h1 - h0;
+    int nt = oracle_get_threads();
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+    for (int64_t w = 0; w < (int64_t)B * nh; ++w) {
+        int64_t b = w / nh, h = h0 + w % nh;
+        double* lg = (double*)malloc(sizeof(double) * (size_t)N);
+        double* o = (double*)malloc(sizeof(double) * (size_t)d);
+        for (int64_t t = 0; t < N; ++t) {
+            const float* qt = q + IDX4(b, t, h, 0, N, H, d);
+            const double* dot = dout + IDX4(b, t, h, 0, N, H, d);
+            double m = -INFINITY;
+            for (int64_t s = 0; s < N; ++s) {
+                int vis = dilated ? dswa_visible(t, s, P, W, dil) : swa_visible(t, s, P, W);
+                if (!vis) { lg[s] = -INFINITY; continue; }
+                const float* ks = k + IDX4(b, s, h, 0, N, H, d);
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += (double)qt[i] * (double)ks[i];
+                lg[s] = scale * acc;
+                if (lg[s] > m) m = lg[s];
+            }
+            double den = 0.0;
+            for (int64_t s = 0; s < N; ++s) {
+                lg[s] = lg[s] == -INFINITY ? 0.0 : exp(lg[s] - m);
+                den += lg[s];
+            }
+            for (int64_t j = 0; j < d; ++j) o[j] = 0.0;
+            for (int64_t s = 0; s < N; ++s) {
+                if (lg[s] == 0.0) continue;
+                lg[s] /= den;  /* p_ts */
+                const float* vs = v + IDX4(b, s, h, 0, N, H, d);
+                for (int64_t j = 0; j < d; ++j) o[j] += lg[s] * (double)vs[j];
+            }
+            double dD = 0.0;
+            for (int64_t j = 0; j < d; ++j) dD += dot[j] * o[j];
+            double* dqt = dq + IDX4(b, t, h, 0, N, H, d);
+            for (int64_t s = 0; s < N; ++s) {
+                if (lg[s] == 0.0) continue;
+                const float* ks = k + IDX4(b, s, h, 0, N, H, d);
+                const float* vs = v + IDX4(b, s, h, 0, N, H, d);
+                double dp = 0.0;
+                for (int64_t j = 0; j < d; ++j) dp += dot[j] * (double)vs[j];
+                double ds = lg[s] * (dp - dD);
+                double* dks = dk + IDX4(b, s, h, 0, N, H, d);
+                double* dvs = dv + IDX4(b, s, h, 0, N, H, d);
+                for (int64_t i = 0; i < d; ++i) {
+                    dqt[i] += scale * ds * (double)ks[i];
+                    dks[i] += scale * ds * (double)qt[i];
+                    dvs[i] += lg[s] * dot[i];
+                }
+            }
+        }
+        free(lg);
+        free(o);
+    }
+    return 0;
+}
+
+/* GLA (vector gate). With G_t = dL/dS_t = scale q_t^T dO_t + diag(alpha_{t+1}) G_{t+1}:
+ * dq_t = scale S_t dO_t^T, dk_t = G_t v_t^T, dv_t = k_t G_t, dalpha_t[i] = sum_j G_t[i][j]
+ * S_{t-1}[i][j], and dS_0 = diag(alpha_1) G_1. States are kept from a forward pass. */
+int oracle_gla_bwd(const float* q, const float* k, const float* v, const float* alpha,
+                   const double* S0, const double* dout, double* dq, double* dk, double* dv,
+                   double* dalpha, double* dS0, int B, int N, int H, int d, int h0, int h1,
+                   double scale) {
+    if (B < 1 || N < 0 || H < 1 || d < 1 || h0 < 0 || h1 > H || h0 >= h1) return 1;
+    zero_heads(dq, B, N, H, d, h0, h1);
+    zero_heads(dk, B, N, H, d, h0, h1);
+    zero_heads(dv, B, N, H, d, h0, h1);
+    int64_t nh = h1 - h0, dd = (int64_t)d * d;
+    int nt = oracle_get_threads();
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+    for (int64_t w = 0; w < (int64_t)B * nh; ++w) {
+        int64_t b = w / nh, hg = w % nh, h = h0 + hg;
+        double* S = (double*)malloc(sizeof(double) * (size_t)((N + 1) * dd));  /* S_0 .. S_N */
+        double* G = (double*)calloc((size_t)dd, sizeof(double));
+        if (S0) memcpy(S, S0 + w * dd, sizeof(double) * (size_t)dd);
+        else memset(S, 0, sizeof(double) * (size_t)dd);
+        for (int64_t t = 0; t < N; ++t) {
+            const float* kt = k + IDX4(b, t, h, 0, N, H, d);
+            const float* vt = v + IDX4(b, t, h, 0, N, H, d);
+            const float* at = alpha + IDX4(b, t, hg, 0, N, nh, d);
+            const double* Sp = S + t * dd;
+            double* Sn = S + (t + 1) * dd;
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j)
+                    Sn[i * d + j] = (double)at[i] * Sp[i * d + j] + (double)kt[i] * (double)vt[j];
+        }
+        for (int64_t t = N - 1; t >= 0; --t) {
+            const float* qt = q + IDX4(b, t, h, 0, N, H, d);
+            const float* kt = k + IDX4(b, t, h, 0, N, H, d);
+            const float* vt = v + IDX4(b, t, h, 0, N, H, d);
+            const float* at = alpha + IDX4(b, t, hg, 0, N, nh, d);
+            const double* dot = dout + IDX4(b, t, h, 0, N, H, d);
+            const double* St = S + (t + 1) * dd;
+            const double* Sp = S + t * dd;
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j) G[i * d + j] += scale * (double)qt[i] * dot[j];
+            double* dqt = dq + IDX4(b, t, h, 0, N, H, d);
+            double* dkt = dk + IDX4(b, t, h, 0, N, H, d);
+            double* dvt = dv + IDX4(b, t, h, 0, N, H, d);
+            double* dat = dalpha + IDX4(b, t, hg, 0, N, nh, d);
+            for (int64_t i = 0; i < d; ++i) {
+                double aq = 0.0, ak = 0.0, aa = 0.0;
+                for (int64_t j = 0; j < d; ++j) {
+                    aq += St[i * d + j] * dot[j];
+                    ak += G[i * d + j] * (double)vt[j];
+                    aa += G[i * d + j] * Sp[i * d + j];
+                }
+                dqt[i] = scale * aq;
+                dkt[i] = ak;
+                dat[i] = aa;
+            }
+            for (int64_t j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += (double)kt[i] * G[i * d + j];
+                dvt[j] = acc;
+            }
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j) G[i * d + j] *= (double)at[i];
+        }
+        if (dS0) memcpy(dS0 + w * dd, G, sizeof(double) * (size_t)dd);
+        free(S);
+        free(G);
+    }
+    return 0;
+}
+
+/* Gated delta rule (row convention: w_t = k_t S_{t-1}, u_t = beta_t (v_t - a_t w_t) with a_t = 1
+ * for the page's form and a_t = alpha_t for the decayed erase, S_t = alpha_t S_{t-1} + k_t^T u_t,
+ * o_t = scale q_t S_t). With G_t = dL/dS_t = scale q_t^T dO_t + [propagated from t+1] and
+ * du_t = k_t G_t:
+ *   dq_t = scale S_t dO_t^T,   dv_t = beta_t du_t,   dbeta_t = du_t . (v_t - a_t w_t),
+ *   dk_t = G_t u_t^T - beta_t a_t S_{t-1} du_t^T,
+ *   dalpha_t = <G_t, S_{t-1}> (- beta_t du_t . w_t for the decayed erase),
+ *   G_{t-1} = alpha_t G_t - beta_t a_t k_t^T du_t. */
+int oracle_delta_bwd(const float* q, const float* k, const float* v, const float* alpha,
+                     const float* beta, const double* S0, const double* dout, double* dq,
+                     double* dk, double* dv, double* dalpha, double* dbeta, double* dS0,
+                     int B, int N, int H, int d, int h0, int h1, double scale, int erase_decayed) {
+    if (B < 1 || N < 0 || H < 1 || d < 1 || h0 < 0 || h1 > H || h0 >= h1) return 1;
+    zero_heads(dq, B, N, H, d, h0, h1);
+    zero_heads(dk, B, N, H, d, h0, h1);
+    zero_heads(dv, B, N, H, d, h0, h1);
+    int64_t nh = h1 - h0, dd = (int64_t)d * d;
+    int nt = oracle_get_threads();
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+    for (int64_t w = 0; w < (int64_t)B * nh; ++w) {
+        int64_t b = w / nh, hg = w % nh, h = h0 + hg;
+        double* S = (double*)malloc(sizeof(double) * (size_t)((N + 1) * dd));
+        double* U = (double*)malloc(sizeof(double) * (size_t)(N * d + 1));
+        double* Wr = (double*)malloc(sizeof(double) * (size_t)(N * d + 1));
+        double* G = (double*)calloc((size_t)dd, sizeof(double));
+        double* du = (double*)malloc(sizeof(double) * (size_t)d);
+        if (S0) memcpy(S, S0 + w * dd, sizeof(double) * (size_t)dd);
+        else memset(S, 0, sizeof(double) * (size_t)dd);
+        for (int64_t t = 0; t < N; ++t) {
+            const float* kt = k + IDX4(b, t, h, 0, N, H, d);
+            const float* vt = v + IDX4(b, t, h, 0, N, H, d);
+            double a = (double)alpha[((int64_t)b * N + t) * nh + hg];
+            double be = (double)beta[((int64_t)b * N + t) * nh + hg];
+            double ae = erase_decayed ? a : 1.0;
+            const double* Sp = S + t * dd;
+            double* Sn = S + (t + 1) * dd;
+            for (int64_t j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += (double)kt[i] * Sp[i * d + j];
+                Wr[t * d + j] = acc;
+                U[t * d + j] = be * ((double)vt[j] - ae * acc);
+            }
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j)
+                    Sn[i * d + j] = a * Sp[i * d + j] + (double)kt[i] * U[t * d + j];
+        }
+        for (int64_t t = N - 1; t >= 0; --t) {
+            const float* qt = q + IDX4(b, t, h, 0, N, H, d);
+            const float* kt = k + IDX4(b, t, h, 0, N, H, d);
+            const float* vt = v + IDX4(b, t, h, 0, N, H, d);
+            const double* dot = dout + IDX4(b, t, h, 0, N, H, d);
+            double a = (double)alpha[((int64_t)b * N + t) * nh + hg];
+            double be = (double)beta[((int64_t)b * N + t) * nh + hg];
+            double ae = erase_decayed ? a : 1.0;
+            const double* St = S + (t + 1) * dd;
+            const double* Sp = S + t * dd;
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j) G[i * d + j] += scale * (double)qt[i] * dot[j];
+            for (int64_t j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += (double)kt[i] * G[i * d + j];
+                du[j] = acc;
+            }
+            double* dqt = dq + IDX4(b, t, h, 0, N, H, d);
+            double* dkt = dk + IDX4(b, t, h, 0, N, H, d);
+            double* dvt = dv + IDX4(b, t, h, 0, N, H, d);
+            double da = 0.0, db = 0.0;
+            for (int64_t i = 0; i < d; ++i) {
+                double aq = 0.0, ak = 0.0, as = 0.0;
+                for (int64_t j = 0; j < d; ++j) {
+                    aq += St[i * d + j] * dot[j];
+                    ak += G[i * d + j] * U[t * d + j];
+                    as += Sp[i * d + j] * du[j];
+                    da += G[i * d + j] * Sp[i * d + j];
+                }
+                dqt[i] = scale * aq;
+                dkt[i] = ak - be * ae * as;
+            }
+            for (int64_t j = 0; j < d; ++j) {
+                dvt[j] = be * du[j];
+                db += du[j] * ((double)vt[j] - ae * Wr[t * d + j]);
+                if (erase_decayed) da -= be * du[j] * Wr[t * d + j];
+            }
+            dalpha[((int64_t)b * N + t) * nh + hg] = da;
+            dbeta[((int64_t)b * N + t) * nh + hg] = db;
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < d; ++j)
+                    G[i * d + j] = a * G[i * d + j] - be * ae * (double)kt[i] * du[j];
+        }
+        if (dS0) memcpy(dS0 + w * dd, G, sizeof(double) * (size_t)dd);
+        free(S);
+        free(U);
+        free(Wr);
+        free(G);
+        free(du);
+    }
+    return 0;
+}
