@@ -21,6 +21,7 @@
 #include "simt_f32.cuh"
 #include "gla_chunk.cuh"
 #include "delta_chunk.cuh"
+#include "bwd_f32.cuh"
 
 namespace {
 
@@ -878,9 +879,148 @@ kta_status ring_put(const kta_stream_s* s, const void* src, char* ring, int h0, 
   return KTA_OK;
 }
 
+// ------------------------------------------------------------------------- backward (fp32)
+
+kta_status bwd_f32_only(const kta_shape& s) {
+  if (s.dtype != KTA_F32)
+    return fail(KTA_ERR_UNSUPPORTED, "the backward is built for KTA_F32 (fp32 reference) only");
+  return KTA_OK;
+}
+
+kta_status zero_heads_f32(void* x, long long rows, int Hd, long long ld, cudaStream_t st) {
+  const long long n = rows * Hd;
+  if (n == 0) return KTA_OK;
+  kta::zero_rows_f32_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      static_cast<float*>(x), rows, Hd, ld);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+kta_status softmax_bwd_common(const void* q, const void* k, const void* v,
+                                     const void* dout, void* dq, void* dk, void* dv, kta_shape s,
+                                     int H, int ld_heads, int W, int dil, float scale,
+                                     void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = bwd_f32_only(s)) || (r = check_heads(H, ld_heads, s)) ||
+      (r = check_ptrs({q, k, v, dout, dq, dk, dv})))
+    return r;
+  if (W < 1 || dil < 1) return fail(KTA_ERR_INVALID_ARG, "W and dil must be >= 1");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be > 0");
+  if (s.B > 65535 || H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B and H must be <= 65535");
+  cudaStream_t st = as_stream(stream);
+  const long long N = static_cast<long long>(s.F) * s.P, ld = static_cast<long long>(ld_heads) * s.d;
+  if ((r = zero_heads_f32(dk, s.B * N, H * s.d, ld, st)) ||
+      (r = zero_heads_f32(dv, s.B * N, H * s.d, ld, st)))
+    return r;
+  kta::SoftmaxBwdParams p{};
+  p.B = s.B;
+  p.N = static_cast<int>(N);
+  p.P = s.P;
+  p.H = H;
+  p.d = s.d;
+  p.W = W;
+  p.dil = dil;
+  p.ld = ld;
+  p.scale = scale;
+  TraceScope ts("softmax_bwd_f32", st);
+  kta::softmax_bwd_f32_kernel<<<dim3(static_cast<unsigned>((N + 3) / 4), H, s.B), 128, 0, st>>>(
+      static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+      static_cast<const float*>(dout), static_cast<float*>(dq), static_cast<float*>(dk),
+      static_cast<float*>(dv), p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+template <int D>
+kta_status launch_lin_bwd(kta::LinBwdParams p, int B, cudaStream_t st) {
+  const long long per = kta::lin_bwd_ws_floats<D>(p.nck);
+  void* ws = nullptr;
+  kta_status r = workspace(static_cast<size_t>(per) * B * p.H * sizeof(float), st, &ws);
+  if (r) return r;
+  p.ws = static_cast<float*>(ws);
+  const size_t smem = (static_cast<size_t>(D) * (D + 1) + 8 * D) * sizeof(float);
+  if ((r = set_smem_attr(kta::lin_bwd_f32_kernel<D>, smem))) return r;
+  TraceScope ts(p.delta ? "delta_bwd_f32" : "gla_bwd_f32", st);
+  kta::lin_bwd_f32_kernel<D><<<dim3(p.H, B), D, smem, st>>>(p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
+kta_status lin_bwd_common(const void* q, const void* k, const void* v, const float* alpha,
+                                 const float* beta, const float* S0, const void* dout, void* dq,
+                                 void* dk, void* dv, float* dalpha, float* dbeta, float* dS0,
+                                 kta_shape s, int H, int ld_heads, float scale, bool delta,
+                                 bool erase_decayed, void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = bwd_f32_only(s)) || (r = check_heads(H, ld_heads, s)) ||
+      (r = check_ptrs({q, k, v, dout, dq, dk, dv})))
+    return r;
+  if (!alpha || !dalpha || (delta && (!beta || !dbeta)))
+    return fail(KTA_ERR_INVALID_ARG, "null gate or gate-gradient pointer");
+  if (!std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be finite");
+  if (s.B > 65535 || H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B and H must be <= 65535");
+  const long long N = static_cast<long long>(s.F) * s.P;
+  kta::LinBwdParams p{};
+  p.q = static_cast<const float*>(q);
+  p.k = static_cast<const float*>(k);
+  p.v = static_cast<const float*>(v);
+  p.alpha = alpha;
+  p.beta = beta;
+  p.S0 = S0;
+  p.dout = static_cast<const float*>(dout);
+  p.dq = static_cast<float*>(dq);
+  p.dk = static_cast<float*>(dk);
+  p.dv = static_cast<float*>(dv);
+  p.dalpha = dalpha;
+  p.dbeta = dbeta;
+  p.dS0 = dS0;
+  p.ld = static_cast<long long>(ld_heads) * s.d;
+  p.rows_b = static_cast<int>(N);
+  p.N = static_cast<int>(N);
+  p.H = H;
+  p.scale = scale;
+  p.delta = delta ? 1 : 0;
+  p.erase_decayed = erase_decayed ? 1 : 0;
+  p.nck = static_cast<int>((N + kta::BWD_CK - 1) / kta::BWD_CK);
+  if (N == 0) return KTA_OK;
+  cudaStream_t st = as_stream(stream);
+  if (s.d == 32) return launch_lin_bwd<32>(p, s.B, st);
+  if (s.d == 64) return launch_lin_bwd<64>(p, s.B, st);
+  return launch_lin_bwd<128>(p, s.B, st);
+}
+
 }  // namespace
 
 extern "C" {
+
+kta_status kta_swa_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                       void* dk, void* dv, kta_shape s, int H, int ld_heads, int W, float scale,
+                       void* stream) {
+  return softmax_bwd_common(q, k, v, dout, dq, dk, dv, s, H, ld_heads, W, 1, scale, stream);
+}
+
+kta_status kta_dswa_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                        void* dk, void* dv, kta_shape s, int H, int ld_heads, int W, int dil,
+                        float scale, void* stream) {
+  return softmax_bwd_common(q, k, v, dout, dq, dk, dv, s, H, ld_heads, W, dil, scale, stream);
+}
+
+kta_status kta_gla_bwd(const void* q, const void* k, const void* v, const float* alpha,
+                       const float* S0, const void* dout, void* dq, void* dk, void* dv,
+                       float* dalpha, float* dS0, kta_shape s, int H, int ld_heads, float scale,
+                       void* stream) {
+  return lin_bwd_common(q, k, v, alpha, nullptr, S0, dout, dq, dk, dv, dalpha, nullptr, dS0, s, H,
+                        ld_heads, scale, false, false, stream);
+}
+
+kta_status kta_gla_delta_bwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, const void* dout, void* dq,
+                             void* dk, void* dv, float* dalpha, float* dbeta, float* dS0,
+                             kta_shape s, int H, int ld_heads, float scale, int erase_decayed,
+                             void* stream) {
+  return lin_bwd_common(q, k, v, alpha, beta, S0, dout, dq, dk, dv, dalpha, dbeta, dS0, s, H,
+                        ld_heads, scale, true, erase_decayed != 0, stream);
+}
 
 kta_status kta_stream_create(const kta_hybrid_cfg* cfg, kta_stream_t* out) {
   if (!out) return fail(KTA_ERR_INVALID_ARG, "null output handle");

@@ -55,6 +55,12 @@ _SIGS = {
     "kta_gla_chunk_fwd_noalloc": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
                                   _st),
     "kta_hybrid_fwd": ([ctypes.POINTER(HybridCfg), _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
+    "kta_swa_bwd": ([_vp] * 7 + [Shape, _i, _i, _i, _f, _vp], _st),
+    "kta_dswa_bwd": ([_vp] * 7 + [Shape, _i, _i, _i, _i, _f, _vp], _st),
+    "kta_gla_bwd": ([_vp, _vp, _vp, _fp, _fp, _vp, _vp, _vp, _vp, _fp, _fp, Shape, _i, _i, _f,
+                     _vp], _st),
+    "kta_gla_delta_bwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, _vp, _vp, _vp, _fp, _fp, _fp, Shape,
+                           _i, _i, _f, _i, _vp], _st),
     "kta_stream_create": ([ctypes.POINTER(HybridCfg), ctypes.POINTER(_vp)], _st),
     "kta_stream_step": ([_vp, _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
     "kta_stream_reset": ([_vp, _vp], _st),
@@ -187,6 +193,74 @@ def gla_delta_fwd(q, k, v, alpha, beta, *, chunk: int = 64, scale: float = 1.0, 
     erase_decayed: the GatedDeltaNet form M = alpha M (I - beta k k^T) + beta v k^T."""
     return _linear(True, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream,
                    erase_decayed)
+
+
+def _softmax_bwd(fn, q, k, v, dout, P, W, dil, scale, heads, stream):
+    for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _need(t, n, torch.float32)
+    Htot, d = q.shape[2], q.shape[3]
+    h0, h1 = heads if heads is not None else (0, Htot)
+    dq, dk, dv = (torch.zeros_like(q) for _ in range(3))
+    s = _shape(q, P)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    args = [_ptr(t, h0 * d) for t in (q, k, v, dout, dq, dk, dv)] + [s, h1 - h0, Htot, W]
+    if dil is not None:
+        args.append(dil)
+    _check(fn(*args, scale, _stream(stream)), fn.__name__)
+    return dq, dk, dv
+
+
+def swa_bwd(q, k, v, dout, *, P: int, W: int, scale: float | None = None, heads=None,
+            stream=None):
+    """Gradients (dq, dk, dv) of sum(dout * swa_fwd(q, k, v)); fp32. Heads outside the range
+    are zero."""
+    return _softmax_bwd(_lib.kta_swa_bwd, q, k, v, dout, P, W, None, scale, heads, stream)
+
+
+def dswa_bwd(q, k, v, dout, *, P: int, W: int, dil: int, scale: float | None = None, heads=None,
+             stream=None):
+    """Gradients (dq, dk, dv) of sum(dout * dswa_fwd(q, k, v)); fp32."""
+    return _softmax_bwd(_lib.kta_dswa_bwd, q, k, v, dout, P, W, dil, scale, heads, stream)
+
+
+def _linear_bwd(delta, q, k, v, alpha, beta, dout, scale, S0, heads, stream, erase_decayed):
+    for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout), ("alpha", alpha)):
+        _need(t, n, torch.float32)
+    if delta:
+        _need(beta, "beta", torch.float32)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32)
+    B, N, Htot, d = q.shape
+    h0, h1 = heads if heads is not None else (0, Htot)
+    H = h1 - h0
+    dq, dk, dv = (torch.zeros_like(q) for _ in range(3))
+    dalpha = torch.empty_like(alpha)
+    dbeta = torch.empty_like(beta) if delta else None
+    dS0 = torch.empty((B, H, d, d), device=q.device, dtype=torch.float32)
+    s = Shape(B, 1, N, d, _DT[q.dtype])
+    ptrs = [_ptr(t, h0 * d) for t in (q, k, v)]
+    grads = [_ptr(t, h0 * d) for t in (dq, dk, dv)]
+    if delta:
+        st = _lib.kta_gla_delta_bwd(*ptrs, _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(dout, h0 * d),
+                                    *grads, _ptr(dalpha), _ptr(dbeta), _ptr(dS0), s, H, Htot,
+                                    scale, int(erase_decayed), _stream(stream))
+        _check(st, "kta_gla_delta_bwd")
+        return dq, dk, dv, dalpha, dbeta, dS0
+    st = _lib.kta_gla_bwd(*ptrs, _ptr(alpha), _ptr(S0), _ptr(dout, h0 * d), *grads, _ptr(dalpha),
+                          _ptr(dS0), s, H, Htot, scale, _stream(stream))
+    _check(st, "kta_gla_bwd")
+    return dq, dk, dv, dalpha, dS0
+
+
+def gla_bwd(q, k, v, alpha, dout, *, scale: float = 1.0, S0=None, heads=None, stream=None):
+    """Gradients (dq, dk, dv, dalpha, dS0) of sum(dout * gla_chunk_fwd(...)); fp32."""
+    return _linear_bwd(False, q, k, v, alpha, None, dout, scale, S0, heads, stream, False)
+
+
+def gla_delta_bwd(q, k, v, alpha, beta, dout, *, scale: float = 1.0, S0=None, heads=None,
+                  stream=None, erase_decayed: bool = False):
+    """Gradients (dq, dk, dv, dalpha, dbeta, dS0) of sum(dout * gla_delta_fwd(...)); fp32."""
+    return _linear_bwd(True, q, k, v, alpha, beta, dout, scale, S0, heads, stream, erase_decayed)
 
 
 def hybrid_cfg(*, B: int, F: int, P: int, d: int, dtype=torch.bfloat16, n_swa: int, n_dswa: int,

@@ -185,6 +185,56 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
                           const float* alpha, const float* beta, void* o, void* stream);
 
 /*
+ * Reverse mode (training). The pages define only the forward operators (paper-read, section 2,
+ * second pillar); these entry points give the gradients of L = sum(dout * o) for the o of the
+ * matching forward call, in fp32 on CUDA cores: s.dtype must be KTA_F32, else
+ * KTA_ERR_UNSUPPORTED. Every tensor uses its forward layout (q, k, v, dout, dq, dk, dv:
+ * [B][N][ld_heads][d]; heads [0, H) are read and written, other heads untouched). Gradients are
+ * overwritten, not accumulated. The linear branches recompute states from checkpoints and take
+ * (ceil(N/32) + 32) * d * d + 64 * d floats of workspace per (sequence, head) from the calling
+ * stream's workspace cache.
+ *
+ * kta_swa_bwd / kta_dswa_bwd: with p_ts the forward's softmax weights over the visible keys,
+ *     ds_ts = p_ts (dout_t . v_s - dout_t . o_t),  dq_t = scale sum_s ds_ts k_s,
+ *     dk_s = scale sum_t ds_ts q_t,                dv_s = sum_t p_ts dout_t.
+ */
+kta_status kta_swa_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                       void* dk, void* dv, kta_shape s, int H, int ld_heads, int W, float scale,
+                       void* stream);
+kta_status kta_dswa_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                        void* dk, void* dv, kta_shape s, int H, int ld_heads, int W, int dil,
+                        float scale, void* stream);
+
+/*
+ * kta_gla_bwd: gradients of kta_gla_chunk_fwd's output. With the state adjoint
+ * G_t = scale q_t^T dout_t + diag(alpha_{t+1}) G_{t+1} (G after the last token = 0):
+ *     dq_t = scale S_t dout_t^T,  dk_t = G_t v_t^T,  dv_t = k_t G_t,
+ *     dalpha_t[i] = sum_j G_t[i][j] S_{t-1}[i][j],  dS0 = diag(alpha_1) G_1.
+ * dalpha: [B][N][H][d] fp32 (required). S0 as in the forward or NULL; dS0: [B][H][d][d] or NULL.
+ */
+kta_status kta_gla_bwd(const void* q, const void* k, const void* v, const float* alpha,
+                       const float* S0, const void* dout, void* dq, void* dk, void* dv,
+                       float* dalpha, float* dS0, kta_shape s, int H, int ld_heads, float scale,
+                       void* stream);
+
+/*
+ * kta_gla_delta_bwd: gradients of kta_gla_delta_fwd (erase_decayed = 0) or kta_gla_gdn_fwd
+ * (erase_decayed = 1). In the key-major state S = M^T both read w_t = k_t S_{t-1},
+ * u_t = beta_t (v_t - e_t w_t), S_t = alpha_t S_{t-1} + k_t^T u_t with e_t = 1 (the page's four
+ * lines) or alpha_t (decayed erase). With du_t = k_t G_t:
+ *     dv_t = beta_t du_t,  dbeta_t = du_t . (v_t - e_t w_t),
+ *     dk_t = G_t u_t^T - beta_t e_t S_{t-1} du_t^T,  dq_t = scale S_t dout_t^T,
+ *     dalpha_t = <G_t, S_{t-1}> (- beta_t du_t . w_t when decayed),
+ *     G_{t-1} = alpha_t G_t - beta_t e_t k_t^T du_t,  dS0 = G_0.
+ * dalpha, dbeta: [B][N][H] fp32 (required); S0 / dS0: [B][H][d][d] or NULL.
+ */
+kta_status kta_gla_delta_bwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, const void* dout, void* dq,
+                             void* dk, void* dv, float* dalpha, float* dbeta, float* dS0,
+                             kta_shape s, int H, int ld_heads, float scale, int erase_decayed,
+                             void* stream);
+
+/*
  * Streaming rollout -- paper-read, section 2, third pillar: low-latency rolling prediction, one
  * frame at a time. A stream holds, per sequence, the GLA state and a ring of the last
  * W_swa frames (SWA heads) or (W_dswa-1)*dil+1 frames (DSWA heads) of k and v. Each step takes
