@@ -44,12 +44,13 @@ def parse_args():
                          "headline line is the default, 21 frames)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="profiling only: override the delta workload's tokens per sequence")
-    ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep"),
+    ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep", "backward"),
                     default="hybrid",
                     help="hybrid: the 21-frame hybrid layer (the headline line); delta: gated "
                          "delta rule, 2 x 65,536 tokens x 16 heads; stream: 240-frame rollout one "
                          "frame per call; sweep: hybrid layer vs full frame-causal attention for "
-                         "F = 8..256 frames of 1,024 tokens (one line per F)")
+                         "F = 8..256 frames of 1,024 tokens (one line per F); backward: the "
+                         "hybrid layer's reverse mode in fp32")
     return ap.parse_args()
 
 
@@ -81,6 +82,18 @@ def delta_bytes(w) -> float:
 def delta_flops(w) -> float:
     """MMA FLOPs of the chunked delta rule: 10 C d + 6 d^2 per token-head."""
     return (10.0 * w.chunk * w.d + 6.0 * w.d * w.d) * w.B * w.N * w.n_gla
+
+
+def softmax_bwd_flops(w) -> dict:
+    """Algorithmic FLOPs of the softmax branches' reverse mode, 2d per product per visible pair:
+    the dq kernel forms S, dP and dQ (6d), the key-major kernel S, dP, dV and dK (8d)."""
+    n = visible_pairs(w)
+    return {"softmax_bwd_q_f32": 6.0 * w.d * n, "softmax_bwd_kv_f32": 8.0 * w.d * n}
+
+
+def fp32_alu_tflops(sm_mhz: float) -> float:
+    """fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP per clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 def full_causal_flops(w) -> float:
@@ -539,6 +552,47 @@ def run_other(args):
                          "peak_source": peaks_kind},
             "kernels": kern})
         st.close()
+    elif args.workload == "backward":
+        w = synth.HYBRID_BWD_F32
+        x = synth.make_inputs_device(w, seed=w.seed_base)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(w.seed_base + 1)
+        dout = torch.randn(x["q"].shape, generator=g, device="cuda")
+        grads = tuple(torch.zeros_like(x["q"]) for _ in range(3))
+        q, k, v, a = x["q"], x["k"], x["v"], x["alpha"]
+        ns, nd = w.n_swa, w.n_dswa
+        side = torch.cuda.Stream()
+
+        def step():
+            # the GLA heads' reverse recurrence (one CTA per head) runs beside the softmax heads
+            main = torch.cuda.current_stream()
+            side.wait_stream(main)
+            kta.gla_bwd(q, k, v, a, dout, heads=(ns + nd, w.H), out=grads, stream=side)
+            kta.swa_bwd(q, k, v, dout, P=w.P, W=w.W_swa, heads=(0, ns), out=grads)
+            kta.dswa_bwd(q, k, v, dout, P=w.P, W=w.W_dswa, dil=w.dil, heads=(ns, ns + nd),
+                         out=grads)
+            main.wait_stream(side)
+        steps, warm = min(args.steps, 5), max(1, min(args.warmup, 3))
+        clk = ClockSampler("0")
+        clk.start()
+        ms = _device_ms(step, steps, warm)
+        clocks = clk.stop() or {}
+        kern = _traced(step, steps)
+        sm_mhz = clocks.get("sm_mhz") or 1965.0
+        peak = fp32_alu_tflops(sm_mhz)
+        fl = softmax_bwd_flops(w)
+        top = max(fl, key=lambda n: kern.get(n, {}).get("ms_per_step", 0.0))
+        k_ms = kern[top]["ms_per_step"]
+        lines.append({
+            "workload": w.name, "metric": "hybrid layer reverse mode tokens/s (fp32)",
+            "unit": "tokens/s", "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms,
+            "steps": steps, "warmup": warm, "dtype": "f32",
+            "config": {"B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d},
+            "roofline": {"kernel": top, "bound": "alu", "unit": "TFLOP/s",
+                         "achieved": fl[top] / (k_ms / 1e3) / 1e12, "peak": peak,
+                         "frac": fl[top] / (k_ms / 1e3) / 1e12 / peak,
+                         "peak_source": f"fp32 FMA lanes x median SM clock {sm_mhz:.0f} MHz"},
+            "clocks": clocks, "kernels": kern})
     else:  # sweep
         for F in (8, 16, 32, 64, 128, 256):
             w = synth.sweep_workload(F)

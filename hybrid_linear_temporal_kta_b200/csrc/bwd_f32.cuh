@@ -27,114 +27,316 @@ struct SoftmaxBwdParams {
   int W, dil;
   long long ld;      // row stride of q / k / v / dO / dq / dk / dv (elements)
   float scale;
+  float* stats;      // [3][B][H][N]: row maximum m, 1 / l, dO_t . o_t
 };
 
-// One warp per (query token, head, sequence): recompute the row's softmax statistics and
-// output, then accumulate dq in registers and dk, dv with atomics.
-__global__ void __launch_bounds__(128) softmax_bwd_f32_kernel(
-    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
-    const float* __restrict__ dout, float* __restrict__ dq, float* dk, float* dv,
-    const SoftmaxBwdParams p) {
-  __shared__ float qs[4][128], dos[4][128];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 4 + warp;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const bool active = t < p.N;
-  const int d = p.d;
-  const long long rb = static_cast<long long>(b) * p.N;
-  const long long qrow = (rb + (active ? t : 0)) * p.ld + static_cast<long long>(h) * d;
-  for (int c = lane; c < d; c += 32) {
-    qs[warp][c] = active ? q[qrow + c] : 0.f;
-    dos[warp][c] = active ? dout[qrow + c] : 0.f;
+// Layout shared by the two softmax-backward kernels. A warp takes SB_R = 4 rows of one frame
+// (a CTA of 4 warps takes 16), its lanes own DPL = d / 32 consecutive dims of every row, and the
+// other side (keys or queries) is walked SB_K = 8 rows at a time, so one block is 4 x 8 = 32
+// (row, other) pairs: lane l ends up owning pair (l / 8, l % 8).
+constexpr int SB_R = 4, SB_K = 8, SB_ROWS_CTA = 16;
+
+template <int DPL>
+__device__ __forceinline__ void load_dims(const float* __restrict__ row, bool ok, float (&x)[DPL]) {
+  if constexpr (DPL == 4) {
+    const float4 u = ok ? __ldg(reinterpret_cast<const float4*>(row)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+  } else if constexpr (DPL == 2) {
+    const float2 u = ok ? __ldg(reinterpret_cast<const float2*>(row)) : make_float2(0.f, 0.f);
+    x[0] = u.x; x[1] = u.y;
+  } else {
+    x[0] = ok ? __ldg(row) : 0.f;
   }
-  __syncwarp();
-  if (!active) return;
-  const int f = t / p.P;
-  const int nfr = p.dil == 1 ? min(p.W, f + 1) : min(p.W, f / p.dil + 1);
-  // pass 1: row maximum m, normaliser l and output o (lanes over keys, then over dims)
-  float m = -INFINITY, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int jf = nfr - 1; jf >= 0; --jf) {
-    const long long base = rb + static_cast<long long>(f - jf * p.dil) * p.P;
-    for (int s0 = 0; s0 < p.P; s0 += 32) {
-      const int s = s0 + lane;
-      float sc = -INFINITY;
-      if (s < p.P) {
-        const float* kr = k + (base + s) * p.ld + static_cast<long long>(h) * d;
-        float dot = 0.f;
-        for (int c = 0; c < d; ++c) dot = fmaf(qs[warp][c], kr[c], dot);
-        sc = dot * p.scale;
-      }
-      float mx = sc;
-      for (int o2 = 16; o2; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-      const float mnew = fmaxf(m, mx);
-      const float corr = expf(m - mnew);
-      const float pr = s < p.P ? expf(sc - mnew) : 0.f;
-      float ps = pr;
-      for (int o2 = 16; o2; o2 >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
-      l = l * corr + ps;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[c] *= corr;
-      const int nk = min(32, p.P - s0);
-      for (int jj = 0; jj < nk; ++jj) {
-        const float pj = __shfl_sync(0xffffffffu, pr, jj);
-        const float* vr = v + (base + s0 + jj) * p.ld + static_cast<long long>(h) * d;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (lane + 32 * c < d) acc[c] = fmaf(pj, vr[lane + 32 * c], acc[c]);
-      }
-      m = mnew;
-    }
-  }
-  const float inv = 1.f / l;
-  float dD = 0.f;  // dO_t . o_t
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    if (lane + 32 * c < d) dD = fmaf(dos[warp][lane + 32 * c], acc[c] * inv, dD);
-  for (int o2 = 16; o2; o2 >>= 1) dD += __shfl_xor_sync(0xffffffffu, dD, o2);
-  // pass 2: ds for every visible key; dq in registers, dk and dv by atomics
-  float gq[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int jf = nfr - 1; jf >= 0; --jf) {
-    const long long base = rb + static_cast<long long>(f - jf * p.dil) * p.P;
-    for (int s0 = 0; s0 < p.P; s0 += 32) {
-      const int s = s0 + lane;
-      float pj = 0.f, ds = 0.f;
-      if (s < p.P) {
-        const float* kr = k + (base + s) * p.ld + static_cast<long long>(h) * d;
-        const float* vr = v + (base + s) * p.ld + static_cast<long long>(h) * d;
-        float dot = 0.f, dp = 0.f;
-        for (int c = 0; c < d; ++c) {
-          dot = fmaf(qs[warp][c], kr[c], dot);
-          dp = fmaf(dos[warp][c], vr[c], dp);
-        }
-        pj = expf(dot * p.scale - m) * inv;
-        ds = pj * (dp - dD);
-      }
-      const int nk = min(32, p.P - s0);
-      for (int jj = 0; jj < nk; ++jj) {
-        const float dsj = __shfl_sync(0xffffffffu, ds, jj) * p.scale;
-        const float pjj = __shfl_sync(0xffffffffu, pj, jj);
-        const long long kr = (base + s0 + jj) * p.ld + static_cast<long long>(h) * d;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int cc = lane + 32 * c;
-          if (cc < d) {
-            gq[c] = fmaf(dsj, k[kr + cc], gq[c]);
-            atomicAdd(&dk[kr + cc], dsj * qs[warp][cc]);
-            atomicAdd(&dv[kr + cc], pjj * dos[warp][cc]);
-          }
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    if (lane + 32 * c < d) dq[qrow + lane + 32 * c] = gq[c];
 }
 
-// Zero a [rows][H][d] head range of a [rows][ld] array (one thread per element).
-__global__ void zero_rows_f32_kernel(float* x, long long rows, int Hd, long long ld) {
-  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e < rows * Hd) x[(e / Hd) * ld + e % Hd] = 0.f;
+template <int DPL>
+__device__ __forceinline__ void store_dims(float* row, const float (&x)[DPL], float mul) {
+  if constexpr (DPL == 4) {
+    *reinterpret_cast<float4*>(row) = make_float4(x[0] * mul, x[1] * mul, x[2] * mul, x[3] * mul);
+  } else if constexpr (DPL == 2) {
+    *reinterpret_cast<float2*>(row) = make_float2(x[0] * mul, x[1] * mul);
+  } else {
+    row[0] = x[0] * mul;
+  }
+}
+
+// 32 per-lane partial sums v[0..31] -> lane l returns the warp-wide sum of entry l (a butterfly
+// reduce-scatter: five exchange steps, each halving the entries a lane keeps).
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool hi = lane & half;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = hi ? v[i] : v[i + half];
+      const float keep = hi ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ float group8_max(float x) {
+#pragma unroll
+  for (int o = 4; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+__device__ __forceinline__ float group8_sum(float x) {
+#pragma unroll
+  for (int o = 4; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// dq pass. Per warp: 4 query rows of frame f. Pass 1 recomputes each row's maximum m, sum l and
+// output o (online softmax over the visible key frames, oldest first); pass 2 forms
+// ds_ts = p_ts (dO_t . v_s - dO_t . o_t) and dq_t = scale sum_s ds_ts k_s. The statistics
+// (m, 1/l, dO_t . o_t) go to p.stats for the key-major pass.
+template <int DPL>
+__global__ void __launch_bounds__(128) softmax_bwd_q_f32_kernel(
+    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    const float* __restrict__ dout, float* __restrict__ dq, const SoftmaxBwdParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int groups = (p.P + SB_ROWS_CTA - 1) / SB_ROWS_CTA;
+  const int f = blockIdx.x / groups;
+  const int i0 = (blockIdx.x % groups) * SB_ROWS_CTA + warp * SB_R;  // row within the frame
+  if (i0 >= p.P) return;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int d = p.d;
+  const long long rb = static_cast<long long>(b) * p.N;
+  const long long col = static_cast<long long>(h) * d + lane * DPL;
+  float qr[SB_R][DPL], dr[SB_R][DPL], acc[SB_R][DPL];
+  float m[SB_R], l[SB_R];
+#pragma unroll
+  for (int r = 0; r < SB_R; ++r) {
+    const bool ok = i0 + r < p.P;
+    const long long row = (rb + static_cast<long long>(f) * p.P + i0 + (ok ? r : 0)) * p.ld + col;
+    load_dims<DPL>(q + row, ok, qr[r]);
+    load_dims<DPL>(dout + row, ok, dr[r]);
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) acc[r][c] = 0.f;
+    m[r] = -INFINITY;
+    l[r] = 0.f;
+  }
+  const int my_r = lane >> 3, my_j = lane & 7;
+  const int nfr = min(p.W, f / p.dil + 1);
+  // ---- pass 1: m, l, o
+  for (int jf = nfr - 1; jf >= 0; --jf) {
+    const long long base = rb + static_cast<long long>(f - jf * p.dil) * p.P;
+    for (int s0 = 0; s0 < p.P; s0 += SB_K) {
+      float part[32];
+#pragma unroll
+      for (int j = 0; j < SB_K; ++j) {
+        float kj[DPL];
+        const bool ok = s0 + j < p.P;
+        load_dims<DPL>(k + (base + (ok ? s0 + j : 0)) * p.ld + col, ok, kj);
+#pragma unroll
+        for (int r = 0; r < SB_R; ++r) {
+          float x = 0.f;
+#pragma unroll
+          for (int c = 0; c < DPL; ++c) x = fmaf(qr[r][c], kj[c], x);
+          part[r * SB_K + j] = x;
+        }
+      }
+      const float dot = reduce_scatter32(part, lane);
+      const float sc = s0 + my_j < p.P ? dot * p.scale : -INFINITY;
+      const float mx = group8_max(sc);
+      float mnew[SB_R], corr[SB_R];
+#pragma unroll
+      for (int r = 0; r < SB_R; ++r) {
+        mnew[r] = fmaxf(m[r], __shfl_sync(0xffffffffu, mx, r * SB_K));
+        corr[r] = expf(m[r] - mnew[r]);
+      }
+      float mine = mnew[0];
+#pragma unroll
+      for (int r = 1; r < SB_R; ++r) mine = my_r == r ? mnew[r] : mine;
+      const float pr = expf(sc - mine);
+      const float ps = group8_sum(pr);
+#pragma unroll
+      for (int r = 0; r < SB_R; ++r) {
+        l[r] = fmaf(l[r], corr[r], __shfl_sync(0xffffffffu, ps, r * SB_K));
+        m[r] = mnew[r];
+#pragma unroll
+        for (int c = 0; c < DPL; ++c) acc[r][c] *= corr[r];
+      }
+#pragma unroll
+      for (int j = 0; j < SB_K; ++j) {
+        float vj[DPL];
+        const bool ok = s0 + j < p.P;
+        load_dims<DPL>(v + (base + (ok ? s0 + j : 0)) * p.ld + col, ok, vj);
+#pragma unroll
+        for (int r = 0; r < SB_R; ++r) {
+          const float pj = __shfl_sync(0xffffffffu, pr, r * SB_K + j);
+#pragma unroll
+          for (int c = 0; c < DPL; ++c) acc[r][c] = fmaf(pj, vj[c], acc[r][c]);
+        }
+      }
+    }
+  }
+  float inv[SB_R], Dr[SB_R];
+#pragma unroll
+  for (int r = 0; r < SB_R; ++r) {
+    inv[r] = 1.f / l[r];
+    float x = 0.f;
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) x = fmaf(dr[r][c], acc[r][c] * inv[r], x);
+    Dr[r] = warp_sum(x);
+  }
+  if (lane < SB_R && i0 + lane < p.P) {
+    float mm = m[0], ii = inv[0], dd = Dr[0];
+#pragma unroll
+    for (int r = 1; r < SB_R; ++r)
+      if (lane == r) { mm = m[r]; ii = inv[r]; dd = Dr[r]; }
+    const long long si = (static_cast<long long>(b) * p.H + h) * p.N +
+                         static_cast<long long>(f) * p.P + i0 + lane;
+    const long long plane = static_cast<long long>(p.B) * p.H * p.N;
+    p.stats[si] = mm;
+    p.stats[plane + si] = ii;
+    p.stats[2 * plane + si] = dd;
+  }
+  float m_mine = m[0], inv_mine = inv[0], D_mine = Dr[0];
+#pragma unroll
+  for (int r = 1; r < SB_R; ++r)
+    if (my_r == r) { m_mine = m[r]; inv_mine = inv[r]; D_mine = Dr[r]; }
+  // ---- pass 2: ds and dq (acc is reused for dq)
+#pragma unroll
+  for (int r = 0; r < SB_R; ++r)
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) acc[r][c] = 0.f;
+  for (int jf = nfr - 1; jf >= 0; --jf) {
+    const long long base = rb + static_cast<long long>(f - jf * p.dil) * p.P;
+    for (int s0 = 0; s0 < p.P; s0 += SB_K) {
+      float ps[32], pd[32], kk[SB_K][DPL];
+#pragma unroll
+      for (int j = 0; j < SB_K; ++j) {
+        float vj[DPL];
+        const bool ok = s0 + j < p.P;
+        const long long row = (base + (ok ? s0 + j : 0)) * p.ld + col;
+        load_dims<DPL>(k + row, ok, kk[j]);
+        load_dims<DPL>(v + row, ok, vj);
+#pragma unroll
+        for (int r = 0; r < SB_R; ++r) {
+          float x = 0.f, y = 0.f;
+#pragma unroll
+          for (int c = 0; c < DPL; ++c) {
+            x = fmaf(qr[r][c], kk[j][c], x);
+            y = fmaf(dr[r][c], vj[c], y);
+          }
+          ps[r * SB_K + j] = x;
+          pd[r * SB_K + j] = y;
+        }
+      }
+      const float dot = reduce_scatter32(ps, lane);
+      const float dp = reduce_scatter32(pd, lane);
+      const float ds = s0 + my_j < p.P
+                           ? expf(dot * p.scale - m_mine) * inv_mine * (dp - D_mine) : 0.f;
+#pragma unroll
+      for (int j = 0; j < SB_K; ++j)
+#pragma unroll
+        for (int r = 0; r < SB_R; ++r) {
+          const float g = __shfl_sync(0xffffffffu, ds, r * SB_K + j);
+#pragma unroll
+          for (int c = 0; c < DPL; ++c) acc[r][c] = fmaf(g, kk[j][c], acc[r][c]);
+        }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < SB_R; ++r)
+    if (i0 + r < p.P)
+      store_dims<DPL>(dq + (rb + static_cast<long long>(f) * p.P + i0 + r) * p.ld + col, acc[r],
+                      p.scale);
+}
+
+// dk / dv pass. Per warp: 4 key rows of frame g, visible to query frames g, g + dil, ...,
+// g + (W-1) dil (those < F). For 8 queries at a time it forms S and dP for the 32 (key, query)
+// pairs, p = exp(scale S - m) / l and ds = p (dP - dO . o) from the stored statistics, then
+// dv_s += p dO_t and dk_s += scale ds q_t.
+template <int DPL>
+__global__ void __launch_bounds__(128) softmax_bwd_kv_f32_kernel(
+    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    const float* __restrict__ dout, float* __restrict__ dk, float* __restrict__ dv,
+    const SoftmaxBwdParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int groups = (p.P + SB_ROWS_CTA - 1) / SB_ROWS_CTA;
+  const int g = blockIdx.x / groups;
+  const int i0 = (blockIdx.x % groups) * SB_ROWS_CTA + warp * SB_R;
+  if (i0 >= p.P) return;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int d = p.d, F = p.N / p.P;
+  const long long rb = static_cast<long long>(b) * p.N;
+  const long long col = static_cast<long long>(h) * d + lane * DPL;
+  float kr[SB_R][DPL], vr[SB_R][DPL], gk[SB_R][DPL], gv[SB_R][DPL];
+#pragma unroll
+  for (int r = 0; r < SB_R; ++r) {
+    const bool ok = i0 + r < p.P;
+    const long long row = (rb + static_cast<long long>(g) * p.P + i0 + (ok ? r : 0)) * p.ld + col;
+    load_dims<DPL>(k + row, ok, kr[r]);
+    load_dims<DPL>(v + row, ok, vr[r]);
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) gk[r][c] = gv[r][c] = 0.f;
+  }
+  const int my_j = lane & 7;
+  const long long plane = static_cast<long long>(p.B) * p.H * p.N;
+  const float* sm = p.stats + (static_cast<long long>(b) * p.H + h) * p.N;
+  for (int j = 0; j < p.W; ++j) {
+    const int f = g + j * p.dil;
+    if (f >= F) break;
+    const long long fb = static_cast<long long>(f) * p.P;
+    for (int t0 = 0; t0 < p.P; t0 += SB_K) {
+      float ps[32], pd[32], qq[SB_K][DPL], dd[SB_K][DPL];
+#pragma unroll
+      for (int jj = 0; jj < SB_K; ++jj) {
+        const bool ok = t0 + jj < p.P;
+        const long long row = (rb + fb + (ok ? t0 + jj : 0)) * p.ld + col;
+        load_dims<DPL>(q + row, ok, qq[jj]);
+        load_dims<DPL>(dout + row, ok, dd[jj]);
+#pragma unroll
+        for (int r = 0; r < SB_R; ++r) {
+          float x = 0.f, y = 0.f;
+#pragma unroll
+          for (int c = 0; c < DPL; ++c) {
+            x = fmaf(kr[r][c], qq[jj][c], x);
+            y = fmaf(vr[r][c], dd[jj][c], y);
+          }
+          ps[r * SB_K + jj] = x;
+          pd[r * SB_K + jj] = y;
+        }
+      }
+      const float dot = reduce_scatter32(ps, lane);
+      const float dpv = reduce_scatter32(pd, lane);
+      float pr = 0.f, ds = 0.f;
+      if (t0 + my_j < p.P) {
+        const long long si = fb + t0 + my_j;
+        pr = expf(dot * p.scale - sm[si]) * sm[plane + si];
+        ds = pr * (dpv - sm[2 * plane + si]);
+      }
+#pragma unroll
+      for (int jj = 0; jj < SB_K; ++jj)
+#pragma unroll
+        for (int r = 0; r < SB_R; ++r) {
+          const float pj = __shfl_sync(0xffffffffu, pr, r * SB_K + jj);
+          const float gj = __shfl_sync(0xffffffffu, ds, r * SB_K + jj);
+#pragma unroll
+          for (int c = 0; c < DPL; ++c) {
+            gv[r][c] = fmaf(pj, dd[jj][c], gv[r][c]);
+            gk[r][c] = fmaf(gj, qq[jj][c], gk[r][c]);
+          }
+        }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < SB_R; ++r)
+    if (i0 + r < p.P) {
+      const long long row = (rb + static_cast<long long>(g) * p.P + i0 + r) * p.ld + col;
+      store_dims<DPL>(dk + row, gk[r], p.scale);
+      store_dims<DPL>(dv + row, gv[r], 1.f);
+    }
 }
 
 constexpr int BWD_CK = 32;  // tokens between stored states in the linear-branch backward
@@ -163,7 +365,8 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
   extern __shared__ float bsm[];
   constexpr int LDG = D + 1;
   float* G = bsm;                 // [D][D + 1]
-  float* qv = G + D * LDG;        // q_t
+  float* Sx = G + D * LDG;        // [2][D][D + 1]: S_t and S_{t-1} in the reverse pass
+  float* qv = Sx + 2 * D * LDG;   // q_t
   float* kv = qv + D;             // k_t
   float* vv = kv + D;             // v_t
   float* dv_ = vv + D;            // dO_t
@@ -190,17 +393,17 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
     if (p.delta) {
       const float a = av[0], be = gate_b(t), ae = p.erase_decayed ? a : 1.f;
       float w = 0.f;
-#pragma unroll 8
+#pragma unroll
       for (int i = 0; i < D; ++i) w = fmaf(kv[i], S[i], w);
       const float u = be * (vv[j] - ae * w);
       if (keep_uw) {
         Ub[tl * D + j] = u;
         Wb[tl * D + j] = w;
       }
-#pragma unroll 8
+#pragma unroll
       for (int i = 0; i < D; ++i) S[i] = fmaf(a, S[i], kv[i] * u);
     } else {
-#pragma unroll 8
+#pragma unroll
       for (int i = 0; i < D; ++i) S[i] = fmaf(av[i], S[i], kv[i] * vv[j]);
     }
   };
@@ -212,12 +415,12 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
   };
 
   // ---- forward: the state before every BWD_CK-th token
-#pragma unroll 8
+#pragma unroll
   for (int i = 0; i < D; ++i) S[i] = p.S0 ? p.S0[bh * D * D + i * D + j] : 0.f;
   for (int t = 0; t < p.N; ++t) {
     if (t % BWD_CK == 0) {
       float* c = ck + static_cast<long long>(t / BWD_CK) * D * D;
-#pragma unroll 8
+#pragma unroll
       for (int i = 0; i < D; ++i) c[i * D + j] = S[i];
     }
     __syncthreads();
@@ -226,12 +429,12 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
     step(t, 0, false);
   }
   // ---- reverse, one chunk of BWD_CK tokens at a time
-#pragma unroll 8
+#pragma unroll
   for (int i = 0; i < D; ++i) G[i * LDG + j] = 0.f;
   for (int c = p.nck - 1; c >= 0; --c) {
     const int t0 = c * BWD_CK, t1 = min(p.N, t0 + BWD_CK);
     const float* cs = ck + static_cast<long long>(c) * D * D;
-#pragma unroll 8
+#pragma unroll
     for (int i = 0; i < D; ++i) S[i] = cs[i * D + j];
     for (int t = t0; t < t1; ++t) {  // recompute and keep the chunk's states
       __syncthreads();
@@ -239,10 +442,15 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
       __syncthreads();
       step(t, t - t0, true);
       float* st = buf + static_cast<long long>(t - t0) * D * D;
-#pragma unroll 8
+#pragma unroll
       for (int i = 0; i < D; ++i) st[i * D + j] = S[i];
     }
     __syncthreads();
+    // rows of S_t and S_{t-1} are read from shared memory: S_{t1-1} is in registers
+    float* cur = Sx;
+    float* prv = Sx + D * LDG;
+#pragma unroll
+    for (int i = 0; i < D; ++i) cur[i * LDG + j] = S[i];
     for (int t = t1 - 1; t >= t0; --t) {
       const long long r = row_of(t);
       qv[j] = p.q[r + j];
@@ -250,37 +458,39 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
       vv[j] = p.v[r + j];
       dv_[j] = p.dout[r + j];
       av[j] = p.delta ? (j == 0 ? gate_a(t, 0) : 0.f) : gate_a(t, j);
+      const float* src = t == t0 ? cs : buf + static_cast<long long>(t - t0 - 1) * D * D;
+      for (int i = 0; i < D; ++i) prv[i * LDG + j] = src[i * D + j];
       __syncthreads();
-      const float* St = buf + static_cast<long long>(t - t0) * D * D;
-      const float* Sp = t == t0 ? cs : buf + static_cast<long long>(t - t0 - 1) * D * D;
+      const float* St = cur;
+      const float* Sp = prv;
       // G_t: add the output term (column j)
-#pragma unroll 8
+#pragma unroll
       for (int i = 0; i < D; ++i) G[i * LDG + j] = fmaf(p.scale * qv[i], dv_[j], G[i * LDG + j]);
       __syncthreads();
       if (!p.delta) {
         // column j: dv; row j: dq, dk, dalpha
         float acc = 0.f;
-#pragma unroll 8
+#pragma unroll
         for (int i = 0; i < D; ++i) acc = fmaf(kv[i], G[i * LDG + j], acc);
         p.dv[r + j] = acc;
         const int i = j;
         float aq = 0.f, ak = 0.f, aa = 0.f;
         for (int jj = 0; jj < D; ++jj) {
-          aq = fmaf(St[i * D + jj], dv_[jj], aq);
+          aq = fmaf(St[i * LDG + jj], dv_[jj], aq);
           ak = fmaf(G[i * LDG + jj], vv[jj], ak);
-          aa = fmaf(G[i * LDG + jj], Sp[i * D + jj], aa);
+          aa = fmaf(G[i * LDG + jj], Sp[i * LDG + jj], aa);
         }
         p.dq[r + i] = p.scale * aq;
         p.dk[r + i] = ak;
         p.dalpha[((rb + t) * p.H + h) * D + i] = aa;
         __syncthreads();
-#pragma unroll 8
+#pragma unroll
         for (int ii = 0; ii < D; ++ii) G[ii * LDG + j] *= av[ii];
       } else {
         const float a = av[0], be = gate_b(t), ae = p.erase_decayed ? a : 1.f;
         const int tl = t - t0;
         float acc = 0.f;
-#pragma unroll 8
+#pragma unroll
         for (int i = 0; i < D; ++i) acc = fmaf(kv[i], G[i * LDG + j], acc);
         du[j] = acc;
         p.dv[r + j] = be * acc;
@@ -291,10 +501,10 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
         const int i = j;
         float aq = 0.f, ak = 0.f, as = 0.f;
         for (int jj = 0; jj < D; ++jj) {
-          aq = fmaf(St[i * D + jj], dv_[jj], aq);
+          aq = fmaf(St[i * LDG + jj], dv_[jj], aq);
           ak = fmaf(G[i * LDG + jj], Ub[tl * D + jj], ak);
-          as = fmaf(Sp[i * D + jj], du[jj], as);
-          dal = fmaf(G[i * LDG + jj], Sp[i * D + jj], dal);
+          as = fmaf(Sp[i * LDG + jj], du[jj], as);
+          dal = fmaf(G[i * LDG + jj], Sp[i * LDG + jj], dal);
         }
         p.dq[r + i] = p.scale * aq;
         p.dk[r + i] = ak - be * ae * as;
@@ -315,15 +525,18 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
             p.dalpha[(rb + t) * p.H + h] = sa;
           }
         }
-#pragma unroll 8
+#pragma unroll
         for (int ii = 0; ii < D; ++ii)
           G[ii * LDG + j] = a * G[ii * LDG + j] - be * ae * kv[ii] * du[j];
       }
       __syncthreads();
+      float* tmp = cur;
+      cur = prv;
+      prv = tmp;
     }
   }
   if (p.dS0) {
-#pragma unroll 8
+#pragma unroll
     for (int i = 0; i < D; ++i) p.dS0[bh * D * D + i * D + j] = G[i * LDG + j];
   }
 }

@@ -887,15 +887,6 @@ kta_status bwd_f32_only(const kta_shape& s) {
   return KTA_OK;
 }
 
-kta_status zero_heads_f32(void* x, long long rows, int Hd, long long ld, cudaStream_t st) {
-  const long long n = rows * Hd;
-  if (n == 0) return KTA_OK;
-  kta::zero_rows_f32_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-      static_cast<float*>(x), rows, Hd, ld);
-  KTA_CUDA(cudaGetLastError());
-  return KTA_OK;
-}
-
 kta_status softmax_bwd_common(const void* q, const void* k, const void* v,
                                      const void* dout, void* dq, void* dk, void* dv, kta_shape s,
                                      int H, int ld_heads, int W, int dil, float scale,
@@ -909,9 +900,8 @@ kta_status softmax_bwd_common(const void* q, const void* k, const void* v,
   if (s.B > 65535 || H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B and H must be <= 65535");
   cudaStream_t st = as_stream(stream);
   const long long N = static_cast<long long>(s.F) * s.P, ld = static_cast<long long>(ld_heads) * s.d;
-  if ((r = zero_heads_f32(dk, s.B * N, H * s.d, ld, st)) ||
-      (r = zero_heads_f32(dv, s.B * N, H * s.d, ld, st)))
-    return r;
+  void* ws = nullptr;
+  if ((r = workspace(static_cast<size_t>(3) * s.B * H * N * sizeof(float), st, &ws))) return r;
   kta::SoftmaxBwdParams p{};
   p.B = s.B;
   p.N = static_cast<int>(N);
@@ -922,11 +912,30 @@ kta_status softmax_bwd_common(const void* q, const void* k, const void* v,
   p.dil = dil;
   p.ld = ld;
   p.scale = scale;
-  TraceScope ts("softmax_bwd_f32", st);
-  kta::softmax_bwd_f32_kernel<<<dim3(static_cast<unsigned>((N + 3) / 4), H, s.B), 128, 0, st>>>(
-      static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-      static_cast<const float*>(dout), static_cast<float*>(dq), static_cast<float*>(dk),
-      static_cast<float*>(dv), p);
+  p.stats = static_cast<float*>(ws);
+  const dim3 grid(static_cast<unsigned>(
+                      s.F * ((s.P + kta::SB_ROWS_CTA - 1) / kta::SB_ROWS_CTA)), H, s.B);
+  const float *fq = static_cast<const float*>(q), *fk = static_cast<const float*>(k),
+              *fv = static_cast<const float*>(v), *fdo = static_cast<const float*>(dout);
+  float *fdq = static_cast<float*>(dq), *fdk = static_cast<float*>(dk),
+        *fdv = static_cast<float*>(dv);
+  {
+    TraceScope ts("softmax_bwd_q_f32", st);
+    if (s.d == 128)
+      kta::softmax_bwd_q_f32_kernel<4><<<grid, 128, 0, st>>>(fq, fk, fv, fdo, fdq, p);
+    else if (s.d == 64)
+      kta::softmax_bwd_q_f32_kernel<2><<<grid, 128, 0, st>>>(fq, fk, fv, fdo, fdq, p);
+    else
+      kta::softmax_bwd_q_f32_kernel<1><<<grid, 128, 0, st>>>(fq, fk, fv, fdo, fdq, p);
+    KTA_CUDA(cudaGetLastError());
+  }
+  TraceScope ts("softmax_bwd_kv_f32", st);
+  if (s.d == 128)
+    kta::softmax_bwd_kv_f32_kernel<4><<<grid, 128, 0, st>>>(fq, fk, fv, fdo, fdk, fdv, p);
+  else if (s.d == 64)
+    kta::softmax_bwd_kv_f32_kernel<2><<<grid, 128, 0, st>>>(fq, fk, fv, fdo, fdk, fdv, p);
+  else
+    kta::softmax_bwd_kv_f32_kernel<1><<<grid, 128, 0, st>>>(fq, fk, fv, fdo, fdk, fdv, p);
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
@@ -938,7 +947,7 @@ kta_status launch_lin_bwd(kta::LinBwdParams p, int B, cudaStream_t st) {
   kta_status r = workspace(static_cast<size_t>(per) * B * p.H * sizeof(float), st, &ws);
   if (r) return r;
   p.ws = static_cast<float*>(ws);
-  const size_t smem = (static_cast<size_t>(D) * (D + 1) + 8 * D) * sizeof(float);
+  const size_t smem = (3 * static_cast<size_t>(D) * (D + 1) + 8 * D) * sizeof(float);
   if ((r = set_smem_attr(kta::lin_bwd_f32_kernel<D>, smem))) return r;
   TraceScope ts(p.delta ? "delta_bwd_f32" : "gla_bwd_f32", st);
   kta::lin_bwd_f32_kernel<D><<<dim3(p.H, B), D, smem, st>>>(p);

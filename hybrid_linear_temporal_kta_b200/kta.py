@@ -195,12 +195,23 @@ def gla_delta_fwd(q, k, v, alpha, beta, *, chunk: int = 64, scale: float = 1.0, 
                    erase_decayed)
 
 
-def _softmax_bwd(fn, q, k, v, dout, P, W, dil, scale, heads, stream):
+def _grads(q, out):
+    """Gradient buffers: `out` (three tensors shaped like q) or fresh zeros."""
+    if out is None:
+        return tuple(torch.zeros_like(q) for _ in range(3))
+    for n, t in zip(("dq", "dk", "dv"), out):
+        _need(t, n, torch.float32)
+        if t.shape != q.shape:
+            raise ValueError(f"{n} must have q's shape")
+    return tuple(out)
+
+
+def _softmax_bwd(fn, q, k, v, dout, P, W, dil, scale, heads, out, stream):
     for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
         _need(t, n, torch.float32)
     Htot, d = q.shape[2], q.shape[3]
     h0, h1 = heads if heads is not None else (0, Htot)
-    dq, dk, dv = (torch.zeros_like(q) for _ in range(3))
+    dq, dk, dv = _grads(q, out)
     s = _shape(q, P)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     args = [_ptr(t, h0 * d) for t in (q, k, v, dout, dq, dk, dv)] + [s, h1 - h0, Htot, W]
@@ -210,20 +221,20 @@ def _softmax_bwd(fn, q, k, v, dout, P, W, dil, scale, heads, stream):
     return dq, dk, dv
 
 
-def swa_bwd(q, k, v, dout, *, P: int, W: int, scale: float | None = None, heads=None,
+def swa_bwd(q, k, v, dout, *, P: int, W: int, scale: float | None = None, heads=None, out=None,
             stream=None):
-    """Gradients (dq, dk, dv) of sum(dout * swa_fwd(q, k, v)); fp32. Heads outside the range
-    are zero."""
-    return _softmax_bwd(_lib.kta_swa_bwd, q, k, v, dout, P, W, None, scale, heads, stream)
+    """Gradients (dq, dk, dv) of sum(dout * swa_fwd(q, k, v)); fp32. Only the heads in range are
+    written (fresh buffers are zero elsewhere); out = (dq, dk, dv) reuses buffers."""
+    return _softmax_bwd(_lib.kta_swa_bwd, q, k, v, dout, P, W, None, scale, heads, out, stream)
 
 
 def dswa_bwd(q, k, v, dout, *, P: int, W: int, dil: int, scale: float | None = None, heads=None,
-             stream=None):
+             out=None, stream=None):
     """Gradients (dq, dk, dv) of sum(dout * dswa_fwd(q, k, v)); fp32."""
-    return _softmax_bwd(_lib.kta_dswa_bwd, q, k, v, dout, P, W, dil, scale, heads, stream)
+    return _softmax_bwd(_lib.kta_dswa_bwd, q, k, v, dout, P, W, dil, scale, heads, out, stream)
 
 
-def _linear_bwd(delta, q, k, v, alpha, beta, dout, scale, S0, heads, stream, erase_decayed):
+def _linear_bwd(delta, q, k, v, alpha, beta, dout, scale, S0, heads, out, stream, erase_decayed):
     for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout), ("alpha", alpha)):
         _need(t, n, torch.float32)
     if delta:
@@ -233,7 +244,7 @@ def _linear_bwd(delta, q, k, v, alpha, beta, dout, scale, S0, heads, stream, era
     B, N, Htot, d = q.shape
     h0, h1 = heads if heads is not None else (0, Htot)
     H = h1 - h0
-    dq, dk, dv = (torch.zeros_like(q) for _ in range(3))
+    dq, dk, dv = _grads(q, out)
     dalpha = torch.empty_like(alpha)
     dbeta = torch.empty_like(beta) if delta else None
     dS0 = torch.empty((B, H, d, d), device=q.device, dtype=torch.float32)
@@ -252,15 +263,17 @@ def _linear_bwd(delta, q, k, v, alpha, beta, dout, scale, S0, heads, stream, era
     return dq, dk, dv, dalpha, dS0
 
 
-def gla_bwd(q, k, v, alpha, dout, *, scale: float = 1.0, S0=None, heads=None, stream=None):
+def gla_bwd(q, k, v, alpha, dout, *, scale: float = 1.0, S0=None, heads=None, out=None,
+            stream=None):
     """Gradients (dq, dk, dv, dalpha, dS0) of sum(dout * gla_chunk_fwd(...)); fp32."""
-    return _linear_bwd(False, q, k, v, alpha, None, dout, scale, S0, heads, stream, False)
+    return _linear_bwd(False, q, k, v, alpha, None, dout, scale, S0, heads, out, stream, False)
 
 
 def gla_delta_bwd(q, k, v, alpha, beta, dout, *, scale: float = 1.0, S0=None, heads=None,
-                  stream=None, erase_decayed: bool = False):
+                  out=None, stream=None, erase_decayed: bool = False):
     """Gradients (dq, dk, dv, dalpha, dbeta, dS0) of sum(dout * gla_delta_fwd(...)); fp32."""
-    return _linear_bwd(True, q, k, v, alpha, beta, dout, scale, S0, heads, stream, erase_decayed)
+    return _linear_bwd(True, q, k, v, alpha, beta, dout, scale, S0, heads, out, stream,
+                       erase_decayed)
 
 
 def hybrid_cfg(*, B: int, F: int, P: int, d: int, dtype=torch.bfloat16, n_swa: int, n_dswa: int,

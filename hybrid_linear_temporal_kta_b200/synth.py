@@ -68,6 +68,9 @@ HYBRID_BF16 = Workload("hybrid_bf16_F21_P1560", B=1, F=21, P=1560, d=128, n_swa=
                        n_gla=8, W_swa=3, W_dswa=4, dil=3, chunk=64, seed_base=2000)
 DELTA_BF16 = Workload("gated_delta_bf16_B2_L65536", B=2, F=64, P=1024, d=128, n_swa=0,
                       n_dswa=0, n_gla=16, chunk=64, gla_delta=True, seed_base=3000)
+HYBRID_BWD_F32 = Workload("hybrid_bwd_f32_F21_P1560", B=1, F=21, P=1560, d=128, n_swa=8,
+                          n_dswa=8, n_gla=8, W_swa=3, W_dswa=4, dil=3, chunk=64, dtype="f32",
+                          seed_base=6000)
 STREAM_BF16 = Workload("stream_bf16_P880_F240", B=1, F=240, P=880, d=128, n_swa=8, n_dswa=8,
                        n_gla=8, W_swa=3, W_dswa=4, dil=3, chunk=64, seed_base=4000)
 
@@ -77,7 +80,8 @@ def sweep_workload(F: int) -> Workload:
     return HYBRID_BF16.replace(name=f"sweep_bf16_P1024_F{F}", F=F, P=1024, seed_base=5000)
 
 
-WORKLOADS = {w.name: w for w in (TINY_F32, HYBRID_BF16, DELTA_BF16, STREAM_BF16)}
+WORKLOADS = {w.name: w for w in (TINY_F32, HYBRID_BF16, DELTA_BF16, STREAM_BF16,
+                                  HYBRID_BWD_F32)}
 
 
 def torch_dtype(name: str) -> torch.dtype:
