@@ -348,8 +348,13 @@ struct LinBwdParams {
   int rows_b, N, H;
   float scale;
   int delta, erase_decayed;
-  int nck;             // stored states per (sequence, head) = ceil(N / BWD_CK)
-  float* ws;           // per (sequence, head): states [nck][D][D], chunk [BWD_CK][D][D], u, w
+  int seg_len, nseg;   // tokens per segment (a multiple of BWD_CK) and segments per sequence
+  int nck;             // stored states per segment = ceil(seg_len / BWD_CK)
+  float* ws;           // per (sequence, head, segment): states [nck][D][D], chunk
+                       // [BWD_CK][D][D], u, w
+  // vector GLA with nseg > 1 only, per (sequence, head, segment) [D][D] (key-major):
+  const float* Sin;    // state before the segment's first token
+  const float* Gin;    // adjoint entering the segment's last token from the right
 };
 
 template <int D>
@@ -357,9 +362,105 @@ __host__ __device__ constexpr long long lin_bwd_ws_floats(int nck) {
   return (static_cast<long long>(nck) + BWD_CK) * D * D + 2LL * BWD_CK * D;
 }
 
-// One CTA of D threads per (head, sequence). Thread j owns column j of the state in the
-// forward passes (registers) and of the adjoint G (shared memory); for the row reductions
-// (dq, dk, dalpha) thread i owns row i.
+// Segment summaries of the vector-GLA backward, one CTA of D threads per (segment, head,
+// sequence), thread j owning column j. From a zero state over the segment's tokens [t0, t1):
+//   E = the end state, c = prod_t alpha_t (all tokens), cx = prod_{t > t0} alpha_t,
+//   R = the adjoint at t0 from the segment's own outputs (G_t = scale q_t^T dO_t +
+//       diag(alpha_{t+1}) G_{t+1}, zero beyond t1 - 1).
+// sum: per (sequence, head, segment) E [D][D], R [D][D], c [D], cx [D].
+template <int D>
+__global__ void __launch_bounds__(D) gla_bwd_summary_kernel(const LinBwdParams p, float* sum) {
+  __shared__ float qv[D], kv[D], av[D];
+  const int j = threadIdx.x;
+  const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int t0 = seg * p.seg_len, t1 = min(p.N, t0 + p.seg_len);
+  const long long rb = static_cast<long long>(b) * p.rows_b;
+  float* E = sum + ((static_cast<long long>(b) * p.H + h) * p.nseg + seg) * (2LL * D * D + 2 * D);
+  float* R = E + D * D;
+  float* c = R + D * D;
+  float* cx = c + D;
+  float X[D];
+#pragma unroll
+  for (int i = 0; i < D; ++i) X[i] = 0.f;
+  float cj = 1.f, cxj = 1.f;
+  for (int t = t0; t < t1; ++t) {
+    const long long r = (rb + t) * p.ld + static_cast<long long>(h) * D;
+    __syncthreads();
+    kv[j] = p.k[r + j];
+    av[j] = p.alpha[((rb + t) * p.H + h) * D + j];
+    const float vj = p.v[r + j];
+    __syncthreads();
+    cj *= av[j];
+    if (t > t0) cxj *= av[j];
+#pragma unroll
+    for (int i = 0; i < D; ++i) X[i] = fmaf(av[i], X[i], kv[i] * vj);
+  }
+#pragma unroll
+  for (int i = 0; i < D; ++i) E[i * D + j] = X[i];
+  c[j] = cj;
+  cx[j] = cxj;
+#pragma unroll
+  for (int i = 0; i < D; ++i) X[i] = 0.f;
+  for (int t = t1 - 1; t >= t0; --t) {
+    const long long r = (rb + t) * p.ld + static_cast<long long>(h) * D;
+    __syncthreads();
+    qv[j] = p.q[r + j];
+    av[j] = p.alpha[((rb + t) * p.H + h) * D + j];
+    const float dj = p.dout[r + j] * p.scale;
+    __syncthreads();
+    if (t > t0) {
+#pragma unroll
+      for (int i = 0; i < D; ++i) X[i] = av[i] * fmaf(qv[i], dj, X[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < D; ++i) X[i] = fmaf(qv[i], dj, X[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < D; ++i) R[i * D + j] = X[i];
+}
+
+// Carry across segments, one thread per (sequence, head, i, j) state element:
+//   Sin_0 = S0, Sin_{s+1} = diag(c_s) Sin_s + E_s;
+//   Gfirst_{last} = R_{last}, Gin_s = diag(alpha_{t1(s)}) Gfirst_{s+1} (0 for the last segment),
+//   Gfirst_s = R_s + diag(cx_s) Gin_s;  dS0 = diag(alpha_0) Gfirst_0.
+// Sin and Gin are written into p.Sin / p.Gin (cast from const: the launcher owns them).
+template <int D>
+__global__ void gla_bwd_carry_kernel(const LinBwdParams p, const float* __restrict__ sum,
+                                     float* Sin, float* Gin) {
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= static_cast<long long>(p.H) * D * D) return;
+  const int b = blockIdx.y;
+  const int h = static_cast<int>(e / (D * D)), i = static_cast<int>((e / D) % D),
+            j = static_cast<int>(e % D);
+  const long long bh = static_cast<long long>(b) * p.H + h;
+  const long long rb = static_cast<long long>(b) * p.rows_b;
+  const long long stride = 2LL * D * D + 2 * D;
+  const float* base = sum + bh * p.nseg * stride;
+  float S = p.S0 ? p.S0[bh * D * D + i * D + j] : 0.f;
+  for (int s = 0; s < p.nseg; ++s) {
+    Sin[(bh * p.nseg + s) * D * D + i * D + j] = S;
+    const float* E = base + s * stride;
+    S = fmaf(E[2 * D * D + i], S, E[i * D + j]);
+  }
+  float Gf = 0.f;
+  for (int s = p.nseg - 1; s >= 0; --s) {
+    const float* E = base + s * stride;
+    float gin = 0.f;
+    if (s < p.nseg - 1) {
+      const long long t1 = static_cast<long long>(s + 1) * p.seg_len;
+      gin = p.alpha[((rb + t1) * p.H + h) * D + i] * Gf;
+    }
+    Gin[(bh * p.nseg + s) * D * D + i * D + j] = gin;
+    Gf = fmaf(E[2 * D * D + D + i], gin, E[D * D + i * D + j]);
+  }
+  if (p.dS0) p.dS0[bh * D * D + i * D + j] = p.alpha[(rb * p.H + h) * D + i] * Gf;
+}
+
+// One CTA of D threads per (head, sequence, segment). Thread j owns column j of the state in
+// the forward passes (registers) and of the adjoint G (shared memory); for the row reductions
+// (dq, dk, dalpha) thread i owns row i. A segment starts from p.Sin / p.Gin when they are
+// given, else from S0 / zero (one segment per sequence).
 template <int D>
 __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
   extern __shared__ float bsm[];
@@ -374,9 +475,11 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
   float* du = av + D;             // du_t (delta)
   float* red = du + D;            // [2][D] block reductions (delta)
   const int j = threadIdx.x;
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.y, seg = blockIdx.z;
   const long long bh = static_cast<long long>(b) * p.H + h;
-  float* ck = p.ws + bh * lin_bwd_ws_floats<D>(p.nck);
+  const long long bhs = bh * p.nseg + seg;
+  const int t_beg = seg * p.seg_len, t_end = min(p.N, t_beg + p.seg_len);
+  float* ck = p.ws + bhs * lin_bwd_ws_floats<D>(p.nck);
   float* buf = ck + static_cast<long long>(p.nck) * D * D;
   float* Ub = buf + static_cast<long long>(BWD_CK) * D * D;
   float* Wb = Ub + BWD_CK * D;
@@ -414,12 +517,17 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
     av[j] = p.delta ? (j == 0 ? gate_a(t, 0) : 0.f) : gate_a(t, j);
   };
 
-  // ---- forward: the state before every BWD_CK-th token
+  // ---- forward: the state before every BWD_CK-th token of the segment
+  if (p.Sin) {
 #pragma unroll
-  for (int i = 0; i < D; ++i) S[i] = p.S0 ? p.S0[bh * D * D + i * D + j] : 0.f;
-  for (int t = 0; t < p.N; ++t) {
-    if (t % BWD_CK == 0) {
-      float* c = ck + static_cast<long long>(t / BWD_CK) * D * D;
+    for (int i = 0; i < D; ++i) S[i] = p.Sin[bhs * D * D + i * D + j];
+  } else {
+#pragma unroll
+    for (int i = 0; i < D; ++i) S[i] = p.S0 ? p.S0[bh * D * D + i * D + j] : 0.f;
+  }
+  for (int t = t_beg; t < t_end; ++t) {
+    if ((t - t_beg) % BWD_CK == 0) {
+      float* c = ck + static_cast<long long>((t - t_beg) / BWD_CK) * D * D;
 #pragma unroll
       for (int i = 0; i < D; ++i) c[i * D + j] = S[i];
     }
@@ -429,10 +537,16 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
     step(t, 0, false);
   }
   // ---- reverse, one chunk of BWD_CK tokens at a time
+  if (p.Gin) {
 #pragma unroll
-  for (int i = 0; i < D; ++i) G[i * LDG + j] = 0.f;
-  for (int c = p.nck - 1; c >= 0; --c) {
-    const int t0 = c * BWD_CK, t1 = min(p.N, t0 + BWD_CK);
+    for (int i = 0; i < D; ++i) G[i * LDG + j] = p.Gin[bhs * D * D + i * D + j];
+  } else {
+#pragma unroll
+    for (int i = 0; i < D; ++i) G[i * LDG + j] = 0.f;
+  }
+  const int nck_here = (t_end - t_beg + BWD_CK - 1) / BWD_CK;
+  for (int c = nck_here - 1; c >= 0; --c) {
+    const int t0 = t_beg + c * BWD_CK, t1 = min(t_end, t0 + BWD_CK);
     const float* cs = ck + static_cast<long long>(c) * D * D;
 #pragma unroll
     for (int i = 0; i < D; ++i) S[i] = cs[i * D + j];
@@ -535,7 +649,7 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
       prv = tmp;
     }
   }
-  if (p.dS0) {
+  if (p.dS0 && p.nseg == 1) {
 #pragma unroll
     for (int i = 0; i < D; ++i) p.dS0[bh * D * D + i * D + j] = G[i * LDG + j];
   }

@@ -942,15 +942,52 @@ kta_status softmax_bwd_common(const void* q, const void* k, const void* v,
 
 template <int D>
 kta_status launch_lin_bwd(kta::LinBwdParams p, int B, cudaStream_t st) {
+  // Vector GLA splits each sequence into segments so that the launch has about one CTA per SM
+  // (the delta rule's segment carry would need dense d x d transitions: one segment).
+  const long long bh = static_cast<long long>(B) * p.H;
+  int nseg = 1;
+  long long seg_len = p.N;
+  if (!p.delta && bh < 148) {
+    const long long want = std::max<long long>(1, 148 / bh);
+    seg_len = ((p.N + want - 1) / want + kta::BWD_CK - 1) / kta::BWD_CK * kta::BWD_CK;
+    nseg = static_cast<int>((p.N + seg_len - 1) / seg_len);
+  }
+  if (nseg == 1) seg_len = p.N;
+  p.nseg = nseg;
+  p.seg_len = static_cast<int>(seg_len);
+  p.nck = static_cast<int>((seg_len + kta::BWD_CK - 1) / kta::BWD_CK);
+  const long long bhs = bh * nseg;
   const long long per = kta::lin_bwd_ws_floats<D>(p.nck);
+  const long long sum_per = 2LL * D * D + 2 * D;
+  const long long floats = bhs * per + (nseg > 1 ? bhs * (sum_per + 2LL * D * D) : 0);
   void* ws = nullptr;
-  kta_status r = workspace(static_cast<size_t>(per) * B * p.H * sizeof(float), st, &ws);
+  kta_status r = workspace(static_cast<size_t>(floats) * sizeof(float), st, &ws);
   if (r) return r;
   p.ws = static_cast<float*>(ws);
+  p.Sin = p.Gin = nullptr;
+  if (nseg > 1) {
+    float* sum = p.ws + bhs * per;
+    float* Sin = sum + bhs * sum_per;
+    float* Gin = Sin + bhs * D * D;
+    {
+      TraceScope ts("gla_bwd_summary_f32", st);
+      kta::gla_bwd_summary_kernel<D><<<dim3(nseg, p.H, B), D, 0, st>>>(p, sum);
+      KTA_CUDA(cudaGetLastError());
+    }
+    {
+      TraceScope ts("gla_bwd_carry_f32", st);
+      const long long n = static_cast<long long>(p.H) * D * D;
+      kta::gla_bwd_carry_kernel<D><<<dim3(static_cast<unsigned>((n + 255) / 256), B), 256, 0, st>>>(
+          p, sum, Sin, Gin);
+      KTA_CUDA(cudaGetLastError());
+    }
+    p.Sin = Sin;
+    p.Gin = Gin;
+  }
   const size_t smem = (3 * static_cast<size_t>(D) * (D + 1) + 8 * D) * sizeof(float);
   if ((r = set_smem_attr(kta::lin_bwd_f32_kernel<D>, smem))) return r;
   TraceScope ts(p.delta ? "delta_bwd_f32" : "gla_bwd_f32", st);
-  kta::lin_bwd_f32_kernel<D><<<dim3(p.H, B), D, smem, st>>>(p);
+  kta::lin_bwd_f32_kernel<D><<<dim3(p.H, B, nseg), D, smem, st>>>(p);
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
@@ -990,7 +1027,6 @@ kta_status lin_bwd_common(const void* q, const void* k, const void* v, const flo
   p.scale = scale;
   p.delta = delta ? 1 : 0;
   p.erase_decayed = erase_decayed ? 1 : 0;
-  p.nck = static_cast<int>((N + kta::BWD_CK - 1) / kta::BWD_CK);
   if (N == 0) return KTA_OK;
   cudaStream_t st = as_stream(stream);
   if (s.d == 32) return launch_lin_bwd<32>(p, s.B, st);

@@ -70,11 +70,14 @@ def test_softmax_backward_parity(kta, d, F, P, W, dil, dilated, heads, Htot):
         assert np.all(gn[:, :, :h0] == 0) and np.all(gn[:, :, h1:] == 0), f"{name} outside heads"
 
 
-@pytest.mark.parametrize("d,N,with_s0", [(32, 45, False), (64, 100, True), (128, 161, True),
-                                         (128, 1000, False)])
-def test_gla_backward_parity(kta, d, N, with_s0):
-    rng = np.random.default_rng(200 + d + N)
-    B, Htot, heads = 2, 3, (1, 3)
+# B * H < 148 splits each sequence into segments (about one CTA per SM, 32-token multiples,
+# ragged last segment); the last case has B * H >= 148 and runs one segment per sequence.
+@pytest.mark.parametrize("d,N,with_s0,B,Htot,heads", [
+    (32, 45, False, 2, 3, (1, 3)), (64, 100, True, 2, 3, (1, 3)), (128, 161, True, 2, 3, (1, 3)),
+    (128, 1000, False, 2, 3, (1, 3)), (128, 1000, True, 1, 1, (0, 1)),
+    (32, 40, True, 1, 150, (0, 150))])
+def test_gla_backward_parity(kta, d, N, with_s0, B, Htot, heads):
+    rng = np.random.default_rng(200 + d + N + Htot)
     H = heads[1] - heads[0]
     q, k, v = qkv(rng, B, N, Htot, d)
     k *= d ** -0.5
