@@ -76,10 +76,14 @@ def _load():
             lib.oracle_delta_bwd.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p,
                                              _f64p, _f64p, _f64p, _f64p, _f64p, _f64p] + [
                 _int] * 6 + [ctypes.c_double, _int]
+            lib.oracle_proj.argtypes = [_f32p, _f32p, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_int64, _i64p, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_int64, _f64p]
             lib.oracle_set_threads.argtypes = [_int]
             lib.oracle_get_threads.restype = _int
             for name in ("oracle_swa", "oracle_dswa", "oracle_gla", "oracle_delta",
-                         "oracle_softmax_bwd", "oracle_gla_bwd", "oracle_delta_bwd"):
+                         "oracle_softmax_bwd", "oracle_gla_bwd", "oracle_delta_bwd",
+                         "oracle_proj"):
                 getattr(lib, name).restype = _int
             _lib = lib
     return _lib
@@ -273,6 +277,28 @@ def delta_bwd(q, k, v, alpha, beta, dout, scale: float = 1.0, S0=None, heads=Non
                                   h1, float(scale), int(bool(erase_decayed)))
     _check(rc, "delta_bwd")
     return dq, dk, dv, da, db, dS0
+
+
+def proj(x, w, rows=None, sigmoid_cols=None) -> np.ndarray:
+    """The projections (q = W_Q x, ..., beta = sigmoid(W_beta x)) as one product: x [..., K]
+    (M rows), w [N, K] -> y [rows, N] float64, y = x w^T with columns in sigmoid_cols = (c0, c1)
+    passed through the logistic sigmoid. rows: indices of the rows of x to compute (all if
+    None)."""
+    x = _f32(x)
+    K = x.shape[-1]
+    x2 = x.reshape(-1, K)
+    w = _f32(w)
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("w must be [N, K]")
+    r, nr = _rows(rows)
+    R = nr if r is not None else x2.shape[0]
+    y = np.empty((R, N))
+    c0, c1 = sigmoid_cols if sigmoid_cols is not None else (0, 0)
+    rc = _load().oracle_proj(_p(x2, _f32p), _p(w, _f32p), x2.shape[0], N, K,
+                             None if r is None else _p(r, _i64p), nr, c0, c1, _p(y, _f64p))
+    _check(rc, "proj")
+    return y
 
 
 def visible(t, s, P: int, W: int, dil: int = 1, dilated: bool = False) -> np.ndarray:
