@@ -76,7 +76,7 @@ def _load():
             lib.oracle_delta_bwd.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p,
                                              _f64p, _f64p, _f64p, _f64p, _f64p, _f64p] + [
                 _int] * 6 + [ctypes.c_double, _int]
-            lib.oracle_proj.argtypes = [_f32p, _f32p, ctypes.c_int64, ctypes.c_int64,
+            lib.oracle_proj.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int64,
                                         ctypes.c_int64, _i64p, ctypes.c_int64, ctypes.c_int64,
                                         ctypes.c_int64, _f64p]
             lib.oracle_set_threads.argtypes = [_int]
@@ -279,11 +279,11 @@ def delta_bwd(q, k, v, alpha, beta, dout, scale: float = 1.0, S0=None, heads=Non
     return dq, dk, dv, da, db, dS0
 
 
-def proj(x, w, rows=None, sigmoid_cols=None) -> np.ndarray:
+def proj(x, w, rows=None, sigmoid_cols=None, bias=None) -> np.ndarray:
     """The projections (q = W_Q x, ..., beta = sigmoid(W_beta x)) as one product: x [..., K]
     (M rows), w [N, K] -> y [rows, N] float64, y = x w^T with columns in sigmoid_cols = (c0, c1)
     passed through the logistic sigmoid. rows: indices of the rows of x to compute (all if
-    None)."""
+    None). bias: optional [N] offsets added to every row before the sigmoid."""
     x = _f32(x)
     K = x.shape[-1]
     x2 = x.reshape(-1, K)
@@ -295,8 +295,12 @@ def proj(x, w, rows=None, sigmoid_cols=None) -> np.ndarray:
     R = nr if r is not None else x2.shape[0]
     y = np.empty((R, N))
     c0, c1 = sigmoid_cols if sigmoid_cols is not None else (0, 0)
-    rc = _load().oracle_proj(_p(x2, _f32p), _p(w, _f32p), x2.shape[0], N, K,
-                             None if r is None else _p(r, _i64p), nr, c0, c1, _p(y, _f64p))
+    b = None if bias is None else _f32(bias)
+    if b is not None and b.shape != (N,):
+        raise ValueError("bias must be [N]")
+    rc = _load().oracle_proj(_p(x2, _f32p), _p(w, _f32p), None if b is None else _p(b, _f32p),
+                             x2.shape[0], N, K, None if r is None else _p(r, _i64p), nr, c0, c1,
+                             _p(y, _f64p))
     _check(rc, "proj")
     return y
 

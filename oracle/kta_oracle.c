@@ -494,10 +494,11 @@ int oracle_delta_bwd(const float* q, const float* k, const float* v, const float
  * paper-read, section 2, second pillar, GLA paragraph: q_t = W_Q x_t, k_t = W_K x_t,
  * v_t = W_V x_t and beta_t = sigmoid(W_beta x_t); the forget gate alpha_t is likewise a sigmoid
  * of a projection of x_t. With every weight stacked as the rows of one matrix w [N][K], row r of
- * the result is y[r][n] = sum_k x[r][k] w[n][k]; columns in [sig_c0, sig_c1) then pass through
- * the logistic sigmoid 1 / (1 + exp(-y)). rows (nrows entries) selects which rows of x to
+ * the result is y[r][n] = sum_k x[r][k] w[n][k] (+ bias[n] when a bias is given: the caller's
+ * gate offset, not a page term); columns in [sig_c0, sig_c1) then pass through the logistic
+ * sigmoid 1 / (1 + exp(-y)). rows (nrows entries) selects which rows of x to
  * compute, NULL = all M rows; y holds one output row per selected row. */
-int oracle_proj(const float* x, const float* w, int64_t M, int64_t N, int64_t K,
+int oracle_proj(const float* x, const float* w, const float* bias, int64_t M, int64_t N, int64_t K,
                 const int64_t* rows, int64_t nrows, int64_t sig_c0, int64_t sig_c1, double* y) {
   if (!x || !w || !y || M < 1 || N < 1 || K < 1) return 1;
   const int64_t R = rows ? nrows : M;
@@ -510,6 +511,7 @@ int oracle_proj(const float* x, const float* w, int64_t M, int64_t N, int64_t K,
       const float* wr = w + n * K;
       double acc = 0.0;
       for (int64_t c = 0; c < K; ++c) acc += (double)xr[c] * (double)wr[c];
+      if (bias) acc += (double)bias[n];
       if (n >= sig_c0 && n < sig_c1) acc = 1.0 / (1.0 + exp(-acc));
       y[i * N + n] = acc;
     }

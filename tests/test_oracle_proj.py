@@ -52,3 +52,15 @@ def test_stacked_weights_and_row_selection():
     np.testing.assert_array_equal(y[:, 4:], oracle.proj(x, wk))
     rows = [8, 0, 3]
     np.testing.assert_array_equal(oracle.proj(x, wq, rows=rows), oracle.proj(x, wq)[rows])
+
+
+def test_bias_shifts_logits_before_the_sigmoid():
+    x = grid((4, 8))
+    w = grid((3, 8))
+    w[1] = 0.0
+    b = np.array([0.5, 3.0, -1.25], dtype=np.float32)
+    y = oracle.proj(x, w, sigmoid_cols=(1, 3), bias=b)
+    raw = oracle.proj(x, w)
+    np.testing.assert_array_equal(y[:, 0], raw[:, 0] + 0.5)
+    np.testing.assert_allclose(y[:, 1], 1.0 / (1.0 + np.exp(-3.0)), rtol=0, atol=1e-16)
+    np.testing.assert_allclose(y[:, 2], 1.0 / (1.0 + np.exp(-(raw[:, 2] - 1.25))), rtol=1e-15)
