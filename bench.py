@@ -44,13 +44,15 @@ def parse_args():
                          "headline line is the default, 21 frames)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="profiling only: override the delta workload's tokens per sequence")
-    ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep", "backward"),
+    ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep", "backward",
+                                           "layer"),
                     default="hybrid",
                     help="hybrid: the 21-frame hybrid layer (the headline line); delta: gated "
                          "delta rule, 2 x 65,536 tokens x 16 heads; stream: 240-frame rollout one "
                          "frame per call; sweep: hybrid layer vs full frame-causal attention for "
                          "F = 8..256 frames of 1,024 tokens (one line per F); backward: the "
-                         "hybrid layer's reverse mode in fp32")
+                         "hybrid layer's reverse mode in fp32; layer: input projections + hybrid "
+                         "operator + output projection")
     return ap.parse_args()
 
 
@@ -89,6 +91,13 @@ def softmax_bwd_flops(w) -> dict:
     the dq kernel forms S, dP and dQ (6d), the key-major kernel S, dP, dV and dK (8d)."""
     n = visible_pairs(w)
     return {"softmax_bwd_q_f32": 6.0 * w.d * n, "softmax_bwd_kv_f32": 8.0 * w.d * n}
+
+
+def layer_proj_flops(w) -> float:
+    """Projection FLOPs of one layer step with model width C = H d: the stacked q/k/v/alpha
+    product (3 H d + n_gla d outputs) and the output projection (C outputs), 2 per MAC."""
+    C = w.H * w.d
+    return 2.0 * w.B * w.N * C * (3 * w.H * w.d + w.n_gla * w.d) + 2.0 * w.B * w.N * C * C
 
 
 def fp32_alu_tflops(sm_mhz: float) -> float:
@@ -592,6 +601,49 @@ def run_other(args):
                          "achieved": fl[top] / (k_ms / 1e3) / 1e12, "peak": peak,
                          "frac": fl[top] / (k_ms / 1e3) / 1e12 / peak,
                          "peak_source": f"fp32 FMA lanes x median SM clock {sm_mhz:.0f} MHz"},
+            "clocks": clocks, "kernels": kern})
+    elif args.workload == "layer":
+        w = synth.HYBRID_BF16
+        C, hd = w.H * w.d, w.H * w.d
+        g = torch.Generator(device="cuda")
+        g.manual_seed(w.seed_base + 7)
+        x = torch.randn((w.B, w.N, C), generator=g, device="cuda").to(torch.bfloat16)
+        n_in = 3 * hd + w.n_gla * w.d
+        w_in = (torch.randn((n_in, C), generator=g, device="cuda") * C ** -0.5).to(torch.bfloat16)
+        w_out = (torch.randn((C, hd), generator=g, device="cuda") * hd ** -0.5).to(torch.bfloat16)
+        # alpha = sigmoid(W_alpha x + mu) with W_alpha x ~ N(0, 1): the input recipe's gates
+        gate_bias = torch.full((w.n_gla * w.d,), w.alpha_mu, device="cuda")
+        cfg = kta.cfg_from_workload(w)
+        o = torch.empty((w.B, w.N, w.H, w.d), device="cuda", dtype=torch.bfloat16)
+        y = torch.empty((w.B, w.N, C), device="cuda", dtype=torch.bfloat16)
+
+        def step():
+            q, k, v, a, _ = kta.qkv_gate_proj(x, w_in, H=w.H, d=w.d, n_gla=w.n_gla,
+                                              gate_bias=gate_bias)
+            kta.hybrid_fwd(cfg, q, k, v, a, out=o)
+            kta.linear(o.view(w.B, w.N, hd), w_out, out=y)
+        clk = ClockSampler("0")
+        clk.start()
+        ms = _device_ms(step, args.steps, args.warmup)
+        clocks = clk.stop() or {}
+        kern = _traced(step, args.steps)
+        pf = layer_proj_flops(w)
+        k_ms = kern["proj_gemm"]["ms_per_step"]
+        tc_s = float(peaks.get("bf16_tflops_sustained", tc))
+        lines.append({
+            "workload": "layer_bf16_F21_P1560_C3072", "unit": "tokens/s",
+            "metric": "attention layer fwd tokens/s (q/k/v/gate projection + hybrid operator + "
+                      "output projection)",
+            "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
+            "dtype": "bf16",
+            "config": {"B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d, "C": C,
+                       "proj_outputs": n_in},
+            "roofline": {"kernel": "proj_gemm", "bound": "tensor", "unit": "TFLOP/s",
+                         "algorithmic_tflop": pf / 1e12,
+                         "achieved": pf / (k_ms / 1e3) / 1e12, "peak": tc,
+                         "frac": pf / (k_ms / 1e3) / 1e12 / tc,
+                         "frac_of_sustained": pf / (k_ms / 1e3) / 1e12 / tc_s,
+                         "peak_source": peaks_kind},
             "clocks": clocks, "kernels": kern})
     else:  # sweep
         for F in (8, 16, 32, 64, 128, 256):

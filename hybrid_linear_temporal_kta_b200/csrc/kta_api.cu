@@ -22,6 +22,7 @@
 #include "gla_chunk.cuh"
 #include "delta_chunk.cuh"
 #include "bwd_f32.cuh"
+#include "proj_gemm.cuh"
 
 namespace {
 
@@ -1034,9 +1035,78 @@ kta_status lin_bwd_common(const void* q, const void* k, const void* v, const flo
   return launch_lin_bwd<128>(p, s.B, st);
 }
 
+int sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!n[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1)
+      v = 148;
+    n[dev] = v;
+  }
+  return n[dev];
+}
+
 }  // namespace
 
 extern "C" {
+
+kta_status kta_proj_fwd(const void* x, const void* w, int M, int N, int K,
+                        const kta_proj_seg* segs, int nseg, void* stream) {
+  if (!x || !w || !segs) return fail(KTA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(w)) return fail(KTA_ERR_ALIGNMENT, "x and w must be 16-byte aligned");
+  if (M < 1 || N < 1 || K < 1) return fail(KTA_ERR_INVALID_ARG, "M, N, K must be >= 1");
+  if (K % 8) return fail(KTA_ERR_ALIGNMENT, "K must be a multiple of 8 (16-byte rows)");
+  if (nseg < 1 || nseg > kta::PG_MAXSEG)
+    return fail(KTA_ERR_INVALID_ARG, "nseg must be in [1, %d]", kta::PG_MAXSEG);
+  kta::ProjParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nseg = nseg;
+  for (int i = 0; i < nseg; ++i) {
+    const kta_proj_seg& g = segs[i];
+    if (g.col_begin < 0 || g.col_end > N || g.col_begin >= g.col_end)
+      return fail(KTA_ERR_INVALID_ARG, "segment %d: need 0 <= col_begin < col_end <= N", i);
+    if (!g.dst) return fail(KTA_ERR_INVALID_ARG, "segment %d: null dst", i);
+    if (g.mode < KTA_PROJ_BF16 || g.mode > KTA_PROJ_F32)
+      return fail(KTA_ERR_INVALID_ARG, "segment %d: bad mode", i);
+    if (g.ld < g.col_end - g.col_begin)
+      return fail(KTA_ERR_INVALID_ARG, "segment %d: ld smaller than its width", i);
+    for (int j = 0; j < i; ++j)
+      if (g.col_begin < segs[j].col_end && segs[j].col_begin < g.col_end)
+        return fail(KTA_ERR_INVALID_ARG, "segments %d and %d overlap", j, i);
+    kta::ProjSeg& d = p.seg[i];
+    d.c0 = g.col_begin;
+    d.c1 = g.col_end;
+    d.dst = g.dst;
+    d.ld = g.ld;
+    d.mode = g.mode;
+    d.bias = g.bias;
+    const long long esz = g.mode == KTA_PROJ_BF16 ? 2 : 4;
+    d.vec = aligned16(g.dst) && (g.ld * esz) % 16 == 0 && (!g.bias || aligned16(g.bias));
+  }
+  CUtensorMap ta, tb;
+  const cuuint64_t sK[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint64_t dA[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint32_t bA[2] = {kta::PG_BK, kta::PG_BM};
+  const cuuint64_t dB[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
+  const cuuint32_t bB[2] = {kta::PG_BK, kta::PG_BN};
+  kta_status r;
+  if ((r = make_map_nd(&ta, x, 2, dA, sK, bA)) || (r = make_map_nd(&tb, w, 2, dB, sK, bB)))
+    return r;
+  const size_t smem = kta::proj_smem_bytes();
+  if ((r = set_smem_attr(kta::proj_gemm_kernel, smem))) return r;
+  const long long tiles = static_cast<long long>((M + kta::PG_BM - 1) / kta::PG_BM) *
+                          ((N + kta::PG_BN - 1) / kta::PG_BN);
+  const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
+  cudaStream_t st = as_stream(stream);
+  TraceScope ts("proj_gemm", st);
+  kta::proj_gemm_kernel<<<grid, 192, smem, st>>>(ta, tb, p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
 
 kta_status kta_swa_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq,
                        void* dk, void* dv, kta_shape s, int H, int ld_heads, int W, float scale,

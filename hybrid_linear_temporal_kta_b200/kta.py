@@ -31,6 +31,14 @@ class Shape(ctypes.Structure):
                 ("dtype", ctypes.c_int)]
 
 
+class ProjSeg(ctypes.Structure):
+    _fields_ = [("col_begin", ctypes.c_int), ("col_end", ctypes.c_int), ("dst", ctypes.c_void_p),
+                ("ld", ctypes.c_longlong), ("mode", ctypes.c_int), ("bias", ctypes.c_void_p)]
+
+
+PROJ_BF16, PROJ_SIGMOID_F32, PROJ_F32 = 0, 1, 2
+
+
 class HybridCfg(ctypes.Structure):
     _fields_ = [("s", Shape), ("n_swa", ctypes.c_int), ("n_dswa", ctypes.c_int),
                 ("n_gla", ctypes.c_int), ("W_swa", ctypes.c_int), ("W_dswa", ctypes.c_int),
@@ -55,6 +63,7 @@ _SIGS = {
     "kta_gla_chunk_fwd_noalloc": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
                                   _st),
     "kta_hybrid_fwd": ([ctypes.POINTER(HybridCfg), _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
+    "kta_proj_fwd": ([_vp, _vp, _i, _i, _i, ctypes.POINTER(ProjSeg), _i, _vp], _st),
     "kta_swa_bwd": ([_vp] * 7 + [Shape, _i, _i, _i, _f, _vp], _st),
     "kta_dswa_bwd": ([_vp] * 7 + [Shape, _i, _i, _i, _i, _f, _vp], _st),
     "kta_gla_bwd": ([_vp, _vp, _vp, _fp, _fp, _vp, _vp, _vp, _vp, _fp, _fp, Shape, _i, _i, _f,
@@ -193,6 +202,72 @@ def gla_delta_fwd(q, k, v, alpha, beta, *, chunk: int = 64, scale: float = 1.0, 
     erase_decayed: the GatedDeltaNet form M = alpha M (I - beta k k^T) + beta v k^T."""
     return _linear(True, q, k, v, alpha, beta, chunk, scale, S0, return_state, heads, out, stream,
                    erase_decayed)
+
+
+def proj_fwd(x, w, segs, stream=None):
+    """Y = x w^T on the tensor cores, routed by column ranges. x [..., K] bf16 (M rows), w [N, K]
+    bf16; segs: list of (col_begin, col_end, dst tensor, mode[, bias]) with mode PROJ_BF16 (dst
+    bf16), PROJ_SIGMOID_F32 or PROJ_F32 (dst fp32) and an optional fp32 bias of the range's width;
+    dst row r holds columns [col_begin, col_end) of row r (dst viewed as [M, -1])."""
+    _need(x, "x", torch.bfloat16)
+    _need(w, "w", torch.bfloat16)
+    K = x.shape[-1]
+    M = x.numel() // K
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("w must be [N, K] with K = x.shape[-1]")
+    arr = (ProjSeg * len(segs))()
+    for i, sg in enumerate(segs):
+        c0, c1, dst, mode = sg[:4]
+        bias = sg[4] if len(sg) > 4 else None
+        _need(dst, f"segment {i} dst", torch.bfloat16 if mode == PROJ_BF16 else torch.float32)
+        if dst.numel() % M:
+            raise ValueError(f"segment {i}: dst does not have M = {M} rows")
+        if bias is not None:
+            _need(bias, f"segment {i} bias", torch.float32)
+            if bias.numel() != c1 - c0:
+                raise ValueError(f"segment {i}: bias must have {c1 - c0} entries")
+        arr[i] = ProjSeg(c0, c1, dst.data_ptr(), dst.numel() // M, mode,
+                         None if bias is None else bias.data_ptr())
+    _check(_lib.kta_proj_fwd(_ptr(x), _ptr(w), M, N, K, arr, len(segs), _stream(stream)),
+           "kta_proj_fwd")
+
+
+def linear(x, w, *, out=None, stream=None):
+    """x [..., K] bf16 times w [N, K]^T -> [..., N] bf16 (e.g. the output projection)."""
+    y = torch.empty(x.shape[:-1] + (w.shape[0],), device=x.device, dtype=torch.bfloat16) \
+        if out is None else out
+    proj_fwd(x, w, [(0, w.shape[0], y, PROJ_BF16)], stream)
+    return y
+
+
+def qkv_gate_proj(x, w, *, H: int, d: int, n_gla: int, gla_delta: bool = False, gate_bias=None,
+                  stream=None):
+    """One launch for every input of hybrid_fwd: x [B, N, C] bf16 and the stacked weight
+    w = [W_Q; W_K; W_V; W_alpha (; W_beta)] ([3 H d + n_gla d, C] for vector GLA,
+    [3 H d + 2 n_gla, C] for the delta rule). Returns q, k, v [B, N, H, d] bf16 and
+    alpha = sigmoid(W_alpha x) ([B, N, n_gla, d] or [B, N, n_gla] fp32), beta = sigmoid(W_beta x)
+    ([B, N, n_gla] fp32, delta rule only, else None). gate_bias: optional fp32 offsets of the
+    alpha logits (one per alpha column)."""
+    B, N, _ = x.shape
+    hd = H * d
+    q, k, v = (torch.empty((B, N, H, d), device=x.device, dtype=torch.bfloat16)
+               for _ in range(3))
+    segs = [(0, hd, q, PROJ_BF16), (hd, 2 * hd, k, PROJ_BF16), (2 * hd, 3 * hd, v, PROJ_BF16)]
+    alpha = beta = None
+    if n_gla:
+        ga = n_gla if gla_delta else n_gla * d
+        alpha = torch.empty((B, N, n_gla) if gla_delta else (B, N, n_gla, d), device=x.device,
+                            dtype=torch.float32)
+        segs.append((3 * hd, 3 * hd + ga, alpha, PROJ_SIGMOID_F32, gate_bias))
+        if gla_delta:
+            beta = torch.empty((B, N, n_gla), device=x.device, dtype=torch.float32)
+            segs.append((3 * hd + ga, 3 * hd + 2 * ga, beta, PROJ_SIGMOID_F32))
+    want = segs[-1][1]
+    if w.shape[0] != want:
+        raise ValueError(f"stacked weight must have {want} rows, got {w.shape[0]}")
+    proj_fwd(x, w, segs, stream)
+    return q, k, v, alpha, beta
 
 
 def _grads(q, out):

@@ -185,6 +185,35 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
                           const float* alpha, const float* beta, void* o, void* stream);
 
 /*
+ * Projections around the operator -- paper-read, section 2, second pillar, GLA paragraph:
+ * q_t = W_Q x_t, k_t = W_K x_t, v_t = W_V x_t, beta_t = sigmoid(W_beta x_t), the forget gate
+ * alpha_t likewise a sigmoid of a projection of x_t, and the output projection of the mixed
+ * heads. kta_proj_fwd computes Y = X W^T on the tensor cores:
+ *   x: [M][K] bf16 (row-major), w: [N][K] bf16 (one row per output column, the layout of a
+ *   linear layer's weight), fp32 accumulation. K % 8 == 0; x and w 16-byte aligned.
+ * and writes column ranges of Y through `segs` (1..8 non-overlapping ranges; columns outside
+ * every range are dropped): row r, column c of range s goes to dst_s[r * ld_s + (c - col_begin_s)]
+ * as bf16 (KTA_PROJ_BF16), sigmoid(Y) in fp32 (KTA_PROJ_SIGMOID_F32) or Y in fp32 (KTA_PROJ_F32),
+ * after adding bias_s[c - col_begin_s] when the range has a bias (fp32, device; NULL = none; a
+ * gate's offset, e.g. one that keeps forget gates near 1, which the pages' bias-free
+ * projections leave to the caller).
+ * With W = [W_Q; W_K; W_V; W_alpha; W_beta] one call produces every input of kta_hybrid_fwd.
+ * Outputs must not overlap x or w.
+ */
+typedef enum { KTA_PROJ_BF16 = 0, KTA_PROJ_SIGMOID_F32 = 1, KTA_PROJ_F32 = 2 } kta_proj_mode;
+
+typedef struct {
+  int col_begin, col_end;   /* columns [col_begin, col_end) of Y */
+  void* dst;                /* device pointer */
+  long long ld;             /* row stride of dst in elements (>= col_end - col_begin) */
+  int mode;                 /* kta_proj_mode */
+  const float* bias;        /* [col_end - col_begin] fp32 device array, or NULL */
+} kta_proj_seg;
+
+kta_status kta_proj_fwd(const void* x, const void* w, int M, int N, int K,
+                        const kta_proj_seg* segs, int nseg, void* stream);
+
+/*
  * Reverse mode (training). The pages define only the forward operators (paper-read, section 2,
  * second pillar); these entry points give the gradients of L = sum(dout * o) for the o of the
  * matching forward call, in fp32 on CUDA cores: s.dtype must be KTA_F32, else
