@@ -763,11 +763,15 @@ static kta_status check_cfg(const kta_hybrid_cfg* c) {
   return check_heads(H, H, c->s);
 }
 
-kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* k, const void* v,
-                          const float* alpha, const float* beta, void* o, void* stream) {
+static kta_status hybrid_common(const kta_hybrid_cfg* cfg, int f0, const void* q, const void* k,
+                                const void* v, const float* alpha, const float* beta,
+                                const float* S0, float* S_out, void* o, void* stream) {
   kta_status r;
   if ((r = check_cfg(cfg)) || (r = check_ptrs({q, k, v, o}))) return r;
   const kta_shape& s = cfg->s;
+  if (f0 < 0 || f0 >= s.F) return fail(KTA_ERR_INVALID_ARG, "need 0 <= f0 < F (got f0 = %d)", f0);
+  if (f0 > 0 && s.B != 1)
+    return fail(KTA_ERR_UNSUPPORTED, "a query-frame offset f0 > 0 needs B == 1");
   const int H = cfg->n_swa + cfg->n_dswa + cfg->n_gla;
   if (cfg->n_gla > 0) {
     if (!alpha || (cfg->gla_delta && !beta)) return fail(KTA_ERR_INVALID_ARG, "null gate pointer");
@@ -778,6 +782,9 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
   cudaStream_t st = as_stream(stream);
 
   WinLaunch W = seq_win_launch(q, k, v, o, s, H, cfg->scale_softmax);
+  W.Fq = s.F - f0;  // query frames f0 .. F-1 of the key / value frames
+  W.f_base = f0;
+  W.q_rows_b = W.Fq * s.P;
   W.g[0] = seq_group(k, v, s, cfg->n_swa, cfg->n_swa + cfg->n_dswa, H, cfg->W_swa, 1);
   W.g[1] = seq_group(k, v, s, cfg->n_dswa, cfg->n_swa + cfg->n_dswa, H, cfg->W_dswa, cfg->dil);
   if (cfg->n_swa == 0) {  // DSWA heads only: make them group 0
@@ -787,7 +794,7 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
 
   LinLaunch L;
   L.B = s.B;
-  L.N = s.F * s.P;
+  L.N = (s.F - f0) * s.P;
   L.H = cfg->n_gla;
   L.d = s.d;
   L.rows_b = L.N;
@@ -795,13 +802,16 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
   L.dt = s.dtype;
   const size_t hoff = static_cast<size_t>(cfg->n_swa + cfg->n_dswa) * s.d * es;
   L.q = static_cast<const char*>(q) + hoff;
-  L.k = static_cast<const char*>(k) + hoff;
-  L.v = static_cast<const char*>(v) + hoff;
+  const size_t koff = static_cast<size_t>(f0) * s.P * ld * es;  // the query frames' keys
+  L.k = static_cast<const char*>(k) + koff + hoff;
+  L.v = static_cast<const char*>(v) + koff + hoff;
   L.o = static_cast<char*>(o) + hoff;
   L.ld = ld;
   L.alpha = alpha;
   L.beta = beta;
   L.scale = cfg->scale_gla;
+  L.S0 = S0;
+  L.S_out = S_out;
   L.delta = cfg->gla_delta != 0;
   L.erase_decayed = cfg->gla_delta == 2;
 
@@ -822,6 +832,32 @@ kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* 
   KTA_CUDA(cudaStreamWaitEvent(st, ts->join, 0));
   if (r_win) return r_win;
   return r_lin;
+}
+
+kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* beta, void* o, void* stream) {
+  return hybrid_common(cfg, 0, q, k, v, alpha, beta, nullptr, nullptr, o, stream);
+}
+
+kta_status kta_hybrid_fwd_window(const kta_hybrid_cfg* cfg, int f0, const void* q, const void* k,
+                                 const void* v, const float* alpha, const float* beta,
+                                 const float* S0, float* S_out, void* o, void* stream) {
+  if ((S0 && !aligned16(S0)) || (S_out && !aligned16(S_out)))
+    return fail(KTA_ERR_ALIGNMENT, "S0 / S_out not 16-byte aligned");
+  return hybrid_common(cfg, f0, q, k, v, alpha, beta, S0, S_out, o, stream);
+}
+
+kta_status kta_state_affine(const float* A, const float* X, const float* E, float* Y, int n, int d,
+                            void* stream) {
+  if (!A || !X || !Y) return fail(KTA_ERR_INVALID_ARG, "null pointer");
+  if (n < 1 || d < 1 || d > 4096) return fail(KTA_ERR_INVALID_ARG, "need n >= 1 and 1 <= d <= 4096");
+  if (Y == A || Y == X) return fail(KTA_ERR_INVALID_ARG, "Y must not alias A or X");
+  cudaStream_t st = as_stream(stream);
+  const dim3 grid((d + 31) / 32, (d + 31) / 32, n);
+  TraceScope ts("state_affine", st);
+  kta::state_affine_kernel<<<grid, dim3(32, 8), 0, st>>>(A, X, E, Y, d);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
 }
 
 // --------------------------------------------------------------------------- streaming

@@ -189,4 +189,43 @@ __global__ void __launch_bounds__(D) delta_rec_f32_kernel(const float* __restric
   }
 }
 
+// Y_m = A_m X_m (+ E_m) for m < gridDim.z, d x d fp32 row-major matrices: the composition of two
+// affine state maps (a segment's transition applied to the state entering it, plus the state the
+// segment builds from zero). A 32 x 32 output tile per CTA of 32 x 8 threads, both operands staged
+// through shared memory in 32-wide K steps.
+__global__ void __launch_bounds__(256) state_affine_kernel(const float* __restrict__ A,
+                                                           const float* __restrict__ X,
+                                                           const float* __restrict__ E,
+                                                           float* __restrict__ Y, int d) {
+  __shared__ float as[32][33], xs[32][33];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int col = blockIdx.x * 32 + tx, row0 = blockIdx.y * 32;
+  const long long off = static_cast<long long>(blockIdx.z) * d * d;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < d; k0 += 32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 8 * i;
+      as[r][tx] = (row0 + r < d && k0 + tx < d) ? A[off + (row0 + r) * static_cast<long long>(d) + k0 + tx] : 0.f;
+      xs[r][tx] = (k0 + r < d && col < d) ? X[off + (k0 + r) * static_cast<long long>(d) + col] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 32; ++kk) {
+      const float xv = xs[kk][tx];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(as[ty + 8 * i][kk], xv, acc[i]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = row0 + ty + 8 * i;
+    if (r < d && col < d) {
+      const long long e = off + static_cast<long long>(r) * d + col;
+      Y[e] = acc[i] + (E ? E[e] : 0.f);
+    }
+  }
+}
+
 }  // namespace kta

@@ -70,6 +70,9 @@ _SIGS = {
                      _vp], _st),
     "kta_gla_delta_bwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, _vp, _vp, _vp, _fp, _fp, _fp, Shape,
                            _i, _i, _f, _i, _vp], _st),
+    "kta_hybrid_fwd_window": ([ctypes.POINTER(HybridCfg), _i, _vp, _vp, _vp, _fp, _fp, _fp, _fp,
+                               _vp, _vp], _st),
+    "kta_state_affine": ([_fp, _fp, _fp, _fp, _i, _i, _vp], _st),
     "kta_stream_create": ([ctypes.POINTER(HybridCfg), ctypes.POINTER(_vp)], _st),
     "kta_stream_step": ([_vp, _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
     "kta_stream_reset": ([_vp, _vp], _st),
@@ -377,6 +380,39 @@ def hybrid_fwd(cfg: HybridCfg, q, k, v, alpha=None, beta=None, *, out=None, stre
     _check(_lib.kta_hybrid_fwd(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                                _ptr(beta), _ptr(o), _stream(stream)), "kta_hybrid_fwd")
     return o
+
+
+def hybrid_fwd_window(cfg: HybridCfg, f0: int, q, k, v, alpha=None, beta=None, *, S0=None,
+                      return_state: bool = False, out=None, stream=None):
+    """Hybrid layer for the query frames f0 .. F-1 of a key / value span of cfg.s.F frames (one
+    sequence): q, alpha, beta cover the query frames, k and v the whole span; the GLA heads start
+    from S0 ([1, n_gla, d, d] fp32 or None) and, with return_state, also return their end state."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.dtype)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32)
+    o = torch.empty_like(q) if out is None else out
+    S_out = None
+    if return_state:
+        S_out = torch.empty((q.shape[0], cfg.n_gla, cfg.s.d, cfg.s.d), device=q.device,
+                            dtype=torch.float32)
+    _check(_lib.kta_hybrid_fwd_window(ctypes.byref(cfg), f0, _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(S_out), _ptr(o),
+                                      _stream(stream)), "kta_hybrid_fwd_window")
+    return (o, S_out) if return_state else o
+
+
+def state_affine(A, X, E=None, *, out=None, stream=None):
+    """Y = A X + E for stacks of square fp32 matrices [..., d, d] (E optional)."""
+    for n, t in (("A", A), ("X", X)):
+        _need(t, n, torch.float32)
+    if E is not None:
+        _need(E, "E", torch.float32)
+    d = A.shape[-1]
+    Y = torch.empty_like(X) if out is None else out
+    _check(_lib.kta_state_affine(_ptr(A), _ptr(X), _ptr(E), _ptr(Y), A.numel() // (d * d), d,
+                                 _stream(stream)), "kta_state_affine")
+    return Y
 
 
 class Stream:

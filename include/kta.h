@@ -264,6 +264,32 @@ kta_status kta_gla_delta_bwd(const void* q, const void* k, const void* v, const 
                              void* stream);
 
 /*
+ * kta_hybrid_fwd for the query frames f0 .. F-1 of a longer key / value span: the building block
+ * of a sequence split across devices (each holds a run of frames and receives from its
+ * predecessors the K/V frames its windows reach back to, plus the GLA state at its first token).
+ *   cfg->s.F = frames in k and v; q, o, alpha, beta cover the last F - f0 of them
+ *   ([B][(F - f0)*P][...]), k and v all F ([B][F*P][H][d]). Window frames are numbered within
+ *   k / v, so the span must start at the sequence's frame 0 or reach back at least
+ *   max(W_swa - 1, (W_dswa - 1) * dil) frames before f0 (otherwise the first windows are cut).
+ *   The GLA / delta heads run over the query frames' tokens from the state S0 ([B][n_gla][d][d]
+ *   key-major fp32, NULL = zero) and write their end state to S_out (or NULL).
+ *   f0 = 0 with NULL S0 and S_out is kta_hybrid_fwd. f0 > 0 needs B == 1.
+ */
+kta_status kta_hybrid_fwd_window(const kta_hybrid_cfg* cfg, int f0, const void* q, const void* k,
+                                 const void* v, const float* alpha, const float* beta,
+                                 const float* S0, float* S_out, void* o, void* stream);
+
+/*
+ * Y_m = A_m X_m + E_m for n row-major d x d fp32 matrices (E may be NULL): composes the affine
+ * state maps of consecutive token runs. The GLA and delta-rule state after a run is
+ * T S_start + S_loc, where S_loc is the run's end state from a zero start and T its transition
+ * (the end state of the run started from the identity with v = 0), so the state entering run j
+ * is obtained by folding the runs before it. Y must not alias A or X.
+ */
+kta_status kta_state_affine(const float* A, const float* X, const float* E, float* Y, int n, int d,
+                            void* stream);
+
+/*
  * Streaming rollout -- paper-read, section 2, third pillar: low-latency rolling prediction, one
  * frame at a time. A stream holds, per sequence, the GLA state and a ring of the last
  * W_swa frames (SWA heads) or (W_dswa-1)*dil+1 frames (DSWA heads) of k and v. Each step takes
