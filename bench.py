@@ -45,14 +45,15 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=None,
                     help="profiling only: override the delta workload's tokens per sequence")
     ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep", "backward",
-                                           "layer"),
+                                           "layer", "seqshard"),
                     default="hybrid",
                     help="hybrid: the 21-frame hybrid layer (the headline line); delta: gated "
                          "delta rule, 2 x 65,536 tokens x 16 heads; stream: 240-frame rollout one "
                          "frame per call; sweep: hybrid layer vs full frame-causal attention for "
                          "F = 8..256 frames of 1,024 tokens (one line per F); backward: the "
                          "hybrid layer's reverse mode in fp32; layer: input projections + hybrid "
-                         "operator + output projection")
+                         "operator + output projection; seqshard: the hybrid layer split by frames "
+                         "over 4 ranks, emulated one after another on one GPU")
     return ap.parse_args()
 
 
@@ -645,6 +646,34 @@ def run_other(args):
                          "frac_of_sustained": pf / (k_ms / 1e3) / 1e12 / tc_s,
                          "peak_source": peaks_kind},
             "clocks": clocks, "kernels": kern})
+    elif args.workload == "seqshard":
+        from hybrid_linear_temporal_kta_b200 import seqshard
+        w = synth.HYBRID_BF16
+        R = 4
+        c = seqshard.ShardCfg(F=w.F, P=w.P, d=w.d, n_swa=w.n_swa, n_dswa=w.n_dswa,
+                              n_gla=w.n_gla, W_swa=w.W_swa, W_dswa=w.W_dswa, dil=w.dil,
+                              chunk=w.chunk)
+        x = synth.make_inputs_device(w, seed=w.seed_base)
+        ops = seqshard.KtaOps()
+        cfg = kta.cfg_from_workload(w)
+        o = torch.empty_like(x["q"])
+
+        def whole():
+            kta.hybrid_fwd(cfg, x["q"], x["k"], x["v"], x["alpha"], out=o)
+
+        def split():
+            seqshard.emulate_ranks(c, R, x["q"], x["k"], x["v"], x["alpha"], ops=ops)
+        ms_w = _device_ms(whole, args.steps, args.warmup)
+        ms_s = _device_ms(split, args.steps, args.warmup)
+        kern = _traced(split, args.steps)
+        lines.append({
+            "workload": f"seqshard_bf16_F21_P1560_R{R}_emulated", "unit": "tokens/s",
+            "metric": "hybrid layer split by frames over 4 ranks, all ranks run one after another "
+                      "on one GPU (work and exchange overhead of the split, not a multi-GPU time)",
+            "value": w.B * w.N / (ms_s / 1e3), "ms_per_step": ms_s, "steps": args.steps,
+            "unsharded_ms": ms_w, "overhead": ms_s / ms_w,
+            "frames_per_rank": [n for _, n in seqshard.frame_split(w.F, R)],
+            "halo_frames": c.halo, "kernels": kern})
     else:  # sweep
         for F in (8, 16, 32, 64, 128, 256):
             w = synth.sweep_workload(F)
