@@ -132,3 +132,16 @@ def test_full_layer_size_sampled_rows(kta):
     got = torch.cat([t[0, rows].reshape(len(rows), -1).float() for t in (q, k, v)], 1)
     assert rel(got.cpu().numpy(), ref[:, :hd]) <= BF16_TOL
     assert rel(a[0, rows].reshape(len(rows), -1).cpu().numpy(), ref[:, hd:]) <= F32_TOL
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 8), (1, 300, 16), (129, 257, 72)])
+def test_degenerate_and_odd_shapes(kta, M, N, K):
+    """One row, one column, K below one 64-wide step, and tile edges plus one."""
+    rng = np.random.default_rng(M * 7 + N + K)
+    x, xh = bf16_pair(rng, (M, K))
+    w, wh = bf16_pair(rng, (N, K))
+    y = torch.empty((M, N), device="cuda", dtype=torch.float32)
+    kta.proj_fwd(x, w, [(0, N, y, kta.PROJ_F32)])
+    torch.cuda.synchronize()
+    kta.device_status()
+    assert rel(y.cpu().numpy(), oracle.proj(xh, wh)) <= F32_TOL

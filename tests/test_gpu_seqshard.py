@@ -87,3 +87,23 @@ def test_window_argument_checks(kta):
     Y = kta.state_affine(A, X, X)
     torch.cuda.synchronize()
     assert torch.allclose(Y, 2 * X)
+
+
+def test_ranks_with_one_frame_and_fp32(kta):
+    """More ranks than the halo's worth of frames per rank (every rank holds one or two frames,
+    halos span up to four predecessors), in the fp32 reference mode."""
+    w = synth.TINY_F32.replace(name="shard_f32", F=7, P=20, d=32, n_swa=1, n_dswa=1, n_gla=1,
+                               W_swa=2, W_dswa=3, dil=2)
+    x = synth.make_inputs(w, seed_base=5)
+    dev = {n: (None if t is None else t.cuda()) for n, t in x.items()}
+    c = shard_cfg(w)
+    c.chunk = w.chunk
+    o = seqshard.emulate_ranks(c, 5, dev["q"], dev["k"], dev["v"], dev["alpha"],
+                               ops=seqshard.KtaOps())
+    torch.cuda.synchronize()
+    kta.device_status()
+    ref, _ = oracle.hybrid(x["q"], x["k"], x["v"], x["alpha"], None, P=w.P, n_swa=1, n_dswa=1,
+                           n_gla=1, W_swa=2, W_dswa=3, dil=2, scale_softmax=w.scale_softmax)
+    got = o.float().cpu().numpy()
+    for h in range(w.H):
+        assert rel(got[:, :, h], ref[:, :, h]) <= 1e-4, f"head {h}"
