@@ -23,6 +23,7 @@
 #include "delta_chunk.cuh"
 #include "bwd_f32.cuh"
 #include "proj_gemm.cuh"
+#include "win_bwd_tc.cuh"
 
 namespace {
 
@@ -240,6 +241,7 @@ struct WinLaunch {
   void* o = nullptr;
   long long o_ld = 0;
   float scale = 1.f;
+  float* lse = nullptr;      // optional row log-sum-exp output (bf16 tensor-core path only)
   WinGroup g[2];
 };
 
@@ -275,6 +277,7 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   p.scale_log2 = L.scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(L.o);
   p.o_ld = L.o_ld;
+  p.lse = L.lse;
   // one CTA per pair of query tiles of a (frame, head, sequence); one per tile when pairs would
   // leave SMs idle (a streaming step's single frame)
   const long long units = static_cast<long long>(L.Fq) * Htot * L.B;
@@ -1084,9 +1087,106 @@ int sm_count() {
   return n[dev];
 }
 
+template <int D>
+kta_status launch_win_bwd_tc(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             const kta_shape& s, int H, int ld_heads, int W, int dil, float scale,
+                             cudaStream_t st) {
+  const long long N = static_cast<long long>(s.F) * s.P;
+  const long long rows = static_cast<long long>(s.B) * N;
+  const long long ld = static_cast<long long>(ld_heads) * D;
+  void* ws = nullptr;
+  kta_status r;
+  if ((r = workspace(static_cast<size_t>(s.B) * H * N * sizeof(float), st, &ws))) return r;
+  float* Dt = static_cast<float*>(ws);
+  {
+    TraceScope ts("row_dot", st);
+    const long long warps = rows * H;
+    kta::row_dot_kernel<D><<<static_cast<unsigned>((warps + 7) / 8), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), Dt, rows,
+        static_cast<int>(N), H, ld);
+    KTA_CUDA(cudaGetLastError());
+  }
+  CUtensorMap tq, tdo, tk, tv;
+  if ((r = make_map(&tq, q, D, H, rows, ld)) || (r = make_map(&tdo, dout, D, H, rows, ld)) ||
+      (r = make_map(&tk, k, D, H, rows, ld)) || (r = make_map(&tv, v, D, H, rows, ld)))
+    return r;
+  kta::WinBwdParams p{};
+  p.B = s.B;
+  p.P = s.P;
+  p.F = s.F;
+  p.Htot = H;
+  p.H0 = H;
+  p.W[0] = p.W[1] = W;
+  p.dil[0] = p.dil[1] = dil;
+  p.n_t = (s.P + 127) / 128;
+  p.rows_b = static_cast<int>(N);
+  p.ld = ld;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.lse = lse;
+  p.Dt = Dt;
+  const long long nblk = static_cast<long long>(s.F) * H * s.B * p.n_t;
+  if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "too many tiles (%lld)", nblk);
+  const size_t smem = kta::win_bwd_smem_bytes<D>();
+  if ((r = set_smem_attr(kta::win_bwd_dq_kernel<D>, smem)) ||
+      (r = set_smem_attr(kta::win_bwd_dkv_kernel<D>, smem)))
+    return r;
+  {
+    p.out0 = static_cast<__nv_bfloat16*>(dq);
+    p.out1 = nullptr;
+    TraceScope ts("win_bwd_dq", st);
+    kta::win_bwd_dq_kernel<D><<<static_cast<unsigned>(nblk), 256, smem, st>>>(tq, tdo, tk, tv, p);
+    KTA_CUDA(cudaGetLastError());
+  }
+  p.out0 = static_cast<__nv_bfloat16*>(dk);
+  p.out1 = static_cast<__nv_bfloat16*>(dv);
+  TraceScope ts("win_bwd_dkv", st);
+  kta::win_bwd_dkv_kernel<D><<<static_cast<unsigned>(nblk), 256, smem, st>>>(tq, tdo, tk, tv, p);
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+kta_status kta_softmax_fwd_lse(const void* q, const void* k, const void* v, void* o, float* lse,
+                               kta_shape s, int H, int ld_heads, int W, int dil, float scale,
+                               void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) || (r = check_ptrs({q, k, v, o})) ||
+      (r = check_softmax_dtype(s)))
+    return r;
+  if (s.dtype != KTA_BF16 || (s.d != 64 && s.d != 128))
+    return fail(KTA_ERR_UNSUPPORTED, "the row log-sum-exp output needs bf16 and d in {64, 128}");
+  if (!lse) return fail(KTA_ERR_INVALID_ARG, "null lse");
+  if (W < 1 || dil < 1) return fail(KTA_ERR_INVALID_ARG, "W and dil must be >= 1");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be > 0");
+  WinLaunch L = seq_win_launch(q, k, v, o, s, ld_heads, scale);
+  L.g[0] = seq_group(k, v, s, H, H, ld_heads, W, dil);
+  L.lse = lse;
+  return launch_win(L, as_stream(stream));
+}
+
+kta_status kta_softmax_bwd_bf16(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                kta_shape s, int H, int ld_heads, int W, int dil, float scale,
+                                void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) ||
+      (r = check_ptrs({q, k, v, o, dout, dq, dk, dv})))
+    return r;
+  if (s.dtype != KTA_BF16 || (s.d != 64 && s.d != 128))
+    return fail(KTA_ERR_UNSUPPORTED, "the tensor-core backward needs bf16 and d in {64, 128}");
+  if (!lse) return fail(KTA_ERR_INVALID_ARG, "null lse");
+  if (W < 1 || dil < 1) return fail(KTA_ERR_INVALID_ARG, "W and dil must be >= 1");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(KTA_ERR_INVALID_ARG, "scale must be > 0");
+  cudaStream_t st = as_stream(stream);
+  if (s.d == 128)
+    return launch_win_bwd_tc<128>(q, k, v, o, lse, dout, dq, dk, dv, s, H, ld_heads, W, dil, scale, st);
+  return launch_win_bwd_tc<64>(q, k, v, o, lse, dout, dq, dk, dv, s, H, ld_heads, W, dil, scale, st);
+}
 
 kta_status kta_proj_fwd(const void* x, const void* w, int M, int N, int K,
                         const kta_proj_seg* segs, int nseg, void* stream) {

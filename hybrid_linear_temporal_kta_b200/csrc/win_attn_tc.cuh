@@ -52,6 +52,8 @@ struct WinParams {
   float scale_log2; // softmax scale * log2(e)
   __nv_bfloat16* o; // output, already offset to the launch's first head
   long long o_ld;   // output row stride in elements
+  float* lse;       // optional [B][Htot][q_rows_b]: m + log2(l), the base-2 log-sum-exp of
+                    // scale * log2(e) * S over each row's visible keys (null = not written)
 };
 
 __device__ __forceinline__ int win_num_tiles(int f, int P, int W, int dil) {
@@ -367,6 +369,9 @@ __global__ void __launch_bounds__(384, 1)
       if (__all_sync(0xffffffffu, fin)) {
         tc_fence_after();
         const float inv = 1.0f / l;
+        if (p.lse && row < nq)
+          p.lse[(static_cast<long long>(b) * p.Htot + h) * p.q_rows_b + f_local * p.P +
+                (p.pair * pr + x) * 128 + row] = m + __log2f(l);
         __nv_bfloat16* orow =
             p.o + static_cast<long long>(q_row0 + 128 * x + row) * p.o_ld + h * D;
 #pragma unroll

@@ -64,6 +64,9 @@ _SIGS = {
                                   _st),
     "kta_hybrid_fwd": ([ctypes.POINTER(HybridCfg), _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
     "kta_proj_fwd": ([_vp, _vp, _i, _i, _i, ctypes.POINTER(ProjSeg), _i, _vp], _st),
+    "kta_softmax_fwd_lse": ([_vp, _vp, _vp, _vp, _fp, Shape, _i, _i, _i, _i, _f, _vp], _st),
+    "kta_softmax_bwd_bf16": ([_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, Shape, _i, _i, _i, _i,
+                              _f, _vp], _st),
     "kta_swa_bwd": ([_vp] * 7 + [Shape, _i, _i, _i, _f, _vp], _st),
     "kta_dswa_bwd": ([_vp] * 7 + [Shape, _i, _i, _i, _i, _f, _vp], _st),
     "kta_gla_bwd": ([_vp, _vp, _vp, _fp, _fp, _vp, _vp, _vp, _vp, _fp, _fp, Shape, _i, _i, _f,
@@ -271,6 +274,44 @@ def qkv_gate_proj(x, w, *, H: int, d: int, n_gla: int, gla_delta: bool = False, 
         raise ValueError(f"stacked weight must have {want} rows, got {w.shape[0]}")
     proj_fwd(x, w, segs, stream)
     return q, k, v, alpha, beta
+
+
+def softmax_fwd_lse(q, k, v, *, P: int, W: int, dil: int = 1, scale: float | None = None,
+                    heads=None, out=None, stream=None):
+    """SWA (dil = 1) / DSWA forward, bf16, that also returns each row's base-2 log-sum-exp:
+    (o, lse) with lse [B, H, N] fp32 for the heads in range (the bf16 backward's input)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16)
+    B, N, Htot, d = q.shape
+    h0, h1 = heads if heads is not None else (0, Htot)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, h1 - h0, N), device=q.device, dtype=torch.float32)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check(_lib.kta_softmax_fwd_lse(_ptr(q, h0 * d), _ptr(k, h0 * d), _ptr(v, h0 * d),
+                                    _ptr(o, h0 * d), _ptr(lse), _shape(q, P), h1 - h0, Htot, W, dil,
+                                    scale, _stream(stream)), "kta_softmax_fwd_lse")
+    return o, lse
+
+
+def softmax_bwd_bf16(q, k, v, o, lse, dout, *, P: int, W: int, dil: int = 1,
+                     scale: float | None = None, heads=None, out=None, stream=None):
+    """Tensor-core gradients (dq, dk, dv) of sum(dout * o) for SWA / DSWA heads, bf16, from the
+    forward's o and lse (softmax_fwd_lse). Heads outside the range are left zero."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _need(t, n, torch.bfloat16)
+    _need(lse, "lse", torch.float32)
+    B, N, Htot, d = q.shape
+    h0, h1 = heads if heads is not None else (0, Htot)
+    if out is None:
+        dq, dk, dv = (torch.zeros_like(q) for _ in range(3))
+    else:
+        dq, dk, dv = out
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    args = [_ptr(t, h0 * d) for t in (q, k, v, o)] + [_ptr(lse), _ptr(dout, h0 * d)]
+    args += [_ptr(t, h0 * d) for t in (dq, dk, dv)]
+    _check(_lib.kta_softmax_bwd_bf16(*args, _shape(q, P), h1 - h0, Htot, W, dil, scale,
+                                     _stream(stream)), "kta_softmax_bwd_bf16")
+    return dq, dk, dv
 
 
 def _grads(q, out):

@@ -235,6 +235,23 @@ kta_status kta_dswa_bwd(const void* q, const void* k, const void* v, const void*
                         float scale, void* stream);
 
 /*
+ * bf16 reverse mode of the softmax heads on the tensor cores (SWA: dil = 1; DSWA: dil > 1).
+ * kta_softmax_fwd_lse is kta_dswa_fwd (bf16, d in {64, 128}) that also writes each query row's
+ * base-2 log-sum-exp lse_t = log2(sum_s 2^(scale log2(e) q_t . k_s)) over its visible keys to
+ * lse ([B][H][N] fp32, head-major). kta_softmax_bwd_bf16 takes that forward's q, k, v, o and
+ * lse with dout and writes dq, dk, dv (bf16, the forward's layout; every computed row written)
+ * by the formulas of kta_swa_bwd with P_ts = 2^(scale log2(e) q_t . k_s - lse_t), accumulating in
+ * fp32. Workspace: B * H * N floats for dout_t . o_t, from the calling stream's cache.
+ */
+kta_status kta_softmax_fwd_lse(const void* q, const void* k, const void* v, void* o, float* lse,
+                               kta_shape s, int H, int ld_heads, int W, int dil, float scale,
+                               void* stream);
+kta_status kta_softmax_bwd_bf16(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                kta_shape s, int H, int ld_heads, int W, int dil, float scale,
+                                void* stream);
+
+/*
  * kta_gla_bwd: gradients of kta_gla_chunk_fwd's output. With the state adjoint
  * G_t = scale q_t^T dout_t + diag(alpha_{t+1}) G_{t+1} (G after the last token = 0):
  *     dq_t = scale S_t dout_t^T,  dk_t = G_t v_t^T,  dv_t = k_t G_t,
