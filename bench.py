@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=None,
                     help="profiling only: override the delta workload's tokens per sequence")
     ap.add_argument("--workload", choices=("hybrid", "delta", "stream", "sweep", "backward",
-                                           "layer", "seqshard"),
+                                           "layer", "seqshard", "backward_bf16"),
                     default="hybrid",
                     help="hybrid: the 21-frame hybrid layer (the headline line); delta: gated "
                          "delta rule, 2 x 65,536 tokens x 16 heads; stream: 240-frame rollout one "
@@ -53,7 +53,8 @@ def parse_args():
                          "F = 8..256 frames of 1,024 tokens (one line per F); backward: the "
                          "hybrid layer's reverse mode in fp32; layer: input projections + hybrid "
                          "operator + output projection; seqshard: the hybrid layer split by frames "
-                         "over 4 ranks, emulated one after another on one GPU")
+                         "over 4 ranks, emulated one after another on one GPU; backward_bf16: the "
+                         "hybrid layer's reverse mode with the softmax heads on tensor cores")
     return ap.parse_args()
 
 
@@ -674,6 +675,55 @@ def run_other(args):
             "unsharded_ms": ms_w, "overhead": ms_s / ms_w,
             "frames_per_rank": [n for _, n in seqshard.frame_split(w.F, R)],
             "halo_frames": c.halo, "kernels": kern})
+    elif args.workload == "backward_bf16":
+        w = synth.HYBRID_BF16
+        x = synth.make_inputs_device(w, seed=w.seed_base + 9)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(w.seed_base + 10)
+        dout = torch.randn(x["q"].shape, generator=g, device="cuda").to(torch.bfloat16)
+        q, k, v, a = x["q"], x["k"], x["v"], x["alpha"]
+        ns, nd = w.n_swa, w.n_dswa
+        o = torch.empty_like(q)
+        lse = [kta.softmax_fwd_lse(q, k, v, P=w.P, W=w.W_swa, heads=(0, ns), out=o)[1],
+               kta.softmax_fwd_lse(q, k, v, P=w.P, W=w.W_dswa, dil=w.dil, heads=(ns, ns + nd),
+                                   out=o)[1]]
+        hg = (ns + nd, w.H)
+        # the GLA heads' reverse mode is fp32: their inputs converted once, outside the timed steps
+        qf, kf, vf, dof = (t.float() for t in (q, k, v, dout))
+        grads = tuple(torch.zeros_like(q) for _ in range(3))
+        grads_f = tuple(torch.zeros_like(qf) for _ in range(3))
+
+        def step():
+            # one after another: the fp32 GLA backward holds most SMs for its whole run (one
+            # ~200 KB CTA per SM), so beside it the softmax kernels would only get leftover SMs
+            kta.softmax_bwd_bf16(q, k, v, o, lse[0], dout, P=w.P, W=w.W_swa, heads=(0, ns),
+                                 out=grads)
+            kta.softmax_bwd_bf16(q, k, v, o, lse[1], dout, P=w.P, W=w.W_dswa, dil=w.dil,
+                                 heads=(ns, ns + nd), out=grads)
+            kta.gla_bwd(qf, kf, vf, a, dof, heads=hg, out=grads_f)
+        clk = ClockSampler("0")
+        clk.start()
+        ms = _device_ms(step, args.steps, args.warmup)
+        clocks = clk.stop() or {}
+        kern = _traced(step, args.steps)
+        n = visible_pairs(w)
+        fl = {"win_bwd_dq": 6.0 * w.d * n, "win_bwd_dkv": 8.0 * w.d * n}
+        roof = {}
+        for kname, f_alg in fl.items():
+            k_ms = kern[kname]["ms_per_step"]
+            roof[kname] = {"bound": "tensor", "unit": "TFLOP/s",
+                           "achieved": f_alg / (k_ms / 1e3) / 1e12, "peak": tc,
+                           "frac": f_alg / (k_ms / 1e3) / 1e12 / tc, "peak_source": peaks_kind,
+                           "algorithmic_tflop": f_alg / 1e12}
+        top = max(fl, key=lambda kn: kern[kn]["ms_per_step"])
+        lines.append({
+            "workload": "hybrid_bwd_bf16_F21_P1560", "unit": "tokens/s",
+            "metric": "hybrid layer reverse mode tokens/s (softmax heads bf16 on tensor cores, "
+                      "GLA heads fp32)",
+            "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
+            "dtype": "bf16", "config": {"B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d},
+            "roofline": dict(roof[top], kernel=top), "kernel_rooflines": roof,
+            "clocks": clocks, "kernels": kern})
     else:  # sweep
         for F in (8, 16, 32, 64, 128, 256):
             w = synth.sweep_workload(F)

@@ -656,3 +656,139 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
 }
 
 }  // namespace kta
+
+namespace kta {
+
+// Vector-GLA backward without stored states, one CTA of D threads per (segment, head, sequence),
+// thread j owning column j of S (forward sweep) and of G (reverse sweep) in registers; row
+// reductions go through a transposed copy in shared memory. The gate gradient uses the closed
+// form of the log-gate derivative: with b_t = sum_{u <= t} log alpha_u, q enters as
+// q_t * e^{b_t} and k as k_t * e^{-b_t}, so dL/db_t = q_t (.) dq_t - k_t (.) dk_t and
+//   dalpha_u = (1 / alpha_u) sum_{t >= u} (q_t (.) dq_t - k_t (.) dk_t).
+//   forward sweep (from the segment's entering state): S_t, dq_t = scale S_t dO_t^T, and
+//     y_t = q_t (.) dq_t kept in `ybuf`;
+//   reverse sweep (from the adjoint entering from the right): G_t += scale q_t^T dO_t,
+//     dv_t = k_t G_t, dk_t = G_t v_t^T, the segment-local suffix X_t = sum_{t' >= t, in segment}
+//     (y - k (.) dk) in fp64 (xbuf), then G <- diag(alpha_t) G;
+//   ytot: per (sequence, head, segment) the segment's full sum X_{t0} (for the suffix carry).
+// A segment that is the only one of its sequence writes dS0 = diag(alpha_0) G_0.
+template <int D>
+__global__ void __launch_bounds__(D) gla_bwd_sweep_kernel(const LinBwdParams p, float* ybuf,
+                                                          double* xbuf, double* ytot) {
+  extern __shared__ float gsm[];
+  constexpr int LDT = D + 1;
+  float* T = gsm;              // [D][D + 1] transposed state / adjoint
+  float* qv = T + D * LDT;
+  float* kv = qv + D;
+  float* vv = kv + D;
+  float* dv_ = vv + D;
+  float* av = dv_ + D;
+  const int j = threadIdx.x;
+  const int h = blockIdx.x, b = blockIdx.y, seg = blockIdx.z;
+  const long long bh = static_cast<long long>(b) * p.H + h;
+  const long long bhs = bh * p.nseg + seg;
+  const int t0 = seg * p.seg_len, t1 = min(p.N, t0 + p.seg_len);
+  const long long rb = static_cast<long long>(b) * p.rows_b;
+  auto row_of = [&](int t) { return (rb + t) * p.ld + static_cast<long long>(h) * D; };
+  auto load_vecs = [&](int t) {
+    const long long r = row_of(t);
+    qv[j] = p.q[r + j];
+    kv[j] = p.k[r + j];
+    vv[j] = p.v[r + j];
+    dv_[j] = p.dout[r + j];
+    av[j] = p.alpha[((rb + t) * p.H + h) * D + j];
+  };
+  // scratch rows of this sequence-head: token t of the sequence at (bh * N + t) * D
+  float* yrow = ybuf + bh * static_cast<long long>(p.N) * D;
+  double* xrow = xbuf + bh * static_cast<long long>(p.N) * D;
+
+  float X[D];
+  // ---- forward sweep: S column j, dq_t, y_t
+  if (p.Sin) {
+#pragma unroll
+    for (int i = 0; i < D; ++i) X[i] = p.Sin[bhs * D * D + i * D + j];
+  } else {
+#pragma unroll
+    for (int i = 0; i < D; ++i) X[i] = p.S0 ? p.S0[bh * D * D + i * D + j] : 0.f;
+  }
+  for (int t = t0; t < t1; ++t) {
+    __syncthreads();
+    load_vecs(t);
+    __syncthreads();
+    const float vj = vv[j];
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      X[i] = fmaf(av[i], X[i], kv[i] * vj);
+      T[i * LDT + j] = X[i];
+    }
+    __syncthreads();
+    const int i = j;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int jj = 0; jj < D; ++jj) acc = fmaf(T[i * LDT + jj], dv_[jj], acc);
+    const float dqi = acc * p.scale;
+    p.dq[row_of(t) + i] = dqi;
+    yrow[static_cast<long long>(t) * D + i] = qv[i] * dqi;
+  }
+  // ---- reverse sweep: G column j, dv_t, dk_t, local suffix of the gate terms
+  if (p.Gin) {
+#pragma unroll
+    for (int i = 0; i < D; ++i) X[i] = p.Gin[bhs * D * D + i * D + j];
+  } else {
+#pragma unroll
+    for (int i = 0; i < D; ++i) X[i] = 0.f;
+  }
+  double suf = 0.0;  // thread j's key dim: sum over this segment's tokens >= t
+  for (int t = t1 - 1; t >= t0; --t) {
+    __syncthreads();
+    load_vecs(t);
+    __syncthreads();
+    const float dj = dv_[j] * p.scale;
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      X[i] = fmaf(qv[i], dj, X[i]);
+      acc = fmaf(kv[i], X[i], acc);
+      T[i * LDT + j] = X[i];
+    }
+    p.dv[row_of(t) + j] = acc;
+    __syncthreads();
+    const int i = j;
+    float dk = 0.f;
+#pragma unroll 8
+    for (int jj = 0; jj < D; ++jj) dk = fmaf(T[i * LDT + jj], vv[jj], dk);
+    p.dk[row_of(t) + i] = dk;
+    suf += static_cast<double>(yrow[static_cast<long long>(t) * D + i]) -
+           static_cast<double>(kv[i]) * static_cast<double>(dk);
+    xrow[static_cast<long long>(t) * D + i] = suf;
+#pragma unroll
+    for (int ii = 0; ii < D; ++ii) X[ii] *= av[ii];
+  }
+  ytot[bhs * D + j] = suf;
+  if (p.dS0 && p.nseg == 1) {
+    // X = diag(alpha_0) G_0 after the last step
+#pragma unroll
+    for (int i = 0; i < D; ++i) p.dS0[bh * D * D + i * D + j] = X[i];
+  }
+}
+
+// dalpha_t[i] = (X_t[i] + sum of later segments' totals) / alpha_t[i], one thread per element of
+// [B][N][H][D] (the later segments' totals are summed here: a handful per sequence-head).
+template <int D>
+__global__ void gla_bwd_dalpha_kernel(const LinBwdParams p, const double* __restrict__ xbuf,
+                                      const double* __restrict__ ytot) {
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int b = blockIdx.y;
+  if (e >= static_cast<long long>(p.N) * p.H * D) return;
+  const int i = static_cast<int>(e % D);
+  const int h = static_cast<int>((e / D) % p.H);
+  const int t = static_cast<int>(e / (static_cast<long long>(D) * p.H));
+  const long long bh = static_cast<long long>(b) * p.H + h;
+  const int seg = t / p.seg_len;
+  double x = xbuf[(bh * p.N + t) * D + i];
+  for (int s = seg + 1; s < p.nseg; ++s) x += ytot[(bh * p.nseg + s) * D + i];
+  const long long a = ((static_cast<long long>(b) * p.rows_b + t) * p.H + h) * D + i;
+  p.dalpha[a] = static_cast<float>(x / static_cast<double>(p.alpha[a]));
+}
+
+}  // namespace kta

@@ -982,31 +982,53 @@ kta_status softmax_bwd_common(const void* q, const void* k, const void* v,
 
 template <int D>
 kta_status launch_lin_bwd(kta::LinBwdParams p, int B, cudaStream_t st) {
-  // Vector GLA splits each sequence into segments so that the launch has about one CTA per SM
-  // (the delta rule's segment carry would need dense d x d transitions: one segment).
   const long long bh = static_cast<long long>(B) * p.H;
+  if (p.delta) {
+    // The delta rule's segment carry would need dense d x d transitions: one segment per
+    // (sequence, head), states checkpointed every BWD_CK tokens and recomputed per chunk.
+    p.nseg = 1;
+    p.seg_len = p.N;
+    p.nck = (p.N + kta::BWD_CK - 1) / kta::BWD_CK;
+    p.Sin = p.Gin = nullptr;
+    void* ws = nullptr;
+    kta_status r = workspace(static_cast<size_t>(kta::lin_bwd_ws_floats<D>(p.nck)) * bh *
+                                 sizeof(float), st, &ws);
+    if (r) return r;
+    p.ws = static_cast<float*>(ws);
+    const size_t smem = (3 * static_cast<size_t>(D) * (D + 1) + 8 * D) * sizeof(float);
+    if ((r = set_smem_attr(kta::lin_bwd_f32_kernel<D>, smem))) return r;
+    TraceScope ts("delta_bwd_f32", st);
+    kta::lin_bwd_f32_kernel<D><<<dim3(p.H, B, 1), D, smem, st>>>(p);
+    KTA_CUDA(cudaGetLastError());
+    return KTA_OK;
+  }
+  // Vector GLA: segments of the sequence for about three CTAs per SM; a forward sweep and a
+  // reverse sweep per segment from the carried state and adjoint.
   int nseg = 1;
   long long seg_len = p.N;
-  if (!p.delta && bh < 148) {
-    const long long want = std::max<long long>(1, 148 / bh);
+  if (bh < 3 * 148) {
+    const long long want = std::max<long long>(1, 3 * 148 / bh);
     seg_len = ((p.N + want - 1) / want + kta::BWD_CK - 1) / kta::BWD_CK * kta::BWD_CK;
     nseg = static_cast<int>((p.N + seg_len - 1) / seg_len);
   }
   if (nseg == 1) seg_len = p.N;
   p.nseg = nseg;
   p.seg_len = static_cast<int>(seg_len);
-  p.nck = static_cast<int>((seg_len + kta::BWD_CK - 1) / kta::BWD_CK);
   const long long bhs = bh * nseg;
-  const long long per = kta::lin_bwd_ws_floats<D>(p.nck);
   const long long sum_per = 2LL * D * D + 2 * D;
-  const long long floats = bhs * per + (nseg > 1 ? bhs * (sum_per + 2LL * D * D) : 0);
+  const long long tokD = bh * p.N * D;
+  // floats: ybuf, then (nseg > 1) summaries, Sin, Gin; doubles: xbuf, ytot
+  const long long n_f = tokD + (nseg > 1 ? bhs * (sum_per + 2LL * D * D) : 0);
+  const long long n_d = tokD + bhs * D;
   void* ws = nullptr;
-  kta_status r = workspace(static_cast<size_t>(floats) * sizeof(float), st, &ws);
+  kta_status r = workspace(static_cast<size_t>(n_d) * 8 + static_cast<size_t>(n_f) * 4, st, &ws);
   if (r) return r;
-  p.ws = static_cast<float*>(ws);
+  double* xbuf = static_cast<double*>(ws);
+  double* ytot = xbuf + tokD;
+  float* ybuf = reinterpret_cast<float*>(ytot + bhs * D);
   p.Sin = p.Gin = nullptr;
   if (nseg > 1) {
-    float* sum = p.ws + bhs * per;
+    float* sum = ybuf + tokD;
     float* Sin = sum + bhs * sum_per;
     float* Gin = Sin + bhs * D * D;
     {
@@ -1024,10 +1046,17 @@ kta_status launch_lin_bwd(kta::LinBwdParams p, int B, cudaStream_t st) {
     p.Sin = Sin;
     p.Gin = Gin;
   }
-  const size_t smem = (3 * static_cast<size_t>(D) * (D + 1) + 8 * D) * sizeof(float);
-  if ((r = set_smem_attr(kta::lin_bwd_f32_kernel<D>, smem))) return r;
-  TraceScope ts(p.delta ? "delta_bwd_f32" : "gla_bwd_f32", st);
-  kta::lin_bwd_f32_kernel<D><<<dim3(p.H, B, nseg), D, smem, st>>>(p);
+  const size_t smem = (static_cast<size_t>(D) * (D + 1) + 5 * D) * sizeof(float);
+  if ((r = set_smem_attr(kta::gla_bwd_sweep_kernel<D>, smem))) return r;
+  {
+    TraceScope ts("gla_bwd_f32", st);
+    kta::gla_bwd_sweep_kernel<D><<<dim3(p.H, B, nseg), D, smem, st>>>(p, ybuf, xbuf, ytot);
+    KTA_CUDA(cudaGetLastError());
+  }
+  TraceScope ts("gla_bwd_dalpha_f32", st);
+  const long long n = static_cast<long long>(p.N) * p.H * D;
+  kta::gla_bwd_dalpha_kernel<D><<<dim3(static_cast<unsigned>((n + 255) / 256), B), 256, 0, st>>>(
+      p, xbuf, ytot);
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
