@@ -286,16 +286,22 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   if (nblk <= 0) return KTA_OK;
   if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "too many tiles (%lld)", nblk);
   const size_t smem = kta::win_smem_bytes<D>();
-  if ((s = set_smem_attr(kta::win_attn_tc_kernel<D>, smem))) return s;
+  if ((s = set_smem_attr(kta::win_attn_tc_kernel<D, false>, smem)) ||
+      (s = set_smem_attr(kta::win_attn_tc_kernel<D, true>, smem)))
+    return s;
   {
     TraceScope ts("win_attn_tc", st);
-    kta::win_attn_tc_kernel<D><<<static_cast<unsigned>(nblk), 384, smem, st>>>(tq, tk0, tv0, tk1,
-                                                                               tv1, p);
+    if (L.lse)
+      kta::win_attn_tc_kernel<D, true><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
+          tq, tk0, tv0, tk1, tv1, p);
+    else
+      kta::win_attn_tc_kernel<D, false><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
+          tq, tk0, tv0, tk1, tv1, p);
   }
   const cudaError_t le = cudaGetLastError();
   if (le != cudaSuccess) {
     cudaFuncAttributes fa{};
-    cudaFuncGetAttributes(&fa, kta::win_attn_tc_kernel<D>);
+    cudaFuncGetAttributes(&fa, kta::win_attn_tc_kernel<D, false>);
     return fail(KTA_ERR_CUDA,
                 "win_attn_tc launch failed: %s (grid %lld x 384, dyn smem %zu, regs %d, max threads "
                 "%d, max dyn smem %d)",

@@ -102,7 +102,9 @@ constexpr size_t win_smem_bytes() {
   return sizeof(WinSmem<D>) + 1024;  // + manual 1024-byte alignment of the dynamic base
 }
 
-template <int D>
+// LSE: also store each row's base-2 log-sum-exp to p.lse (a separate instantiation, so that the
+// plain forward's code is unchanged).
+template <int D, bool LSE = false>
 __global__ void __launch_bounds__(384, 1)
     win_attn_tc_kernel(const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk0,
@@ -369,7 +371,7 @@ __global__ void __launch_bounds__(384, 1)
       if (__all_sync(0xffffffffu, fin)) {
         tc_fence_after();
         const float inv = 1.0f / l;
-        if (p.lse && row < nq)
+        if (LSE && row < nq)
           p.lse[(static_cast<long long>(b) * p.Htot + h) * p.q_rows_b + f_local * p.P +
                 (p.pair * pr + x) * 128 + row] = m + __log2f(l);
         __nv_bfloat16* orow =
