@@ -348,9 +348,9 @@ struct LinBwdParams {
   int rows_b, N, H;
   float scale;
   int delta, erase_decayed;
-  int seg_len, nseg;   // tokens per segment (a multiple of BWD_CK) and segments per sequence
-  int nck;             // stored states per segment = ceil(seg_len / BWD_CK)
-  float* ws;           // per (sequence, head, segment): states [nck][D][D], chunk
+  int seg_len, nseg;   // vector GLA: tokens per segment and segments per sequence
+  int nck;             // delta rule: stored states per sequence = ceil(N / BWD_CK)
+  float* ws;           // delta rule, per (sequence, head): states [nck][D][D], chunk
                        // [BWD_CK][D][D], u, w
   // vector GLA with nseg > 1 only, per (sequence, head, segment) [D][D] (key-major):
   const float* Sin;    // state before the segment's first token
@@ -457,12 +457,13 @@ __global__ void gla_bwd_carry_kernel(const LinBwdParams p, const float* __restri
   if (p.dS0) p.dS0[bh * D * D + i * D + j] = p.alpha[(rb * p.H + h) * D + i] * Gf;
 }
 
-// One CTA of D threads per (head, sequence, segment). Thread j owns column j of the state in
-// the forward passes (registers) and of the adjoint G (shared memory); for the row reductions
-// (dq, dk, dalpha) thread i owns row i. A segment starts from p.Sin / p.Gin when they are
-// given, else from S0 / zero (one segment per sequence).
+// Delta-rule backward (both erase forms), one CTA of D threads per (head, sequence). Thread j
+// owns column j of the state in the forward passes (registers) and of the adjoint G (shared
+// memory); for the row reductions (dq, dk, dalpha) thread i owns row i. States are checkpointed
+// every BWD_CK tokens; each chunk is recomputed (its states, u and w kept in the workspace)
+// before its reverse pass, which reads S_t and S_{t-1} rows from shared memory.
 template <int D>
-__global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
+__global__ void __launch_bounds__(D) delta_bwd_f32_kernel(const LinBwdParams p) {
   extern __shared__ float bsm[];
   constexpr int LDG = D + 1;
   float* G = bsm;                 // [D][D + 1]
@@ -471,63 +472,49 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
   float* kv = qv + D;             // k_t
   float* vv = kv + D;             // v_t
   float* dv_ = vv + D;            // dO_t
-  float* av = dv_ + D;            // alpha_t (vector gate) or alpha_t in av[0]
-  float* du = av + D;             // du_t (delta)
-  float* red = du + D;            // [2][D] block reductions (delta)
+  float* av = dv_ + D;            // alpha_t in av[0]
+  float* du = av + D;             // du_t
+  float* red = du + D;            // [2][D] block reductions
   const int j = threadIdx.x;
-  const int h = blockIdx.x, b = blockIdx.y, seg = blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const long long bh = static_cast<long long>(b) * p.H + h;
-  const long long bhs = bh * p.nseg + seg;
-  const int t_beg = seg * p.seg_len, t_end = min(p.N, t_beg + p.seg_len);
-  float* ck = p.ws + bhs * lin_bwd_ws_floats<D>(p.nck);
+  float* ck = p.ws + bh * lin_bwd_ws_floats<D>(p.nck);
   float* buf = ck + static_cast<long long>(p.nck) * D * D;
   float* Ub = buf + static_cast<long long>(BWD_CK) * D * D;
   float* Wb = Ub + BWD_CK * D;
   const long long rb = static_cast<long long>(b) * p.rows_b;
   auto row_of = [&](int t) { return (rb + t) * p.ld + static_cast<long long>(h) * D; };
-  auto gate_a = [&](int t, int i) {
-    return p.delta ? p.alpha[(rb + t) * p.H + h] : p.alpha[((rb + t) * p.H + h) * D + i];
-  };
+  auto gate_a = [&](int t) { return p.alpha[(rb + t) * p.H + h]; };
   auto gate_b = [&](int t) { return p.beta[(rb + t) * p.H + h]; };
 
   // one forward step of column j of S, given the token's vectors in shared memory
   float S[D];
   auto step = [&](int t, int tl, bool keep_uw) {
-    if (p.delta) {
-      const float a = av[0], be = gate_b(t), ae = p.erase_decayed ? a : 1.f;
-      float w = 0.f;
+    const float a = av[0], be = gate_b(t), ae = p.erase_decayed ? a : 1.f;
+    float w = 0.f;
 #pragma unroll
-      for (int i = 0; i < D; ++i) w = fmaf(kv[i], S[i], w);
-      const float u = be * (vv[j] - ae * w);
-      if (keep_uw) {
-        Ub[tl * D + j] = u;
-        Wb[tl * D + j] = w;
-      }
-#pragma unroll
-      for (int i = 0; i < D; ++i) S[i] = fmaf(a, S[i], kv[i] * u);
-    } else {
-#pragma unroll
-      for (int i = 0; i < D; ++i) S[i] = fmaf(av[i], S[i], kv[i] * vv[j]);
+    for (int i = 0; i < D; ++i) w = fmaf(kv[i], S[i], w);
+    const float u = be * (vv[j] - ae * w);
+    if (keep_uw) {
+      Ub[tl * D + j] = u;
+      Wb[tl * D + j] = w;
     }
+#pragma unroll
+    for (int i = 0; i < D; ++i) S[i] = fmaf(a, S[i], kv[i] * u);
   };
   auto load_kva = [&](int t) {
     const long long r = row_of(t);
     kv[j] = p.k[r + j];
     vv[j] = p.v[r + j];
-    av[j] = p.delta ? (j == 0 ? gate_a(t, 0) : 0.f) : gate_a(t, j);
+    av[j] = j == 0 ? gate_a(t) : 0.f;
   };
 
-  // ---- forward: the state before every BWD_CK-th token of the segment
-  if (p.Sin) {
+  // ---- forward: the state before every BWD_CK-th token
 #pragma unroll
-    for (int i = 0; i < D; ++i) S[i] = p.Sin[bhs * D * D + i * D + j];
-  } else {
-#pragma unroll
-    for (int i = 0; i < D; ++i) S[i] = p.S0 ? p.S0[bh * D * D + i * D + j] : 0.f;
-  }
-  for (int t = t_beg; t < t_end; ++t) {
-    if ((t - t_beg) % BWD_CK == 0) {
-      float* c = ck + static_cast<long long>((t - t_beg) / BWD_CK) * D * D;
+  for (int i = 0; i < D; ++i) S[i] = p.S0 ? p.S0[bh * D * D + i * D + j] : 0.f;
+  for (int t = 0; t < p.N; ++t) {
+    if (t % BWD_CK == 0) {
+      float* c = ck + static_cast<long long>(t / BWD_CK) * D * D;
 #pragma unroll
       for (int i = 0; i < D; ++i) c[i * D + j] = S[i];
     }
@@ -537,16 +524,10 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
     step(t, 0, false);
   }
   // ---- reverse, one chunk of BWD_CK tokens at a time
-  if (p.Gin) {
 #pragma unroll
-    for (int i = 0; i < D; ++i) G[i * LDG + j] = p.Gin[bhs * D * D + i * D + j];
-  } else {
-#pragma unroll
-    for (int i = 0; i < D; ++i) G[i * LDG + j] = 0.f;
-  }
-  const int nck_here = (t_end - t_beg + BWD_CK - 1) / BWD_CK;
-  for (int c = nck_here - 1; c >= 0; --c) {
-    const int t0 = t_beg + c * BWD_CK, t1 = min(t_end, t0 + BWD_CK);
+  for (int i = 0; i < D; ++i) G[i * LDG + j] = 0.f;
+  for (int c = p.nck - 1; c >= 0; --c) {
+    const int t0 = c * BWD_CK, t1 = min(p.N, t0 + BWD_CK);
     const float* cs = ck + static_cast<long long>(c) * D * D;
 #pragma unroll
     for (int i = 0; i < D; ++i) S[i] = cs[i * D + j];
@@ -571,7 +552,7 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
       kv[j] = p.k[r + j];
       vv[j] = p.v[r + j];
       dv_[j] = p.dout[r + j];
-      av[j] = p.delta ? (j == 0 ? gate_a(t, 0) : 0.f) : gate_a(t, j);
+      av[j] = j == 0 ? gate_a(t) : 0.f;
       const float* src = t == t0 ? cs : buf + static_cast<long long>(t - t0 - 1) * D * D;
       for (int i = 0; i < D; ++i) prv[i * LDG + j] = src[i * D + j];
       __syncthreads();
@@ -581,75 +562,54 @@ __global__ void __launch_bounds__(D) lin_bwd_f32_kernel(const LinBwdParams p) {
 #pragma unroll
       for (int i = 0; i < D; ++i) G[i * LDG + j] = fmaf(p.scale * qv[i], dv_[j], G[i * LDG + j]);
       __syncthreads();
-      if (!p.delta) {
-        // column j: dv; row j: dq, dk, dalpha
-        float acc = 0.f;
+      const float a = av[0], be = gate_b(t), ae = p.erase_decayed ? a : 1.f;
+      const int tl = t - t0;
+      float acc = 0.f;
 #pragma unroll
-        for (int i = 0; i < D; ++i) acc = fmaf(kv[i], G[i * LDG + j], acc);
-        p.dv[r + j] = acc;
-        const int i = j;
-        float aq = 0.f, ak = 0.f, aa = 0.f;
-        for (int jj = 0; jj < D; ++jj) {
-          aq = fmaf(St[i * LDG + jj], dv_[jj], aq);
-          ak = fmaf(G[i * LDG + jj], vv[jj], ak);
-          aa = fmaf(G[i * LDG + jj], Sp[i * LDG + jj], aa);
-        }
-        p.dq[r + i] = p.scale * aq;
-        p.dk[r + i] = ak;
-        p.dalpha[((rb + t) * p.H + h) * D + i] = aa;
-        __syncthreads();
-#pragma unroll
-        for (int ii = 0; ii < D; ++ii) G[ii * LDG + j] *= av[ii];
-      } else {
-        const float a = av[0], be = gate_b(t), ae = p.erase_decayed ? a : 1.f;
-        const int tl = t - t0;
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < D; ++i) acc = fmaf(kv[i], G[i * LDG + j], acc);
-        du[j] = acc;
-        p.dv[r + j] = be * acc;
-        const float wj = Wb[tl * D + j];
-        red[j] = acc * (vv[j] - ae * wj);                         // dbeta terms
-        float dal = p.erase_decayed ? -be * acc * wj : 0.f;       // dalpha terms (column part)
-        __syncthreads();
-        const int i = j;
-        float aq = 0.f, ak = 0.f, as = 0.f;
-        for (int jj = 0; jj < D; ++jj) {
-          aq = fmaf(St[i * LDG + jj], dv_[jj], aq);
-          ak = fmaf(G[i * LDG + jj], Ub[tl * D + jj], ak);
-          as = fmaf(Sp[i * LDG + jj], du[jj], as);
-          dal = fmaf(G[i * LDG + jj], Sp[i * LDG + jj], dal);
-        }
-        p.dq[r + i] = p.scale * aq;
-        p.dk[r + i] = ak - be * ae * as;
-        red[D + j] = dal;
-        __syncthreads();
-        if (j < 32) {  // block sums of the dbeta and dalpha terms
-          float sb = 0.f, sa = 0.f;
-          for (int e = j; e < D; e += 32) {
-            sb += red[e];
-            sa += red[D + e];
-          }
-          for (int o2 = 16; o2; o2 >>= 1) {
-            sb += __shfl_xor_sync(0xffffffffu, sb, o2);
-            sa += __shfl_xor_sync(0xffffffffu, sa, o2);
-          }
-          if (j == 0) {
-            p.dbeta[(rb + t) * p.H + h] = sb;
-            p.dalpha[(rb + t) * p.H + h] = sa;
-          }
-        }
-#pragma unroll
-        for (int ii = 0; ii < D; ++ii)
-          G[ii * LDG + j] = a * G[ii * LDG + j] - be * ae * kv[ii] * du[j];
+      for (int i = 0; i < D; ++i) acc = fmaf(kv[i], G[i * LDG + j], acc);
+      du[j] = acc;
+      p.dv[r + j] = be * acc;
+      const float wj = Wb[tl * D + j];
+      red[j] = acc * (vv[j] - ae * wj);                         // dbeta terms
+      float dal = p.erase_decayed ? -be * acc * wj : 0.f;       // dalpha terms (column part)
+      __syncthreads();
+      const int i = j;
+      float aq = 0.f, ak = 0.f, as = 0.f;
+      for (int jj = 0; jj < D; ++jj) {
+        aq = fmaf(St[i * LDG + jj], dv_[jj], aq);
+        ak = fmaf(G[i * LDG + jj], Ub[tl * D + jj], ak);
+        as = fmaf(Sp[i * LDG + jj], du[jj], as);
+        dal = fmaf(G[i * LDG + jj], Sp[i * LDG + jj], dal);
       }
+      p.dq[r + i] = p.scale * aq;
+      p.dk[r + i] = ak - be * ae * as;
+      red[D + j] = dal;
+      __syncthreads();
+      if (j < 32) {  // block sums of the dbeta and dalpha terms
+        float sb = 0.f, sa = 0.f;
+        for (int e = j; e < D; e += 32) {
+          sb += red[e];
+          sa += red[D + e];
+        }
+        for (int o2 = 16; o2; o2 >>= 1) {
+          sb += __shfl_xor_sync(0xffffffffu, sb, o2);
+          sa += __shfl_xor_sync(0xffffffffu, sa, o2);
+        }
+        if (j == 0) {
+          p.dbeta[(rb + t) * p.H + h] = sb;
+          p.dalpha[(rb + t) * p.H + h] = sa;
+        }
+      }
+#pragma unroll
+      for (int ii = 0; ii < D; ++ii)
+        G[ii * LDG + j] = a * G[ii * LDG + j] - be * ae * kv[ii] * du[j];
       __syncthreads();
       float* tmp = cur;
       cur = prv;
       prv = tmp;
     }
   }
-  if (p.dS0 && p.nseg == 1) {
+  if (p.dS0) {
 #pragma unroll
     for (int i = 0; i < D; ++i) p.dS0[bh * D * D + i * D + j] = G[i * LDG + j];
   }

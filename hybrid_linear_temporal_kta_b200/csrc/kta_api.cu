@@ -990,21 +990,18 @@ template <int D>
 kta_status launch_lin_bwd(kta::LinBwdParams p, int B, cudaStream_t st) {
   const long long bh = static_cast<long long>(B) * p.H;
   if (p.delta) {
-    // The delta rule's segment carry would need dense d x d transitions: one segment per
+    // The delta rule's segment carry would need dense d x d transitions: one CTA per
     // (sequence, head), states checkpointed every BWD_CK tokens and recomputed per chunk.
-    p.nseg = 1;
-    p.seg_len = p.N;
     p.nck = (p.N + kta::BWD_CK - 1) / kta::BWD_CK;
-    p.Sin = p.Gin = nullptr;
     void* ws = nullptr;
     kta_status r = workspace(static_cast<size_t>(kta::lin_bwd_ws_floats<D>(p.nck)) * bh *
                                  sizeof(float), st, &ws);
     if (r) return r;
     p.ws = static_cast<float*>(ws);
     const size_t smem = (3 * static_cast<size_t>(D) * (D + 1) + 8 * D) * sizeof(float);
-    if ((r = set_smem_attr(kta::lin_bwd_f32_kernel<D>, smem))) return r;
+    if ((r = set_smem_attr(kta::delta_bwd_f32_kernel<D>, smem))) return r;
     TraceScope ts("delta_bwd_f32", st);
-    kta::lin_bwd_f32_kernel<D><<<dim3(p.H, B, 1), D, smem, st>>>(p);
+    kta::delta_bwd_f32_kernel<D><<<dim3(p.H, B), D, smem, st>>>(p);
     KTA_CUDA(cudaGetLastError());
     return KTA_OK;
   }

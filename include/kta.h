@@ -219,9 +219,10 @@ kta_status kta_proj_fwd(const void* x, const void* w, int M, int N, int K,
  * matching forward call, in fp32 on CUDA cores: s.dtype must be KTA_F32, else
  * KTA_ERR_UNSUPPORTED. Every tensor uses its forward layout (q, k, v, dout, dq, dk, dv:
  * [B][N][ld_heads][d]; heads [0, H) are read and written, other heads untouched). Gradients are
- * overwritten, not accumulated. The linear branches recompute states from checkpoints and take
- * (ceil(N/32) + 32) * d * d + 64 * d floats of workspace per (sequence, head) from the calling
- * stream's workspace cache.
+ * overwritten, not accumulated. Workspace, from the calling stream's cache: the softmax branches
+ * 3 floats per (row, head); vector GLA N * d floats + N * d doubles per (sequence, head) plus
+ * 2 d*d + 2 d + 2 d*d floats and d doubles per sequence segment; the delta rule
+ * (ceil(N/32) + 32) * d * d + 64 * d floats per (sequence, head) (checkpointed states).
  *
  * kta_swa_bwd / kta_dswa_bwd: with p_ts the forward's softmax weights over the visible keys,
  *     ds_ts = p_ts (dout_t . v_s - dout_t . o_t),  dq_t = scale sum_s ds_ts k_s,
@@ -255,7 +256,10 @@ kta_status kta_softmax_bwd_bf16(const void* q, const void* k, const void* v, con
  * kta_gla_bwd: gradients of kta_gla_chunk_fwd's output. With the state adjoint
  * G_t = scale q_t^T dout_t + diag(alpha_{t+1}) G_{t+1} (G after the last token = 0):
  *     dq_t = scale S_t dout_t^T,  dk_t = G_t v_t^T,  dv_t = k_t G_t,
- *     dalpha_t[i] = sum_j G_t[i][j] S_{t-1}[i][j],  dS0 = diag(alpha_1) G_1.
+ *     dalpha_t[i] = sum_j G_t[i][j] S_{t-1}[i][j],  dS0 = diag(alpha_1) G_1,
+ * the gate gradient evaluated through its equal log-gate form
+ * dalpha_t = (1/alpha_t) sum_{u >= t} (q_u (.) dq_u - k_u (.) dk_u) (sums in fp64; accuracy
+ * degrades for gates near 0).
  * dalpha: [B][N][H][d] fp32 (required). S0 as in the forward or NULL; dS0: [B][H][d][d] or NULL.
  */
 kta_status kta_gla_bwd(const void* q, const void* k, const void* v, const float* alpha,
