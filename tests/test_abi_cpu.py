@@ -23,12 +23,15 @@ def declared_entry_points():
     return sorted(set(re.findall(r"\b(kta_[a-z0-9_]+)\s*\(", text)))
 
 
-def test_header_declares_the_survey_entry_points():
+def test_header_declares_the_operator_entry_points():
     names = declared_entry_points()
     for n in ("kta_swa_fwd", "kta_dswa_fwd", "kta_gla_chunk_fwd", "kta_gla_delta_fwd",
-              "kta_hybrid_fwd", "kta_stream_create", "kta_stream_step", "kta_stream_reset",
+              "kta_gla_gdn_fwd", "kta_hybrid_fwd", "kta_hybrid_fwd_window", "kta_state_affine",
+              "kta_stream_create", "kta_stream_step", "kta_stream_reset",
               "kta_stream_state_bytes", "kta_stream_save", "kta_stream_load",
-              "kta_stream_destroy", "kta_status_str"):
+              "kta_stream_destroy", "kta_status_str", "kta_proj_fwd", "kta_softmax_fwd_lse",
+              "kta_softmax_bwd_bf16", "kta_swa_bwd", "kta_dswa_bwd", "kta_gla_bwd",
+              "kta_gla_delta_bwd"):
         assert n in names
 
 

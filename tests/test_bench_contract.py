@@ -52,3 +52,20 @@ def test_workload_algebra_matches_the_layer():
     assert bench.gla_bytes(w) == 12 * 128 * 32760 * 8
     d = synth.DELTA_BF16
     assert bench.delta_bytes(d) == pytest.approx(2.164e9, rel=1e-3)
+
+
+def test_projection_and_backward_algebra():
+    sys.path.insert(0, ROOT)
+    import bench
+    from hybrid_linear_temporal_kta_b200 import synth
+    w = synth.HYBRID_BF16
+    # stacked q/k/v/alpha projection: 32,760 rows x 3,072 inputs x (3 x 3,072 + 8 x 128 = 10,240)
+    # outputs, plus the 3,072 x 3,072 output projection; 2 FLOP per multiply-add
+    assert bench.layer_proj_flops(w) == 2 * 32760 * 3072 * 10240 + 2 * 32760 * 3072 * 3072
+    assert bench.layer_proj_flops(w) == 2_679_405_281_280
+    # fp32 backward: S, dP, dQ (6d) in the query-major kernel, S, dP, dV, dK (8d) key-major
+    fl = bench.softmax_bwd_flops(w)
+    assert fl["softmax_bwd_q_f32"] == 6 * 128 * 2_453_068_800
+    assert fl["softmax_bwd_kv_f32"] == 8 * 128 * 2_453_068_800
+    # fp32 FMA peak at 1965 MHz: 148 SMs x 128 lanes x 2 FLOP
+    assert bench.fp32_alu_tflops(1965.0) == pytest.approx(74.44992)

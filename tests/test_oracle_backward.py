@@ -110,3 +110,44 @@ def test_delta_backward_matches_finite_differences(erase_decayed):
                                                erase_decayed=erase_decayed)
     for arr, g in ((q, dq), (k, dk), (v, dv), (a, da), (be, db), (S0, dS0)):
         check(loss, arr, g)
+
+
+def test_gla_gate_gradient_equals_log_gate_form():
+    """The GLA gate gradient the oracle forms directly, sum_j G_t[i][j] S_{t-1}[i][j], equals the
+    log-gate form (1 / alpha_t) sum_{u >= t} (q_u dq_u - k_u dk_u) built from the oracle's own dq
+    and dk (q enters as q e^{b_t}, k as k e^{-b_t}, b_t the cumulative log gate): the identity
+    the GPU's stateless GLA backward evaluates."""
+    B, N, H, d = 2, 23, 2, 5
+    q, k, v = grid((B, N, H, d)), grid((B, N, H, d)), grid((B, N, H, d))
+    a = grid((B, N, H, d), 0.3, 0.97)
+    S0 = RNG.standard_normal((B, H, d, d))
+    do = RNG.standard_normal((B, N, H, d))
+    dq, dk, dv, da, dS0 = oracle.gla_bwd(q, k, v, a, do, scale=0.7, S0=S0)
+    y = q.astype(np.float64) * dq - k.astype(np.float64) * dk
+    suffix = np.flip(np.cumsum(np.flip(y, axis=1), axis=1), axis=1)
+    np.testing.assert_allclose(suffix / a.astype(np.float64), da, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("form", ["gla", "delta", "gdn"])
+def test_state_after_a_run_is_affine_in_the_entering_state(form):
+    """S_end(S0) = T S0 + E with E = S_end(0) and T = S_end(I) for v = 0: the map the
+    sequence-sharded forward folds across ranks (checked on random entering states)."""
+    B, N, H, d = 1, 17, 2, 4
+    q, k, v = grid((B, N, H, d)), grid((B, N, H, d)), grid((B, N, H, d))
+    if form == "gla":
+        a = grid((B, N, H, d), 0.5, 0.99)
+
+        def run(vv, S):
+            return oracle.gla(q, k, vv, a, S0=S)[1]
+    else:
+        k = (k / np.linalg.norm(k, axis=-1, keepdims=True)).astype(np.float32)
+        a = grid((B, N, H), 0.5, 0.99)
+        be = grid((B, N, H), 0.1, 0.9)
+
+        def run(vv, S):
+            return oracle.delta(q, k, vv, a, be, S0=S, erase_decayed=form == "gdn")[1]
+    E = run(v, np.zeros((B, H, d, d)))
+    T = run(np.zeros_like(v), np.broadcast_to(np.eye(d), (B, H, d, d)).copy())
+    for _ in range(3):
+        S0 = RNG.standard_normal((B, H, d, d))
+        np.testing.assert_allclose(run(v, S0), T @ S0 + E, rtol=1e-10, atol=1e-12)
