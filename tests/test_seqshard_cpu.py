@@ -144,7 +144,7 @@ def _worker(rank, world, port, cfg_kw, qout):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,gla_delta", [(2, 0), (3, 0), (3, 1), (2, 2)])
+@pytest.mark.parametrize("world,gla_delta", [(2, 0), (3, 0), (3, 1), (2, 2), (4, 0)])
 def test_sharded_forward_equals_whole_sequence(world, gla_delta):
     cfg_kw = dict(F=7, P=6, d=8, n_swa=1, n_dswa=1, n_gla=1, W_swa=2, W_dswa=3, dil=2,
                   gla_delta=gla_delta, chunk=16)
