@@ -108,6 +108,10 @@ kta_status kta_dswa_fwd(const void* q, const void* k, const void* v, void* o, kt
  * dims). alpha: [B][N][H][d] fp32 in (0,1). S0: [B][H][d][d] initial state or NULL (= 0).
  * S_out: [B][H][d][d] final state or NULL. chunk in {16, 32, 64} (the token block of the
  * chunked form; results do not depend on it beyond rounding).
+ * Range (bf16 chunked path): the kernel scales q and k by gate products taken from the middle
+ * token of each chunk, so the product of any chunk/2 consecutive gates of one key dim must stay
+ * above 2^-126 (average gate above ~0.065 for chunk 64, ~4e-3 for 32, ~2e-5 for 16); smaller
+ * products overflow to inf. The KTA_F32 path and the delta rule have no such limit.
  */
 kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
                              const float* S0, float* S_out, void* o, kta_shape s, int H,
