@@ -124,3 +124,58 @@ def test_selftest_budget_is_validated(kta):
     assert kta.raw_call("kta_selftest_wait_timeout", ctypes.c_longlong(0), ctypes.c_void_p(0)) == 1
     assert kta.raw_call("kta_selftest_wait_timeout", ctypes.c_longlong(1 << 40),
                         ctypes.c_void_p(0)) == 1
+
+
+def test_new_entry_points_validate_before_any_launch(kta):
+    """Projection, reverse-mode and sequence-split entry points: argument errors come back before
+    any CUDA call (fake pointers are never dereferenced)."""
+    good = ctypes.c_void_p(0x10000)
+    null = ctypes.c_void_p(0)
+    st = ctypes.c_void_p(0)
+    seg = (kta.ProjSeg * 2)()
+    seg[0] = kta.ProjSeg(0, 8, 0x10000, 8, kta.PROJ_BF16, None)
+    seg[1] = kta.ProjSeg(8, 16, 0x20000, 8, kta.PROJ_SIGMOID_F32, None)
+    assert kta.raw_call("kta_proj_fwd", null, good, 4, 16, 64, seg, 2, st) == 1      # null x
+    assert kta.raw_call("kta_proj_fwd", ctypes.c_void_p(0x10004), good, 4, 16, 64, seg, 2, st) == 3
+    assert kta.raw_call("kta_proj_fwd", good, good, 4, 16, 12, seg, 2, st) == 3       # K % 8
+    assert kta.raw_call("kta_proj_fwd", good, good, 4, 16, 64, seg, 0, st) == 1       # no ranges
+    assert kta.raw_call("kta_proj_fwd", good, good, 4, 12, 64, seg, 2, st) == 1       # past N
+    over = (kta.ProjSeg * 2)()
+    over[0] = kta.ProjSeg(0, 8, 0x10000, 8, kta.PROJ_BF16, None)
+    over[1] = kta.ProjSeg(4, 12, 0x20000, 8, kta.PROJ_F32, None)
+    assert kta.raw_call("kta_proj_fwd", good, good, 4, 16, 64, over, 2, st) == 1      # overlap
+    over[1] = kta.ProjSeg(8, 16, 0x20000, 8, 7, None)
+    assert kta.raw_call("kta_proj_fwd", good, good, 4, 16, 64, over, 2, st) == 1      # bad mode
+    over[1] = kta.ProjSeg(8, 16, 0x20000, 4, kta.PROJ_F32, None)
+    assert kta.raw_call("kta_proj_fwd", good, good, 4, 16, 64, over, 2, st) == 1      # ld < width
+
+    s_bf = _shape(kta)
+    s_f32 = _shape(kta, dt=1)
+    # bf16 reverse mode and its forward: bf16 and d in {64, 128} only; lse required
+    assert kta.raw_call("kta_softmax_fwd_lse", good, good, good, good, good, s_f32, 1, 1, 2, 1,
+                        0.1, st) == 2
+    assert kta.raw_call("kta_softmax_fwd_lse", good, good, good, good, null, s_bf, 1, 1, 2, 1,
+                        0.1, st) == 1
+    assert kta.raw_call("kta_softmax_bwd_bf16", good, good, good, good, good, good, good, good,
+                        good, s_f32, 1, 1, 2, 1, 0.1, st) == 2
+    assert kta.raw_call("kta_softmax_bwd_bf16", good, good, good, good, null, good, good, good,
+                        good, s_bf, 1, 1, 2, 1, 0.1, st) == 1
+    assert kta.raw_call("kta_softmax_bwd_bf16", good, good, good, good, good, good, good, good,
+                        good, s_bf, 1, 1, 0, 1, 0.1, st) == 1
+    # fp32 reverse mode refuses bf16; GLA gates required
+    assert kta.raw_call("kta_swa_bwd", good, good, good, good, good, good, good, s_bf, 1, 1, 2,
+                        0.1, st) == 2
+    assert kta.raw_call("kta_gla_bwd", good, good, good, null, null, good, good, good, good, good,
+                        null, s_f32, 1, 1, 1.0, st) == 1
+    # windowed hybrid: f0 range, one sequence for f0 > 0, aligned states
+    cfg = kta.hybrid_cfg(B=2, F=3, P=16, d=64, n_swa=1, n_dswa=0, n_gla=0)
+    assert kta.raw_call("kta_hybrid_fwd_window", ctypes.byref(cfg), 3, good, good, good, None,
+                        None, None, None, good, st) == 1
+    assert kta.raw_call("kta_hybrid_fwd_window", ctypes.byref(cfg), 1, good, good, good, None,
+                        None, None, None, good, st) == 2
+    assert kta.raw_call("kta_hybrid_fwd_window", ctypes.byref(cfg), 0, good, good, good, None,
+                        None, ctypes.c_void_p(0x10004), None, good, st) == 3
+    # state composition: sizes and aliasing
+    assert kta.raw_call("kta_state_affine", good, good, None, good, 0, 8, st) == 1
+    assert kta.raw_call("kta_state_affine", good, ctypes.c_void_p(0x20000), None, good, 1, 8,
+                        st) == 1
