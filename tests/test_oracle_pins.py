@@ -48,6 +48,59 @@ def gla_closed_form(q, k, v, a, scale, S0=None):
     return scale * o
 
 
+def gla_chunked_middle_reference(q, k, v, a, scale, C, S0, dtype=np.float64):
+    """The chunked GLA algebra of the bf16 kernel, written out: per chunk, b_t = cumulative log2
+    gate, m the middle token, Qi_t = q_t 2^(b_t - b_m), Ki_s = k_s 2^(b_m - b_s),
+    o_t = scale [Qi_t (2^(b_m) S_0) + sum_{s<=t} (Qi_t . Ki_s) v_s],
+    S_end = 2^(b_C - b_m) (2^(b_m) S_0 + Ki^T V). Evaluated in `dtype`."""
+    q, k, v, a = (x.astype(dtype) for x in (q, k, v, a))
+    N, d = q.shape
+    S = S0.astype(dtype).copy()
+    o = np.zeros((N, d), dtype=dtype)
+    with np.errstate(over="ignore", invalid="ignore"):
+        for c0 in range(0, N, C):
+            n = min(C, N - c0)
+            b = np.cumsum(np.log2(a[c0:c0 + n]), axis=0)
+            bm = b[min(C // 2, n - 1)]
+            Qi = q[c0:c0 + n] * np.exp2(b - bm)
+            Ki = k[c0:c0 + n] * np.exp2(bm - b)
+            Sm = np.exp2(bm)[:, None] * S
+            A = np.tril(Qi @ Ki.T)
+            o[c0:c0 + n] = scale * (Qi @ Sm + A @ v[c0:c0 + n])
+            S = np.exp2(b[-1] - bm)[:, None] * (Sm + Ki.T @ v[c0:c0 + n])
+    return o, S
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+def test_gla_equals_middle_reference_chunked_form(C):
+    """The bf16 kernel's chunked algebra equals the oracle's token recurrence (fp64)."""
+    N, d = 150, 8
+    q, k, v = rnd(N, d), rnd(N, d), rnd(N, d)
+    a = gates(N, d, lo=0.5)
+    S0 = RNG.standard_normal((d, d))
+    o, S = oracle.gla(q[None, :, None], k[None, :, None], v[None, :, None], a[None, :, None],
+                      scale=0.8, S0=S0[None, None])
+    ref, Sref = gla_chunked_middle_reference(q, k, v, a, 0.8, C, S0)
+    assert relerr(o[0, :, 0], ref) < 1e-11
+    assert relerr(S[0, 0], Sref) < 1e-11
+
+
+def test_middle_reference_range_limit_in_fp32():
+    """In fp32 the middle-reference factors overflow once the product of C/2 consecutive gates
+    falls below 2^-126 (the documented limit of the bf16 kernel), and not before."""
+    N, d, C = 64, 4, 64
+    q, k, v = rnd(N, d), rnd(N, d), rnd(N, d)
+    S0 = np.zeros((d, d))
+    inside = np.full((N, d), 0.08, dtype=np.float32)     # 32 * log2(0.08) = -116.6
+    outside = np.full((N, d), 0.05, dtype=np.float32)    # 32 * log2(0.05) = -138.3
+    o_in, _ = gla_chunked_middle_reference(q, k, v, inside, 1.0, C, S0, dtype=np.float32)
+    o_out, _ = gla_chunked_middle_reference(q, k, v, outside, 1.0, C, S0, dtype=np.float32)
+    ref_in = oracle.gla(q[None, :, None], k[None, :, None], v[None, :, None],
+                        inside[None, :, None])[0][0, :, 0]
+    assert np.all(np.isfinite(o_in)) and relerr(o_in, ref_in) < 1e-5
+    assert not np.all(np.isfinite(o_out))
+
+
 @pytest.mark.parametrize("N,d,with_s0", [(1, 4, False), (37, 8, False), (24, 6, True)])
 def test_gla_recurrence_equals_quadratic_closed_form(N, d, with_s0):
     B, H = 2, 3
