@@ -480,3 +480,49 @@ def test_delta_error_stays_below_contraction_bound():
         assert err <= xi / (1 - rho) * (1 + 1e-9)
         err_prev = err
     assert err_prev > 0
+
+
+# ----------------------------------------------------------------------------- hybrid head split
+
+
+@pytest.mark.parametrize("gla_delta", [0, 1, 2])
+def test_hybrid_head_slices_equal_branches_on_those_heads_alone(gla_delta):
+    """The hybrid (per-head split, outputs concatenated by head) places each branch on its own
+    head range: every head slice equals the branch run on a tensor holding only those heads, so
+    a wrong head offset, a swapped branch or a branch reading another head's data fails here."""
+    B, F, P, d = 2, 5, 6, 8
+    n_swa, n_dswa, n_gla = 2, 1, 2
+    H, N = n_swa + n_dswa + n_gla, F * P
+    q, k, v = rnd(B, N, H, d), rnd(B, N, H, d), rnd(B, N, H, d)
+    if gla_delta:
+        kn = k[:, :, n_swa + n_dswa:]
+        k[:, :, n_swa + n_dswa:] = kn / np.linalg.norm(kn, axis=-1, keepdims=True)
+        alpha, beta = gates(B, N, n_gla), gates(B, N, n_gla, lo=0.1, hi=0.9)
+    else:
+        alpha, beta = gates(B, N, n_gla, d), None
+    W_swa, W_dswa, dil, sc = 2, 2, 2, d ** -0.5
+    o, S = oracle.hybrid(q, k, v, alpha, beta, P=P, n_swa=n_swa, n_dswa=n_dswa, n_gla=n_gla,
+                         W_swa=W_swa, W_dswa=W_dswa, dil=dil, gla_delta=gla_delta,
+                         scale_softmax=sc, scale_gla=0.5)
+    assert np.all(np.isfinite(o))
+
+    def only(x, h0, h1):
+        return np.ascontiguousarray(x[:, :, h0:h1])
+
+    hs = (0, n_swa)
+    r = oracle.swa(only(q, *hs), only(k, *hs), only(v, *hs), P, W_swa, sc)
+    np.testing.assert_array_equal(o[:, :, 0:n_swa], r)
+    hd = (n_swa, n_swa + n_dswa)
+    r = oracle.dswa(only(q, *hd), only(k, *hd), only(v, *hd), P, W_dswa, dil, sc)
+    np.testing.assert_array_equal(o[:, :, hd[0]:hd[1]], r)
+    hg = (n_swa + n_dswa, H)
+    if gla_delta:
+        r, Sr = oracle.delta(only(q, *hg), only(k, *hg), only(v, *hg), alpha, beta, 0.5,
+                             erase_decayed=gla_delta == 2)
+    else:
+        r, Sr = oracle.gla(only(q, *hg), only(k, *hg), only(v, *hg), alpha, 0.5)
+    np.testing.assert_array_equal(o[:, :, hg[0]:], r)
+    np.testing.assert_array_equal(S, Sr)
+    # the three branches really differ on these inputs (the check above is not vacuous)
+    r_swa_on_gla = oracle.swa(only(q, *hg), only(k, *hg), only(v, *hg), P, W_swa, sc)
+    assert relerr(r_swa_on_gla, o[:, :, hg[0]:]) > 0.1
