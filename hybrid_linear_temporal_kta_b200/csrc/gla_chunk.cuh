@@ -4,17 +4,24 @@
 // Operator (paper-read "Kairos: A Native World Model Stack for Physical AI", section 2, second
 // pillar, GLA paragraph): S_t = diag(alpha_t) S_{t-1} + k_t^T v_t, o_t = scale * q_t S_t.
 //
-// Chunked form used here (exact algebra, C tokens per chunk, chunks aligned to multiples of C
-// from token 0). Let b_t = sum_{r <= t in chunk} log2 alpha_r (a vector over key dims), m the
-// chunk's middle token, S_0 the state at the chunk start, and
+// Chunked form used here (exact algebra; spans of C tokens aligned to multiples of C from token
+// 0). Let b_t = sum_{r <= t in span} log2 alpha_r (a vector over key dims), m = n/2 the span's
+// middle token (n valid tokens), S_0 the state at the span start, and
 //   Qi_t = q_t * 2^{b_t - b_m},   Ki_s = k_s * 2^{b_m - b_s}   (elementwise over key dims).
 // Then
 //   o_t   = scale * [ Qi_t (diag(2^{b_m}) S_0) + sum_{s <= t} (Qi_t . Ki_s) v_s ]
 //   S_end = diag(2^{b_C - b_m}) [ diag(2^{b_m}) S_0 + Ki^T V ]
 // so one pair of decayed operands (one exp2 each per element) serves the intra-chunk scores, the
-// inter-chunk read-out and the state update. The middle reference point keeps both factors of the
-// intra-chunk product within 2^{|b| over half a chunk}; every other factor is <= 1.
+// inter-chunk read-out and the state update.
 //
+// Gate range. Qi and Ki carry 2^{b_t - b_m} and 2^{b_m - b_s}, which exceed 1 on one side of the
+// middle token; for gates near 0 they would leave the fp32 / bf16 range. So every span checks,
+// per key dim, that |b_t - b_m| <= KTA_GLA_LIM (64 bits) for all its tokens. If any dim fails,
+// the span is redone as sub-spans of 16 tokens (each with its own middle token), and a 16-token
+// sub-span that still fails is redone token by token (n = 1: both factors are exactly 1). All
+// three granularities are exact forms of the same recurrence, so the result is exact for every
+// gate in [0, 1]; the finer levels only cost time (about 4x and 64x per affected chunk).
+// log2 of a gate is clamped at -200 so that alpha = 0 gives a factor of 0, not a NaN.
 // Sequence parallelism: the tokens of a sequence are split into segments of whole chunks.
 //   pass 1 (OUTPUT = false): each segment's end state from a zero start, and its total log2 decay;
 //   carry:                   S_start(0) = S0, S_start(s+1) = diag(2^{L_s}) S_start(s) + S_loc(s),
@@ -29,6 +36,10 @@
 #include "mma_sync.cuh"
 
 namespace kta {
+
+#ifndef KTA_GLA_LIM
+#define KTA_GLA_LIM 64.0f
+#endif
 
 struct GlaParams {
   const __nv_bfloat16* q;
@@ -70,7 +81,6 @@ __global__ void __launch_bounds__(128, 3) gla_chunk_kernel(const GlaParams p) {
   constexpr int MT = RW / 16;         // m16 tiles of state per warp
   constexpr int NT = BV / 8;          // n8 tiles across the value slice
   constexpr int RT = C / 16;          // 16-row query tiles per chunk
-  constexpr int MID = C / 2;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SM& sm = *reinterpret_cast<SM*>(smem_raw);
 
@@ -129,9 +139,16 @@ __global__ void __launch_bounds__(128, 3) gla_chunk_kernel(const GlaParams p) {
     }
   };
 
-  for (int c0 = t_begin; c0 < t_end; c0 += C) {
-    const int n = min(C, t_end - c0);
-    // ---- load the chunk: q, k (OUTPUT only for q), v slice, alpha (rows >= n: zeros / alpha = 1)
+  // Spans: C tokens (level 0), 16-token sub-spans (level 1) or single tokens (level 2) when the
+  // coarser span's decayed operands would leave the representable range. lvl_end[l] is where the
+  // region handed down to level l ends.
+  int lvl = 0;
+  int lvl_end[3] = {t_end, t_end, t_end};
+  for (int c0 = t_begin; c0 < t_end;) {
+    const int span = lvl == 0 ? C : (lvl == 1 ? 16 : 1);
+    const int n = min(span, min(t_end, lvl_end[lvl]) - c0);
+    const int mid = n >> 1;
+    // ---- load the span: q, k (OUTPUT only for q), v slice, alpha (rows >= n: zeros / alpha = 1)
     {
       constexpr int QCH = D / 8;  // 16-byte pieces per bf16 row
       for (int idx = tid; idx < C * QCH; idx += 128) {
@@ -159,19 +176,38 @@ __global__ void __launch_bounds__(128, 3) gla_chunk_kernel(const GlaParams p) {
 #pragma unroll
       for (int t = 0; t < C; ++t) bt[t] = t < n ? __ldg(ap + static_cast<long long>(t) * p.H * D) : 1.f;
     }
-    cp_async_wait_all();
-    __syncthreads();
     // ---- per key dim (thread tid < D owns column tid): the cumulative log2 gate b_t in
-    // registers, the factors 2^{b_m}, 2^{b_C - b_m}, and the decayed operands of its column,
-    // Ki_t = k_t 2^{b_m - b_t} and Qi_t = q_t 2^{b_t - b_m}, written in place
+    // registers and the range check of the decayed operands against the middle token
+    float bm = 0.f, acc = 0.f;
+    bool in_range = true;
     if (tid < D) {
-      float acc = 0.f;
 #pragma unroll
       for (int t = 0; t < C; ++t) {
-        acc += __log2f(bt[t]);
+        acc += fmaxf(__log2f(bt[t]), -200.f);
         bt[t] = acc;
       }
-      const float bm = bt[MID];
+#pragma unroll
+      for (int t = 0; t < C; ++t) bm = t == mid ? bt[t] : bm;
+      float dev = 0.f;
+#pragma unroll
+      for (int t = 0; t < C; ++t) dev = fmaxf(dev, fabsf(bt[t] - bm));
+      in_range = !(dev > KTA_GLA_LIM);
+    }
+    if (lvl < 2 && !__syncthreads_and(in_range ? 1 : 0)) {
+      // redo this span at the next finer level (the copies above are simply overwritten)
+      cp_async_wait_all();
+      __syncthreads();
+      const int next = (lvl == 0 && C > 16) ? 1 : 2;
+      lvl_end[next] = c0 + n;
+      if (lvl == 0 && next == 2) lvl_end[1] = c0 + n;
+      lvl = next;
+      continue;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // the factors 2^{b_m}, 2^{b_C - b_m}, and the decayed operands of this thread's column,
+    // Ki_t = k_t 2^{b_m - b_t} and Qi_t = q_t 2^{b_t - b_m}, written in place
+    if (tid < D) {
       sm.emid[tid] = ex2_approx(bm);
       sm.cend[tid] = ex2_approx(acc - bm);
       ltot += acc;
@@ -293,6 +329,8 @@ __global__ void __launch_bounds__(128, 3) gla_chunk_kernel(const GlaParams p) {
       }
     }
     __syncthreads();
+    c0 += n;
+    while (lvl > 0 && c0 >= lvl_end[lvl]) --lvl;
   }
 
   if (!OUTPUT) {

@@ -373,11 +373,20 @@ struct LinLaunch {
   bool allow_segments = true;
 };
 
+// Segment plan of the chunked GLA kernels: enough (segment, value slice, sequence-head) CTAs for
+// one wave of three per SM, segments of whole chunks. ws_bytes is the workspace the state pass and
+// the carry pass need (segment end states and total log2 decays; none for a single segment).
+struct GlaPlan {
+  int nseg = 1, seg_len = 0, slices = 1;
+  size_t ws_bytes = 0;
+};
+
 template <int D, int C>
-kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
+GlaPlan gla_plan(const LinLaunch& L) {
   using SM = kta::GlaSmem<D, C>;
-  const int slices = D / SM::BV;
-  const long long base = static_cast<long long>(L.B) * L.H * slices;
+  GlaPlan g;
+  g.slices = D / SM::BV;
+  const long long base = static_cast<long long>(L.B) * L.H * g.slices;
   const int nchunks = (L.N + C - 1) / C;
   int nseg = 1;
   if (L.allow_segments) {
@@ -385,8 +394,18 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
     nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
   }
   const int seg_chunks = (nchunks + nseg - 1) / nseg;
-  const int seg_len = seg_chunks * C;
-  nseg = (L.N + seg_len - 1) / seg_len;
+  g.seg_len = seg_chunks * C;
+  g.nseg = (L.N + g.seg_len - 1) / g.seg_len;
+  g.ws_bytes = g.nseg > 1 ? static_cast<size_t>(L.B) * L.H * g.nseg * (size_t(D) * D + D) * 4 : 0;
+  return g;
+}
+
+// Launch the chunked GLA kernels of a plan with `ws` (ws_bytes of device memory, or null when
+// the plan needs none) as the segment workspace.
+template <int D, int C>
+kta_status launch_gla_planned(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStream_t st) {
+  using SM = kta::GlaSmem<D, C>;
+  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
   kta::GlaParams p{};
   p.q = static_cast<const __nv_bfloat16*>(L.q);
   p.k = static_cast<const __nv_bfloat16*>(L.k);
@@ -397,27 +416,25 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
   p.rows_b = L.rows_b;
   p.N = L.N;
   p.H = L.H;
-  p.seg_len = seg_len;
-  p.nseg = nseg;
+  p.seg_len = g.seg_len;
+  p.nseg = g.nseg;
   p.scale = L.scale;
   p.S0 = L.S0;
   p.S_out = L.S_out;
-  if (nseg > 1) {
-    void* ws = nullptr;
-    const size_t bytes = static_cast<size_t>(L.B) * L.H * nseg * (size_t(D) * D + D) * 4;
-    kta_status s = workspace(bytes, st, &ws);
-    if (s) return s;
+  if (g.nseg > 1) {
+    // Every word the kernels read from the workspace is written earlier in the same call (the
+    // state pass writes all segment states and decays, the carry pass rewrites them in place),
+    // so nothing has to be cleared.
     p.ws_S = static_cast<float*>(ws);
-    p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * nseg * D * D;
+    p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * g.nseg * D * D;
   }
   const size_t smem = sizeof(SM);
   kta_status sa;
   if ((sa = set_smem_attr(kta::gla_chunk_kernel<D, C, false>, smem)) ||
       (sa = set_smem_attr(kta::gla_chunk_kernel<D, C, true>, smem)))
     return sa;
-  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
-  dim3 grid(nseg, slices, L.B * L.H);
-  if (nseg > 1) {
+  dim3 grid(g.nseg, g.slices, L.B * L.H);
+  if (g.nseg > 1) {
     {
       TraceScope ts("gla_chunk_state", st);
       kta::gla_chunk_kernel<D, C, false><<<grid, 128, smem, st>>>(p);
@@ -435,6 +452,17 @@ kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
   }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
+}
+
+template <int D, int C>
+kta_status launch_gla_chunk(const LinLaunch& L, cudaStream_t st) {
+  const GlaPlan g = gla_plan<D, C>(L);
+  void* ws = nullptr;
+  if (g.ws_bytes) {
+    kta_status s = workspace(g.ws_bytes, st, &ws);
+    if (s) return s;
+  }
+  return launch_gla_planned<D, C>(L, g, ws, st);
 }
 
 template <int D>
@@ -1653,66 +1681,21 @@ kta_status noalloc_scratch(void** out) {
   return KTA_OK;
 }
 
-// Same segment plan and kernels as launch_gla_chunk; the workspace is the scratch array.
+// The segment plan and kernels of launch_gla_chunk, with the scratch array as the workspace.
 template <int D, int C>
 kta_status launch_gla_chunk_noalloc(const LinLaunch& L, cudaStream_t st) {
-  using SM = kta::GlaSmem<D, C>;
-  const int slices = D / SM::BV;
-  const long long base = static_cast<long long>(L.B) * L.H * slices;
-  const int nchunks = (L.N + C - 1) / C;
-  const long long want = (3LL * 148 + base - 1) / base;  // one wave of 3 CTAs per SM
-  int nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
-  const int seg_chunks = (nchunks + nseg - 1) / nseg;
-  const int seg_len = seg_chunks * C;
-  nseg = (L.N + seg_len - 1) / seg_len;
-  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
-  const size_t need =
-      nseg > 1 ? static_cast<size_t>(L.B) * L.H * nseg * (size_t(D) * D + D) * 4 : 0;
-  if (need > kNoAllocScratchBytes)
+  const GlaPlan g = gla_plan<D, C>(L);
+  if (g.ws_bytes > kNoAllocScratchBytes)
     return fail(KTA_ERR_UNSUPPORTED,
                 "needs %zu bytes of scratch; the no-allocation variant has %zu (use "
                 "kta_gla_chunk_fwd, or fewer sequences x heads per call)",
-                need, kNoAllocScratchBytes);
-  kta::GlaParams p{};
-  p.q = static_cast<const __nv_bfloat16*>(L.q);
-  p.k = static_cast<const __nv_bfloat16*>(L.k);
-  p.v = static_cast<const __nv_bfloat16*>(L.v);
-  p.alpha = L.alpha;
-  p.o = static_cast<__nv_bfloat16*>(L.o);
-  p.ld = L.ld;
-  p.rows_b = L.rows_b;
-  p.N = L.N;
-  p.H = L.H;
-  p.seg_len = seg_len;
-  p.nseg = nseg;
-  p.scale = L.scale;
-  p.S0 = L.S0;
-  p.S_out = L.S_out;
-  if (nseg > 1) {
-    // Every word the kernels read from the scratch is written earlier in the same call (pass 1
-    // writes all segment states and decays, the carry pass rewrites them in place), so nothing
-    // has to be cleared.
-    void* ws = nullptr;
+                g.ws_bytes, kNoAllocScratchBytes);
+  void* ws = nullptr;
+  if (g.ws_bytes) {
     kta_status r = noalloc_scratch(&ws);
     if (r) return r;
-    p.ws_S = static_cast<float*>(ws);
-    p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * nseg * D * D;
   }
-  const size_t smem = sizeof(SM);
-  KTA_CUDA(cudaFuncSetAttribute(kta::gla_chunk_kernel<D, C, false>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-  KTA_CUDA(cudaFuncSetAttribute(kta::gla_chunk_kernel<D, C, true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-  dim3 grid(nseg, slices, L.B * L.H);
-  if (nseg > 1) {
-    kta::gla_chunk_kernel<D, C, false><<<grid, 128, smem, st>>>(p);
-    KTA_CUDA(cudaGetLastError());
-    kta::gla_carry_kernel<D><<<dim3((D * D + 127) / 128, L.B * L.H), 128, 0, st>>>(p);
-    KTA_CUDA(cudaGetLastError());
-  }
-  kta::gla_chunk_kernel<D, C, true><<<grid, 128, smem, st>>>(p);
-  KTA_CUDA(cudaGetLastError());
-  return KTA_OK;
+  return launch_gla_planned<D, C>(L, g, ws, st);
 }
 
 }  // namespace

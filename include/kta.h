@@ -108,10 +108,12 @@ kta_status kta_dswa_fwd(const void* q, const void* k, const void* v, void* o, kt
  * dims). alpha: [B][N][H][d] fp32 in (0,1). S0: [B][H][d][d] initial state or NULL (= 0).
  * S_out: [B][H][d][d] final state or NULL. chunk in {16, 32, 64} (the token block of the
  * chunked form; results do not depend on it beyond rounding).
- * Range (bf16 chunked path): the kernel scales q and k by gate products taken from the middle
- * token of each chunk, so the product of any chunk/2 consecutive gates of one key dim must stay
- * above 2^-126 (average gate above ~0.065 for chunk 64, ~4e-3 for 32, ~2e-5 for 16); smaller
- * products overflow to inf. The KTA_F32 path and the delta rule have no such limit.
+ * Gate range: every gate in [0, 1] is handled exactly. The bf16 chunked path scales q and k
+ * by gate products taken from the middle token of each chunk; a chunk whose products would
+ * leave the fp32 range (more than 64 bits of decay on one side of the middle token in some key
+ * dim, i.e. gates far below ~0.25 on average) is recomputed as 16-token sub-chunks, and a
+ * sub-chunk that still fails token by token. Small gates therefore cost time (about 4x per
+ * affected chunk, 64x where single tokens are needed, e.g. exact zeros), never accuracy.
  */
 kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
                              const float* S0, float* S_out, void* o, kta_shape s, int H,
@@ -129,7 +131,10 @@ kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const 
  *  - A call whose workspace would exceed 32 MiB (sequences x heads x segments x (d*d + d) x 4
  *    bytes) returns KTA_ERR_UNSUPPORTED with the size it needs, before anything is enqueued.
  *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *    with that device current); make that first call before any stream capture.
+ *    with that device current); make that first call before any stream capture. With lazy
+ *    module loading (the CUDA 12 default) that first call may also load the library's device
+ *    code and so back the array with device memory: make one warm-up call before the region
+ *    in which nothing may allocate. Later calls allocate nothing.
  *  - Every call shares the array and leaves its contents behind; each call writes all the
  *    scratch it reads before reading it, so nothing needs clearing. Calls that overlap on the
  *    GPU (for example on two streams) race on the array: serialise them.

@@ -48,26 +48,45 @@ def gla_closed_form(q, k, v, a, scale, S0=None):
     return scale * o
 
 
-def gla_chunked_middle_reference(q, k, v, a, scale, C, S0, dtype=np.float64):
-    """The chunked GLA algebra of the bf16 kernel, written out: per chunk, b_t = cumulative log2
-    gate, m the middle token, Qi_t = q_t 2^(b_t - b_m), Ki_s = k_s 2^(b_m - b_s),
+GLA_LIM = 64.0  # the bf16 kernel's bound on |b_t - b_m| (bits) for one span's decayed operands
+
+
+def gla_chunked_middle_reference(q, k, v, a, scale, C, S0, dtype=np.float64, fallback=True,
+                                 levels=None):
+    """The chunked GLA algebra of the bf16 kernel, written out. Spans of C tokens; per span
+    b_t = cumulative log2 gate (log2 clamped at -200), m = n // 2 the middle token,
+    Qi_t = q_t 2^(b_t - b_m), Ki_s = k_s 2^(b_m - b_s),
     o_t = scale [Qi_t (2^(b_m) S_0) + sum_{s<=t} (Qi_t . Ki_s) v_s],
-    S_end = 2^(b_C - b_m) (2^(b_m) S_0 + Ki^T V). Evaluated in `dtype`."""
+    S_end = 2^(b_n - b_m) (2^(b_m) S_0 + Ki^T V). With `fallback`, a span whose decayed operands
+    would need |b_t - b_m| > GLA_LIM bits in some key dim is redone as 16-token sub-spans, and a
+    sub-span that still fails token by token. Evaluated in `dtype`; `levels` (a list) collects
+    the granularity used for each span."""
     q, k, v, a = (x.astype(dtype) for x in (q, k, v, a))
     N, d = q.shape
     S = S0.astype(dtype).copy()
     o = np.zeros((N, d), dtype=dtype)
-    with np.errstate(over="ignore", invalid="ignore"):
-        for c0 in range(0, N, C):
-            n = min(C, N - c0)
-            b = np.cumsum(np.log2(a[c0:c0 + n]), axis=0)
-            bm = b[min(C // 2, n - 1)]
+
+    def span(c0, n, lvl):
+        nonlocal S
+        with np.errstate(over="ignore", invalid="ignore", divide="ignore"):
+            b = np.cumsum(np.maximum(np.log2(a[c0:c0 + n]), dtype(-200)), axis=0).astype(dtype)
+            bm = b[n // 2]
+            if fallback and n > 1 and np.max(np.abs(b - bm)) > GLA_LIM:
+                sub = 16 if (lvl == 0 and C > 16) else 1
+                for u in range(0, n, sub):
+                    span(c0 + u, min(sub, n - u), 1 if sub == 16 else 2)
+                return
+            if levels is not None:
+                levels.append(lvl)
             Qi = q[c0:c0 + n] * np.exp2(b - bm)
             Ki = k[c0:c0 + n] * np.exp2(bm - b)
             Sm = np.exp2(bm)[:, None] * S
             A = np.tril(Qi @ Ki.T)
             o[c0:c0 + n] = scale * (Qi @ Sm + A @ v[c0:c0 + n])
             S = np.exp2(b[-1] - bm)[:, None] * (Sm + Ki.T @ v[c0:c0 + n])
+
+    for c0 in range(0, N, C):
+        span(c0, min(C, N - c0), 0)
     return o, S
 
 
@@ -80,25 +99,66 @@ def test_gla_equals_middle_reference_chunked_form(C):
     S0 = RNG.standard_normal((d, d))
     o, S = oracle.gla(q[None, :, None], k[None, :, None], v[None, :, None], a[None, :, None],
                       scale=0.8, S0=S0[None, None])
-    ref, Sref = gla_chunked_middle_reference(q, k, v, a, 0.8, C, S0)
+    lv = []
+    ref, Sref = gla_chunked_middle_reference(q, k, v, a, 0.8, C, S0, levels=lv)
+    assert set(lv) == {0}  # these gates never need the finer spans
     assert relerr(o[0, :, 0], ref) < 1e-11
     assert relerr(S[0, 0], Sref) < 1e-11
 
 
-def test_middle_reference_range_limit_in_fp32():
-    """In fp32 the middle-reference factors overflow once the product of C/2 consecutive gates
-    falls below 2^-126 (the documented limit of the bf16 kernel), and not before."""
+def test_single_middle_reference_overflows_without_the_fallback():
+    """In fp32 one middle reference per 64-token chunk overflows once the product of 32
+    consecutive gates falls below 2^-126: the reason the kernel checks each span's range."""
     N, d, C = 64, 4, 64
     q, k, v = rnd(N, d), rnd(N, d), rnd(N, d)
     S0 = np.zeros((d, d))
-    inside = np.full((N, d), 0.08, dtype=np.float32)     # 32 * log2(0.08) = -116.6
     outside = np.full((N, d), 0.05, dtype=np.float32)    # 32 * log2(0.05) = -138.3
-    o_in, _ = gla_chunked_middle_reference(q, k, v, inside, 1.0, C, S0, dtype=np.float32)
-    o_out, _ = gla_chunked_middle_reference(q, k, v, outside, 1.0, C, S0, dtype=np.float32)
-    ref_in = oracle.gla(q[None, :, None], k[None, :, None], v[None, :, None],
-                        inside[None, :, None])[0][0, :, 0]
-    assert np.all(np.isfinite(o_in)) and relerr(o_in, ref_in) < 1e-5
+    o_out, _ = gla_chunked_middle_reference(q, k, v, outside, 1.0, C, S0, dtype=np.float32,
+                                            fallback=False)
     assert not np.all(np.isfinite(o_out))
+
+
+def _small_gates(kind, N, d):
+    if kind == "const0.05":
+        return np.full((N, d), 0.05, dtype=np.float32)
+    if kind == "uniform":
+        return RNG.uniform(1e-4, 0.1, size=(N, d)).astype(np.float32)
+    if kind == "sigmoid-3":
+        z = RNG.standard_normal((N, d)) - 3.0
+        return (1.0 / (1.0 + np.exp(-z))).astype(np.float32)
+    # mixed: mostly ordinary gates with exact zeros, 1e-30 and 1e-12 sprinkled in
+    a = RNG.uniform(0.3, 0.999, size=(N, d)).astype(np.float32)
+    idx = RNG.choice(N * d, size=N * d // 10, replace=False)
+    a.flat[idx[0::3]] = 0.0
+    a.flat[idx[1::3]] = 1e-30
+    a.flat[idx[2::3]] = 1e-12
+    return a
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("kind", ["const0.05", "uniform", "sigmoid-3", "mixed"])
+def test_ranged_chunked_form_is_finite_and_exact_for_small_gates(C, kind):
+    """With the per-span range check and the 16-token / single-token fallback, the chunked
+    algebra evaluated in fp32 stays finite and equals the oracle's fp64 recurrence (to fp32
+    rounding) for gates down to 0, which are valid forget gates (GLA paragraph: alpha_t in
+    (0, 1))."""
+    N, d = 4 * C + 9, 8
+    q, k, v = rnd(N, d), rnd(N, d), rnd(N, d)
+    a = _small_gates(kind, N, d)
+    S0 = RNG.standard_normal((d, d))
+    o, S = oracle.gla(q[None, :, None], k[None, :, None], v[None, :, None], a[None, :, None],
+                      scale=0.8, S0=S0[None, None])
+    lv = []
+    got, Sg = gla_chunked_middle_reference(q, k, v, a, 0.8, C, S0, dtype=np.float32, levels=lv)
+    assert np.all(np.isfinite(got)) and np.all(np.isfinite(Sg))
+    assert relerr(got, o[0, :, 0]) < 1e-5
+    assert relerr(Sg, S[0, 0]) < 1e-5
+    if kind == "const0.05" and C > 16:
+        # full chunk-level spans fail, their 16-token sub-spans pass (the 9-token tail span is
+        # short enough for level 0)
+        assert lv.count(0) == 1 and lv.count(1) == 4 * (C // 16) and 2 not in lv
+    if kind == "mixed":
+        assert 2 in lv  # zeros need single-token spans
 
 
 @pytest.mark.parametrize("N,d,with_s0", [(1, 4, False), (37, 8, False), (24, 6, True)])
