@@ -884,6 +884,26 @@ kta_status kta_hybrid_fwd_window(const kta_hybrid_cfg* cfg, int f0, const void* 
   return hybrid_common(cfg, f0, q, k, v, alpha, beta, S0, S_out, o, stream);
 }
 
+kta_status kta_gla_transition(const float* alpha, float* T, int B, int N, int H, int d,
+                              void* stream) {
+  if (!alpha || !T) return fail(KTA_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || H <= 0 || N < 0) return fail(KTA_ERR_INVALID_ARG, "need B, H > 0 and N >= 0");
+  if (static_cast<long long>(B) * H > 0x7fffffffLL)
+    return fail(KTA_ERR_UNSUPPORTED, "too many sequences x heads");
+  if (!aligned16(alpha) || !aligned16(T)) return fail(KTA_ERR_ALIGNMENT, "pointers not 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  const unsigned grid = static_cast<unsigned>(B * H);
+  {
+    TraceScope ts("gla_transition", st);
+    if (d == 128) kta::gla_transition_kernel<128><<<grid, 1024, 0, st>>>(alpha, T, N, H);
+    else if (d == 64) kta::gla_transition_kernel<64><<<grid, 512, 0, st>>>(alpha, T, N, H);
+    else if (d == 32) kta::gla_transition_kernel<32><<<grid, 256, 0, st>>>(alpha, T, N, H);
+    else return fail(KTA_ERR_UNSUPPORTED, "d must be 32, 64 or 128 (got %d)", d);
+  }
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
 kta_status kta_state_affine(const float* A, const float* X, const float* E, float* Y, int n, int d,
                             void* stream) {
   if (!A || !X || !Y) return fail(KTA_ERR_INVALID_ARG, "null pointer");

@@ -228,4 +228,36 @@ __global__ void __launch_bounds__(256) state_affine_kernel(const float* __restri
   }
 }
 
+// T = diag(prod_t alpha_t) per (sequence, head): the transition of a vector-gated GLA run, whose
+// end state is S_end = diag(prod_t alpha_t) S_start + S_loc (GLA paragraph: the gate scales the
+// state row of each key dim once per token). alpha: [B][N][H][D] fp32; T: [B][H][D][D]. Eight
+// token groups per key dim sum log2(alpha) (clamped at -200, so a zero gate gives 0), combined
+// in shared memory; the whole D x D matrix is written, zeros off the diagonal.
+template <int D>
+__global__ void __launch_bounds__(D * 8) gla_transition_kernel(const float* __restrict__ alpha,
+                                                               float* __restrict__ T, int N,
+                                                               int H) {
+  __shared__ float part[8][D];
+  __shared__ float diag[D];
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+  const int i = threadIdx.x % D, g = threadIdx.x / D;
+  float acc = 0.f;
+  for (int t = g; t < N; t += 8)
+    acc += fmaxf(__log2f(alpha[((static_cast<long long>(b) * N + t) * H + h) * D + i]), -200.f);
+  part[g][i] = acc;
+  __syncthreads();
+  if (g == 0) {
+    float s = 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s += part[u][i];
+    diag[i] = exp2f(s);
+  }
+  __syncthreads();
+  float* Tb = T + static_cast<long long>(bh) * D * D;
+  for (int e = threadIdx.x; e < D * D; e += D * 8) {
+    const int r = e / D, c = e % D;
+    Tb[e] = r == c ? diag[r] : 0.f;
+  }
+}
+
 }  // namespace kta

@@ -23,9 +23,13 @@
 //                S_X(i+1) finds O_X stable.
 //   warps 2, 3   idle after set-up.
 //   warps 4..7   softmax of tile A; warps 8..11 softmax of tile B: thread <-> query row (TMEM
-//                lane). Row max (three-input max), lazy rescale of O when the max grows by more
-//                than 2^8, P = exp2(S*scale*log2e - m) as bf16 into TMEM (scaling and row sums on
-//                packed fp32 pairs), running row sum; epilogue O / l -> bf16 -> global.
+//                lane). Lazy rescale of O when the row max grows by more than 2^8; after the
+//                first tile the exponentials P = exp2(S*scale*log2e - m) are taken against the
+//                current m while the row max is formed (three-input max), and redone only when
+//                the max grew past that bound, so the max is off the critical path. P goes to
+//                TMEM as bf16 (scaling and row sums on packed fp32 pairs); one arrival per warp
+//                hands P to the MMA thread (128 arrivals on one barrier serialise); epilogue
+//                O / l -> bf16 -> global.
 // While the softmax of one tile runs, the tensor core works on the other tile's products.
 // Every wait is bounded; on a timeout the CTA records it and unwinds to free its TMEM.
 #pragma once
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sm.bar_s[x], 1);
-      mbar_init(&sm.bar_p[x], 128);
+      mbar_init(&sm.bar_p[x], 4);  // one arrival per softmax warp
       mbar_init(&sm.bar_o[x], 1);
     }
     mbar_init(&sm.bar_fin, 1);
@@ -290,57 +294,83 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
       tmem_wait_ld();
       tmem_ld_fence(r);
-      // row maximum of the valid columns (three-input max, four independent partial maxima)
       float mp[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) mp[u] = -INFINITY;
-      if (nv == 128) {
+      const uint64_t sc2 = f32x2_pack(sl2, sl2);
+      uint64_t lp2[2];
+      // P = exp2(S * scale * log2e - mref) as bf16 pairs written over S (the scaling and the row
+      // sums on packed fp32 pairs); with_max also forms the row maximum of a full tile (three-
+      // input max, four partial maxima) alongside the exponentials
+      auto exp_pass = [&](float mref, bool with_max) {
+        const uint64_t nm2 = f32x2_pack(-mref, -mref);
+        lp2[0] = f32x2_pack(0.f, 0.f);
+        lp2[1] = f32x2_pack(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
-          mp[j & 3] = max3f(mp[j & 3], __uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-      } else {
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
-          if (j < nv) mp[j & 3] = fmaxf(mp[j & 3], __uint_as_float(r[j]));
-      }
-      const float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-      const float mnew = fmaxf(m, mx * sl2);
-      // lazy rescale: the reference m moves only when the row maximum grows by more than 2^8
+          for (int j = 0; j < 16; ++j) {
+            const int col = 32 * c + 2 * j;
+            if (with_max)
+              mp[j & 3] = max3f(mp[j & 3], __uint_as_float(r[col]), __uint_as_float(r[col + 1]));
+            float x0, x1;
+            f32x2_unpack(ffma2(f32x2_pack(__uint_as_float(r[col]), __uint_as_float(r[col + 1])), sc2, nm2),
+                         x0, x1);
+            float p0 = ex2_approx(x0);
+            float p1 = ex2_approx(x1);
+            if (nv < 128) {
+              p0 = col < nv ? p0 : 0.f;
+              p1 = col + 1 < nv ? p1 : 0.f;
+            }
+            lp2[j & 1] = fadd2(lp2[j & 1], f32x2_pack(p0, p1));
+            pk[j] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + lane_off + 16 * c, pk);
+        }
+      };
+      // Lazy rescale: the reference m moves only when the row maximum grows by more than 2^8, so
+      // for a full tile after the first the exponentials are taken against the current m while
+      // the maximum is formed, and redone (rarely) when it grew by more than that.
       bool rescale = false;
       float fac = 1.0f;
-      if (i == 0) {
-        m = mnew;
-      } else {
+      if (i > 0 && nv == 128) {
+        exp_pass(m, true);
+        const float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        const float mnew = fmaxf(m, mx * sl2);
         const bool need = mnew > m + 8.0f;
         rescale = __any_sync(0xffffffffu, need);
-        if (need) {
-          fac = ex2_approx(m - mnew);
-          m = mnew;
-        }
-      }
-      // P = exp2(S * scale * log2e - m) as bf16 pairs, written over S (the scaling and the row
-      // sum on packed fp32 pairs)
-      const uint64_t sc2 = f32x2_pack(sl2, sl2), nm2 = f32x2_pack(-m, -m);
-      uint64_t lp2[2] = {f32x2_pack(0.f, 0.f), f32x2_pack(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int col = 32 * c + 2 * j;
-          float x0, x1;
-          f32x2_unpack(ffma2(f32x2_pack(__uint_as_float(r[col]), __uint_as_float(r[col + 1])), sc2, nm2),
-                       x0, x1);
-          float p0 = ex2_approx(x0);
-          float p1 = ex2_approx(x1);
-          if (nv < 128) {
-            p0 = col < nv ? p0 : 0.f;
-            p1 = col + 1 < nv ? p1 : 0.f;
+        if (rescale) {
+          if (need) {
+            fac = ex2_approx(m - mnew);
+            m = mnew;
           }
-          lp2[j & 1] = fadd2(lp2[j & 1], f32x2_pack(p0, p1));
-          pk[j] = pack_bf16x2(p0, p1);
+          tmem_wait_st();
+          exp_pass(m, false);
         }
-        tmem_st16(tS + lane_off + 16 * c, pk);
+      } else {
+        if (nv == 128) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            mp[j & 3] = max3f(mp[j & 3], __uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 128; ++j)
+            if (j < nv) mp[j & 3] = fmaxf(mp[j & 3], __uint_as_float(r[j]));
+        }
+        const float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        const float mnew = fmaxf(m, mx * sl2);
+        if (i == 0) {
+          m = mnew;
+        } else {
+          const bool need = mnew > m + 8.0f;
+          rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            fac = ex2_approx(m - mnew);
+            m = mnew;
+          }
+        }
+        exp_pass(m, false);
       }
       float la, lb, lc, ld;
       f32x2_unpack(lp2[0], la, lb);
@@ -362,7 +392,8 @@ __global__ void __launch_bounds__(384, 1)
       l += (la + lb) + (lc + ld);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.bar_p[x]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.bar_p[x]);
     }
     // epilogue: O / l -> bf16 -> global (rows of this frame only)
     const bool active = x == 0 || has_b;

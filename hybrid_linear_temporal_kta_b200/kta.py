@@ -76,6 +76,7 @@ _SIGS = {
     "kta_hybrid_fwd_window": ([ctypes.POINTER(HybridCfg), _i, _vp, _vp, _vp, _fp, _fp, _fp, _fp,
                                _vp, _vp], _st),
     "kta_state_affine": ([_fp, _fp, _fp, _fp, _i, _i, _vp], _st),
+    "kta_gla_transition": ([_fp, _fp, _i, _i, _i, _i, _vp], _st),
     "kta_stream_create": ([ctypes.POINTER(HybridCfg), ctypes.POINTER(_vp)], _st),
     "kta_stream_step": ([_vp, _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
     "kta_stream_reset": ([_vp, _vp], _st),
@@ -441,6 +442,17 @@ def hybrid_fwd_window(cfg: HybridCfg, f0: int, q, k, v, alpha=None, beta=None, *
                                       _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(S_out), _ptr(o),
                                       _stream(stream)), "kta_hybrid_fwd_window")
     return (o, S_out) if return_state else o
+
+
+def gla_transition(alpha, *, out=None, stream=None):
+    """T = diag(prod_t alpha_t) [B, H, d, d] of a vector-gated GLA run; alpha [B, N, H, d] fp32."""
+    _need(alpha, "alpha", torch.float32)
+    B, N, H, d = alpha.shape
+    T = torch.empty((B, H, d, d), device=alpha.device, dtype=torch.float32) if out is None else out
+    _need(T, "out", torch.float32)
+    _check(_lib.kta_gla_transition(_ptr(alpha), _ptr(T), B, N, H, d, _stream(stream)),
+           "kta_gla_transition")
+    return T
 
 
 def state_affine(A, X, E=None, *, out=None, stream=None):

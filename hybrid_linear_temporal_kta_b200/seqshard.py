@@ -4,11 +4,15 @@ Each rank holds a contiguous run of frames (q, k, v and gates of those frames) a
 their outputs. Two things cross rank boundaries:
 - the softmax heads' K/V halo: the windows of a rank's first frames reach back
   max(W_swa - 1, (W_dswa - 1) * dil) frames (paper-read, section 2, second pillar, SWA and DSWA
-  paragraphs), gathered from the preceding ranks with one all-gather;
+  paragraphs). Each rank sends point to point exactly the frames each successor needs (a rank
+  holding fewer frames than the halo passes on what it has, and the successor takes the rest
+  from earlier ranks);
 - the GLA / delta-rule state at the rank's first token. The state after a run is an affine map
   of the state entering it, S_end = T S_start + E (GLA paragraph: the update is linear in S).
-  Every rank computes its run's E (start from zero) and T (start from the identity with v = 0),
-  the pairs are all-gathered, and each rank folds its predecessors' maps into its entering state.
+  Every rank computes its run's E (the end state from zero) and T (its transition: for the
+  vector-gated GLA the diagonal of gate products over the run, for the delta rule the end state
+  from the identity with v = 0), the pairs are all-gathered, and each rank folds its
+  predecessors' maps into its entering state.
 The rank then runs the hybrid layer on its frames with the halo in front of its K/V and the
 entering state (kta_hybrid_fwd_window).
 
@@ -74,6 +78,50 @@ class ShardCfg:
         return halo_frames(self.n_swa, self.n_dswa, self.W_swa, self.W_dswa, self.dil)
 
 
+def halo_sends(r: int, split: list[tuple[int, int]], halo: int) -> list[tuple[int, int, int]]:
+    """What rank r sends: (destination rank, first frame offset, frame count) within r's halo
+    block, the frames of r that each later rank's halo_plan takes from r."""
+    out = []
+    for r2 in range(r + 1, len(split)):
+        fs = [f for j, f in halo_plan(r2, split, halo) if j == r]
+        if fs:
+            out.append((r2, fs[0], len(fs)))
+    return out
+
+
+def halo_recvs(r: int, split: list[tuple[int, int]], halo: int) -> list[tuple[int, int, int]]:
+    """What rank r receives: (source rank, first frame offset in the source's halo block, frame
+    count), oldest source first."""
+    out: list[tuple[int, int, int]] = []
+    for j, f in halo_plan(r, split, halo):
+        if out and out[-1][0] == j:
+            out[-1] = (j, out[-1][1], out[-1][2] + 1)
+        else:
+            out.append((j, f, 1))
+    return out
+
+
+def _exchange_halo(c: "ShardCfg", r: int, R: int, blk: torch.Tensor, group) -> dict:
+    """Point-to-point halo exchange: {source rank: (first frame offset, [2, n*P, ns, d] K/V)}."""
+    split = frame_split(c.F, R)
+    P = c.P
+    ops, got = [], {}
+    for dst, f0, n in halo_sends(r, split, c.halo):
+        ops.append(dist.P2POp(dist.isend, blk[:, f0 * P:(f0 + n) * P].contiguous(),
+                              dist.get_global_rank(group, dst) if group is not None else dst,
+                              group))
+    for src, f0, n in halo_recvs(r, split, c.halo):
+        buf = torch.empty((2, n * P) + tuple(blk.shape[2:]), dtype=blk.dtype, device=blk.device)
+        got[src] = (f0, buf)
+        ops.append(dist.P2POp(dist.irecv, buf,
+                              dist.get_global_rank(group, src) if group is not None else src,
+                              group))
+    if ops:
+        for w in dist.batch_isend_irecv(ops):
+            w.wait()
+    return got
+
+
 def _all_gather(t: torch.Tensor, group) -> list[torch.Tensor]:
     R = dist.get_world_size(group)
     bufs = [torch.empty_like(t) for _ in range(R)]
@@ -84,8 +132,7 @@ def _all_gather(t: torch.Tensor, group) -> list[torch.Tensor]:
 def local_contribution(c: ShardCfg, r: int, R: int, q, k, v, alpha=None, beta=None, *, ops):
     """What rank r sends to the others: its halo block (the softmax heads' K and V of its last
     min(halo, count) frames, at the end of a block of `halo` frames) and, with GLA heads and
-    R > 1, its run's state map (E: end state from zero; T: transition, the end state from the
-    identity with v = 0)."""
+    R > 1, its run's state map (E: end state from zero; T: its transition, ops.lin_transition)."""
     first, count = frame_split(c.F, R)[r]
     P, d = c.P, c.d
     ns = c.n_swa + c.n_dswa
@@ -102,13 +149,13 @@ def local_contribution(c: ShardCfg, r: int, R: int, q, k, v, alpha=None, beta=No
     E = T = None
     if c.n_gla and R > 1:
         E = ops.lin_state(c, q, k, v, alpha, beta, None)
-        eye = torch.eye(d, dtype=torch.float32, device=q.device).expand(1, c.n_gla, d, d)
-        T = ops.lin_state(c, q, k, torch.zeros_like(v), alpha, beta, eye.contiguous())
+        T = ops.lin_transition(c, q, k, v, alpha, beta)
     return blk, E, T
 
 
-def finish(c: ShardCfg, r: int, R: int, q, k, v, alpha, beta, blocks, Es, Ts, *, ops, S0=None):
-    """Rank r's outputs from every rank's contribution: the halo in front of its K/V, the
+def finish(c: ShardCfg, r: int, R: int, q, k, v, alpha, beta, halo_in, Es, Ts, *, ops, S0=None):
+    """Rank r's outputs from what it received: the halo in front of its K/V (halo_in: {source
+    rank: (first frame offset within the source's halo block, its K/V [2, n*P, ns, d])}), the
     entering GLA state folded from its predecessors' maps, then the windowed hybrid layer."""
     split = frame_split(c.F, R)
     first, count = split[r]
@@ -121,8 +168,9 @@ def finish(c: ShardCfg, r: int, R: int, q, k, v, alpha, beta, blocks, Es, Ts, *,
         k_ext = torch.zeros((1, (hk + count) * P, H, d), dtype=k.dtype, device=k.device)
         v_ext = torch.zeros_like(k_ext)
         for i, (j, f) in enumerate(plan):
-            k_ext[0, i * P:(i + 1) * P, :ns] = blocks[j][0, f * P:(f + 1) * P]
-            v_ext[0, i * P:(i + 1) * P, :ns] = blocks[j][1, f * P:(f + 1) * P]
+            f0, blk = halo_in[j]
+            k_ext[0, i * P:(i + 1) * P, :ns] = blk[0, (f - f0) * P:(f - f0 + 1) * P]
+            v_ext[0, i * P:(i + 1) * P, :ns] = blk[1, (f - f0) * P:(f - f0 + 1) * P]
         k_ext[0, hk * P:] = k[0]
         v_ext[0, hk * P:] = v[0]
     S_in = S0
@@ -140,15 +188,15 @@ def sharded_hybrid_fwd(c: ShardCfg, q, k, v, alpha=None, beta=None, *, ops, grou
     q, k, v: [1, count*P, H, d]; alpha / beta: this rank's gates (vector GLA
     [1, count*P, n_gla, d], delta [1, count*P, n_gla]); S0: the sequence's initial GLA state
     [1, n_gla, d, d] (None = zero). Every rank calls this with the same ShardCfg; ranks take
-    frames by frame_split(F, world size). The exchange is one all-gather of the halo blocks and
-    two of the state maps."""
+    frames by frame_split(F, world size). The exchange is point-to-point sends of halo frames to
+    the ranks that need them and two all-gathers of the (small) state maps."""
     R = dist.get_world_size(group)
     r = dist.get_rank(group)
     blk, E, T = local_contribution(c, r, R, q, k, v, alpha, beta, ops=ops)
-    blocks = _all_gather(blk, group) if blk is not None else None
+    halo_in = _exchange_halo(c, r, R, blk, group) if blk is not None else {}
     Es = _all_gather(E, group) if E is not None else None
     Ts = _all_gather(T, group) if T is not None else None
-    return finish(c, r, R, q, k, v, alpha, beta, blocks, Es, Ts, ops=ops, S0=S0)
+    return finish(c, r, R, q, k, v, alpha, beta, halo_in, Es, Ts, ops=ops, S0=S0)
 
 
 def emulate_ranks(c: ShardCfg, R: int, q, k, v, alpha=None, beta=None, *, ops, S0=None):
@@ -160,10 +208,15 @@ def emulate_ranks(c: ShardCfg, R: int, q, k, v, alpha=None, beta=None, *, ops, S
     loc = [tuple(None if t is None else t[:, s_].contiguous() for t in (q, k, v, alpha, beta))
            for s_ in sl]
     contrib = [local_contribution(c, r, R, *loc[r], ops=ops) for r in range(R)]
-    blocks = [x[0] for x in contrib]
     Es = [x[1] for x in contrib]
     Ts = [x[2] for x in contrib]
-    outs = [finish(c, r, R, *loc[r], blocks, Es, Ts, ops=ops, S0=S0) for r in range(R)]
+    outs = []
+    for r in range(R):
+        halo_in = {}
+        if contrib[r][0] is not None:
+            for src, f0, n in halo_recvs(r, split, c.halo):
+                halo_in[src] = (f0, contrib[src][0][:, f0 * P:(f0 + n) * P])
+        outs.append(finish(c, r, R, *loc[r], halo_in, Es, Ts, ops=ops, S0=S0))
     return torch.cat(outs, 1)
 
 
@@ -192,6 +245,16 @@ class KtaOps:
             _, S = self.kta.gla_chunk_fwd(q, k, v, alpha, chunk=c.chunk, scale=c.scale_gla, S0=S0,
                                           return_state=True, heads=heads, out=scratch)
         return S
+
+    def lin_transition(self, c: ShardCfg, q, k, v, alpha, beta):
+        """T of the run: the diagonal of gate products for vector GLA (one pass over the gates);
+        for the delta rule, whose transition is dense, the end state from the identity with
+        v = 0."""
+        if not c.gla_delta:
+            return self.kta.gla_transition(alpha)
+        d = c.d
+        eye = torch.eye(d, dtype=torch.float32, device=q.device).expand(1, c.n_gla, d, d)
+        return self.lin_state(c, q, k, torch.zeros_like(v), alpha, beta, eye.contiguous())
 
     def state_affine(self, A, X, E):
         return self.kta.state_affine(A, X, E)

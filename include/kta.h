@@ -310,6 +310,18 @@ kta_status kta_hybrid_fwd_window(const kta_hybrid_cfg* cfg, int f0, const void* 
                                  const float* S0, float* S_out, void* o, void* stream);
 
 /*
+ * T = diag(prod_t alpha_t) for each sequence and head: the transition of a vector-gated GLA run
+ * (paper-read, section 2, second pillar, GLA paragraph: S_t = diag(alpha_t) S_{t-1} + k_t^T v_t,
+ * so the state after the run is T S_start + S_loc). alpha: [B][N][H][d] fp32 gates of the run
+ * (their own tensor, heads contiguous); T: [B][H][d][d] fp32, the full matrix, zeros off the
+ * diagonal, ready for kta_state_affine. The product is formed as 2^(sum of log2 alpha) with
+ * log2 clamped at -200 (a zero gate gives 0); N = 0 gives the identity. d in {32, 64, 128};
+ * pointers 16-byte aligned. The caller owns both buffers.
+ */
+kta_status kta_gla_transition(const float* alpha, float* T, int B, int N, int H, int d,
+                              void* stream);
+
+/*
  * Y_m = A_m X_m + E_m for n row-major d x d fp32 matrices (E may be NULL): composes the affine
  * state maps of consecutive token runs. The GLA and delta-rule state after a run is
  * T S_start + S_loc, where S_loc is the run's end state from a zero start and T its transition

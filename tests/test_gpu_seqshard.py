@@ -107,3 +107,28 @@ def test_ranks_with_one_frame_and_fp32(kta):
     got = o.float().cpu().numpy()
     for h in range(w.H):
         assert rel(got[:, :, h], ref[:, :, h]) <= 1e-4, f"head {h}"
+
+
+@pytest.mark.parametrize("d,N", [(128, 3000), (64, 777), (32, 1)])
+def test_gla_transition_equals_state_map_from_identity(kta, d, N):
+    """kta_gla_transition (the diagonal of gate products) equals the oracle's transition of the
+    run: its end state from the identity with v = 0; exact zeros in the gates give 0."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(11)
+    B, H = 2, 3
+    a = rng.uniform(0.97, 0.9999, size=(B, N, H, d)).astype(np.float32)
+    a[0, N // 2, 1, :5] = 0.0
+    q = np.zeros((B, N, H, d), dtype=np.float32)
+    eye = np.broadcast_to(np.eye(d), (B, H, d, d)).copy()
+    _, Tref = oracle.gla(q, q, q, a, S0=eye)
+    T = kta.gla_transition(torch.from_numpy(a).cuda())
+    torch.cuda.synchronize()
+    kta.device_status()
+    got = T.double().cpu().numpy()
+    assert np.all(got[0, 1, np.arange(5), np.arange(5)] == 0.0)
+    off = ~np.eye(d, dtype=bool)
+    assert np.all(got[..., off] == 0.0)
+    err = np.abs(got - Tref).max() / np.abs(Tref).max()
+    assert err < 1e-4, err

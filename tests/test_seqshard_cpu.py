@@ -38,6 +38,23 @@ def test_frame_split_and_halo_plan():
                     assert glob == list(range(split[r][0] - len(plan), split[r][0]))
 
 
+def test_halo_sends_match_receives():
+    """Every frame a rank receives is sent by exactly that source, with the same offset and
+    count, so the point-to-point exchange is matched on both sides."""
+    for F in (1, 5, 7, 21, 64):
+        for R in range(1, 9):
+            split = seqshard.frame_split(F, R)
+            for halo in (0, 1, 4, 9):
+                sends = {(r, dst, f0, n) for r in range(R)
+                         for dst, f0, n in seqshard.halo_sends(r, split, halo)}
+                recvs = {(src, r, f0, n) for r in range(R)
+                         for src, f0, n in seqshard.halo_recvs(r, split, halo)}
+                assert sends == recvs
+                for r in range(R):
+                    got = sum(n for _, _, n in seqshard.halo_recvs(r, split, halo))
+                    assert got == min(halo, split[r][0])
+
+
 class OracleOps:
     """CPU stand-in for the kernels: the fp64 oracle (test infrastructure)."""
 
@@ -55,6 +72,11 @@ class OracleOps:
             _, S = self.o.gla(q[:, :, hs], k[:, :, hs], v[:, :, hs], alpha, scale=c.scale_gla,
                               S0=S0n)
         return torch.from_numpy(np.ascontiguousarray(S))
+
+    def lin_transition(self, c, q, k, v, alpha, beta):
+        """The run's transition: the end state from the identity with v = 0."""
+        eye = torch.eye(c.d, dtype=torch.float64).expand(1, c.n_gla, c.d, c.d)
+        return self.lin_state(c, q, k, torch.zeros_like(v), alpha, beta, eye)
 
     def state_affine(self, A, X, E):
         return torch.from_numpy(A.double().numpy() @ X.double().numpy() + E.double().numpy())
