@@ -60,6 +60,24 @@ struct WinParams {
                     // scale * log2(e) * S over each row's visible keys (null = not written)
 };
 
+// Work item `item` (a CTA index): frames latest first (full windows first), then head, sequence,
+// tile pair.
+struct WinItem {
+  int pr, b, h, f_local;
+};
+__device__ __forceinline__ WinItem win_item(int item, const WinParams& p) {
+  WinItem w;
+  const int n_units = p.pair == 2 ? (p.n_qt + 1) >> 1 : p.n_qt;
+  w.pr = item % n_units;  // first query tile: pr * p.pair
+  item /= n_units;
+  w.b = item % p.B;
+  item /= p.B;
+  w.h = item % p.Htot;
+  item /= p.Htot;
+  w.f_local = p.Fq - 1 - item;
+  return w;
+}
+
 __device__ __forceinline__ int win_num_tiles(int f, int P, int W, int dil) {
   if (dil == 1) {
     const int g0 = max(0, f - W + 1);
@@ -126,16 +144,9 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item: frames latest first (full windows first), then head, sequence, tile pair
-  const int n_units = p.pair == 2 ? (p.n_qt + 1) >> 1 : p.n_qt;
-  int item = blockIdx.x;
-  const int pr = item % n_units;  // first query tile of this CTA: pr * p.pair
-  item /= n_units;
-  const int b = item % p.B;
-  item /= p.B;
-  const int h = item % p.Htot;
-  item /= p.Htot;
-  const int f_local = p.Fq - 1 - item;
+  // ---- work item
+  const WinItem wi = win_item(blockIdx.x, p);
+  const int pr = wi.pr, b = wi.b, h = wi.h, f_local = wi.f_local;
   const int f = f_local + p.f_base;
   const int g = h >= p.H0 ? 1 : 0;
   const int W = g ? p.W[1] : p.W[0];
@@ -244,18 +255,21 @@ __global__ void __launch_bounds__(384, 1)
         const int ks1 = (2 * i + 2) % NSLOT;
         const uint32_t ph1 = ((i + 1) >> 1) & 1;
         if (*abort_flag) { ok = false; break; }
+        // The V tile of step i and the K tile of step i+1 landed long before P: check them first,
+        // so that only the P handoff (an mbarrier wait costs ~200 cycles even when complete)
+        // separates the softmax from the next MMAs.
+        if (!mbar_wait(&sm.full[vs], ph) || (more && !mbar_wait(&sm.full[ks1], ph1))) {
+          ok = false;
+          break;
+        }
         // tile A: PV_A(i), then S_A(i+1)
-        if (!mbar_wait(&sm.bar_p[0], i & 1) || !mbar_wait(&sm.full[vs], ph)) { ok = false; break; }
+        if (!mbar_spin(&sm.bar_p[0], i & 1)) { ok = false; break; }
         tc_fence_after();
         issue_pv(0, vs, i == 0);
-        if (more) {
-          if (!mbar_wait(&sm.full[ks1], ph1)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(0, ks1);
-        }
+        if (more) issue_s(0, ks1);
         // tile B: PV_B(i), then S_B(i+1)
         if (has_b) {
-          if (!mbar_wait(&sm.bar_p[1], i & 1)) { ok = false; break; }
+          if (!mbar_spin(&sm.bar_p[1], i & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv(1, vs, i == 0);
         }
