@@ -20,6 +20,7 @@
 #include "win_attn_tc.cuh"
 #include "simt_f32.cuh"
 #include "gla_chunk.cuh"
+#include "gla_tc.cuh"
 #include "delta_chunk.cuh"
 #include "bwd_f32.cuh"
 #include "proj_gemm.cuh"
@@ -101,6 +102,26 @@ kta_status make_map_nd(CUtensorMap* m, const void* base, int rank, const cuuint6
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return KTA_OK;
+}
+
+// 3-D map (d, heads, rows) of a token-major buffer with a box of box_d x 1 x box_rows; bf16 with
+// 128-byte swizzle or fp32 without swizzle.
+kta_status make_map_box(CUtensorMap* m, const void* base, bool f32, int d, int heads, long long rows,
+                        long long ld, int box_d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const cuuint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * es, static_cast<cuuint64_t>(ld) * es};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_d), 1, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  f32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return KTA_OK;
@@ -378,19 +399,37 @@ struct LinLaunch {
 // the carry pass need (segment end states and total log2 decays; none for a single segment).
 struct GlaPlan {
   int nseg = 1, seg_len = 0, slices = 1;
+  bool tc = false;  // the tcgen05 kernel (d = 128, 64-token chunks)
   size_t ws_bytes = 0;
 };
+
+// SMs of the current device (148 on B200).
+int sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!n[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1)
+      v = 148;
+    n[dev] = v;
+  }
+  return n[dev];
+}
 
 template <int D, int C>
 GlaPlan gla_plan(const LinLaunch& L) {
   using SM = kta::GlaSmem<D, C>;
   GlaPlan g;
-  g.slices = D / SM::BV;
+  g.tc = D == kta::GT_D && C == kta::GT_C;
+  g.slices = g.tc ? 1 : D / SM::BV;
   const long long base = static_cast<long long>(L.B) * L.H * g.slices;
   const int nchunks = (L.N + C - 1) / C;
   int nseg = 1;
   if (L.allow_segments) {
-    const long long want = (3LL * 148 + base - 1) / base;  // one wave of 3 CTAs per SM
+    // one wave: one CTA per SM (tcgen05 kernel) or three (warp-level kernel)
+    const long long slots = g.tc ? sm_count() : 3LL * sm_count();
+    const long long want = g.tc ? slots / base : (slots + base - 1) / base;
     nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
   }
   const int seg_chunks = (nchunks + nseg - 1) / nseg;
@@ -400,11 +439,70 @@ GlaPlan gla_plan(const LinLaunch& L) {
   return g;
 }
 
+// The tcgen05 GLA kernels (d = 128, 64-token chunks): state pass, carry, output pass.
+kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStream_t st) {
+  constexpr int D = kta::GT_D;
+  if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
+  CUtensorMap tq, tk, tv, ta;
+  const long long rows = static_cast<long long>(L.B) * L.rows_b;
+  kta_status r;
+  if ((r = make_map_box(&tq, L.q, false, D, L.H, rows, L.ld, 64, kta::GT_C)) ||
+      (r = make_map_box(&tk, L.k, false, D, L.H, rows, L.ld, 64, kta::GT_C)) ||
+      (r = make_map_box(&tv, L.v, false, D, L.H, rows, L.ld, 64, kta::GT_C)) ||
+      (r = make_map_box(&ta, L.alpha, true, D, L.H, rows, static_cast<long long>(L.H) * D, D,
+                        kta::GT_C)))
+    return r;
+  kta::GlaTcParams p{};
+  p.N = L.N;
+  p.H = L.H;
+  p.rows_b = L.rows_b;
+  p.seg_len = g.seg_len;
+  p.nseg = g.nseg;
+  p.scale = L.scale;
+  p.o = static_cast<__nv_bfloat16*>(L.o);
+  p.ld = L.ld;
+  p.S0 = L.S0;
+  p.S_out = L.S_out;
+  if (g.nseg > 1) {
+    p.ws_S = static_cast<float*>(ws);
+    p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * g.nseg * D * D;
+  }
+  const size_t smem = sizeof(kta::GlaTcSmem) + 1024;
+  if ((r = set_smem_attr(kta::gla_tc_kernel<false>, smem)) ||
+      (r = set_smem_attr(kta::gla_tc_kernel<true>, smem)))
+    return r;
+  const dim3 grid(g.nseg, L.B * L.H);
+  if (g.nseg > 1) {
+    {
+      TraceScope ts("gla_tc_state", st);
+      kta::gla_tc_kernel<false><<<grid, 384, smem, st>>>(tq, tk, tv, ta, p);
+    }
+    KTA_CUDA(cudaGetLastError());
+    kta::GlaParams pc{};  // the carry kernel folds the same workspace layout
+    pc.S0 = L.S0;
+    pc.nseg = g.nseg;
+    pc.ws_S = p.ws_S;
+    pc.ws_L = p.ws_L;
+    {
+      TraceScope ts("gla_carry", st);
+      kta::gla_carry_kernel<D><<<dim3((D * D + 127) / 128, L.B * L.H), 128, 0, st>>>(pc);
+    }
+    KTA_CUDA(cudaGetLastError());
+  }
+  {
+    TraceScope ts("gla_tc_out", st);
+    kta::gla_tc_kernel<true><<<grid, 384, smem, st>>>(tq, tk, tv, ta, p);
+  }
+  KTA_CUDA(cudaGetLastError());
+  return KTA_OK;
+}
+
 // Launch the chunked GLA kernels of a plan with `ws` (ws_bytes of device memory, or null when
 // the plan needs none) as the segment workspace.
 template <int D, int C>
 kta_status launch_gla_planned(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStream_t st) {
   using SM = kta::GlaSmem<D, C>;
+  if (g.tc) return launch_gla_tc(L, g, ws, st);
   if (static_cast<long long>(L.B) * L.H > 65535) return fail(KTA_ERR_UNSUPPORTED, "B*H > 65535");
   kta::GlaParams p{};
   p.q = static_cast<const __nv_bfloat16*>(L.q);
@@ -1154,18 +1252,6 @@ kta_status lin_bwd_common(const void* q, const void* k, const void* v, const flo
   return launch_lin_bwd<128>(p, s.B, st);
 }
 
-int sm_count() {
-  static int n[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!n[dev]) {
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1)
-      v = 148;
-    n[dev] = v;
-  }
-  return n[dev];
-}
 
 template <int D>
 kta_status launch_win_bwd_tc(const void* q, const void* k, const void* v, const void* o,
