@@ -123,8 +123,8 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "win_attn_tc": ("win_attn_tc.cuh", "kta_ptx.cuh"),
-    "gla_chunk_state": ("gla_chunk.cuh", "mma_sync.cuh", "kta_ptx.cuh"),
-    "gla_chunk_out": ("gla_chunk.cuh", "mma_sync.cuh", "kta_ptx.cuh"),
+    "gla_tc_state": ("gla_tc.cuh", "mma_sync.cuh", "kta_ptx.cuh"),
+    "gla_tc_out": ("gla_tc.cuh", "mma_sync.cuh", "kta_ptx.cuh"),
     "delta_prep": ("delta_chunk.cuh", "mma_sync.cuh"),
     "delta_scan": ("delta_chunk.cuh", "mma_sync.cuh", "kta_ptx.cuh"),
 }
