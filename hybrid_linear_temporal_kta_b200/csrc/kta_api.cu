@@ -392,6 +392,7 @@ struct LinLaunch {
   bool delta = false;
   bool erase_decayed = false;  // delta rule: decayed erase (GatedDeltaNet form)
   bool allow_segments = true;
+  int cta_budget = 0;  // SMs the segment plan may fill (0: all of them)
 };
 
 // Segment plan of the chunked GLA kernels: enough (segment, value slice, sequence-head) CTAs for
@@ -428,7 +429,8 @@ GlaPlan gla_plan(const LinLaunch& L) {
   int nseg = 1;
   if (L.allow_segments) {
     // one wave: one CTA per SM (tcgen05 kernel) or three (warp-level kernel)
-    const long long slots = g.tc ? sm_count() : 3LL * sm_count();
+    const long long sms = L.cta_budget > 0 ? std::min(L.cta_budget, sm_count()) : sm_count();
+    const long long slots = g.tc ? sms : 3LL * sms;
     const long long want = g.tc ? slots / base : (slots + base - 1) / base;
     nseg = static_cast<int>(std::min<long long>(std::max<long long>(want, 1), nchunks));
   }
@@ -1055,19 +1057,54 @@ kta_status valid_stream(kta_stream_t st) {
   return KTA_OK;
 }
 
-// Copy heads [h0, h0+nh) of one frame ([B][P][H][d]) into ring slot `slot` ([B][RR][P][nh][d]).
-kta_status ring_put(const kta_stream_s* s, const void* src, char* ring, int h0, int nh, int RR,
-                    int slot, cudaStream_t st) {
+// One frame's keys and values into the rings: up to six row-block copies (SWA k and v into both
+// copies of their slot, DSWA k and v) in one launch, 16 bytes per thread. A copy takes heads
+// [h0, h0+nh) of a frame ([B][P][H][d]) into ring slot `slot` ([B][RR][P][nh][d]).
+struct RingCopy {
+  const char* src = nullptr;
+  char* dst = nullptr;
+  long long src_seq = 0, dst_seq = 0;  // bytes between sequences
+  int src_row = 0, dst_row = 0;        // bytes between rows
+};
+struct RingPutParams {
+  RingCopy c[6];
+  int B = 0, P = 0, chunks = 0;  // chunks: 16-byte pieces per row (nh * d * element size / 16)
+};
+
+__global__ void __launch_bounds__(256) ring_put_kernel(const RingPutParams p) {
+  const RingCopy& c = p.c[blockIdx.y];
+  const long long n = static_cast<long long>(p.B) * p.P * p.chunks;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n; i += static_cast<long long>(gridDim.x) * 256) {
+    const int ch = static_cast<int>(i % p.chunks);
+    const long long r = i / p.chunks;
+    const long long row = r % p.P, b = r / p.P;
+    const uint4 v =
+        *reinterpret_cast<const uint4*>(c.src + b * c.src_seq + row * c.src_row + ch * 16);
+    *reinterpret_cast<uint4*>(c.dst + b * c.dst_seq + row * c.dst_row + ch * 16) = v;
+  }
+}
+
+RingCopy ring_copy(const kta_stream_s* s, const void* src, char* ring, int h0, int nh, int RR,
+                   int slot) {
   const kta_shape& sh = s->cfg.s;
   const int H = s->cfg.n_swa + s->cfg.n_dswa + s->cfg.n_gla;
-  const size_t row_src = static_cast<size_t>(H) * sh.d * s->es;
-  const size_t row_dst = static_cast<size_t>(nh) * sh.d * s->es;
-  for (int b = 0; b < sh.B; ++b) {
-    const char* sp = static_cast<const char*>(src) + static_cast<size_t>(b) * sh.P * row_src +
-                     static_cast<size_t>(h0) * sh.d * s->es;
-    char* dp = ring + (static_cast<size_t>(b) * RR + slot) * sh.P * row_dst;
-    KTA_CUDA(cudaMemcpy2DAsync(dp, row_dst, sp, row_src, row_dst, sh.P, cudaMemcpyDeviceToDevice, st));
-  }
+  RingCopy c;
+  c.src_row = static_cast<int>(static_cast<size_t>(H) * sh.d * s->es);
+  c.dst_row = static_cast<int>(static_cast<size_t>(nh) * sh.d * s->es);
+  c.src = static_cast<const char*>(src) + static_cast<size_t>(h0) * sh.d * s->es;
+  c.dst = ring + static_cast<size_t>(slot) * sh.P * c.dst_row;
+  c.src_seq = static_cast<long long>(sh.P) * c.src_row;
+  c.dst_seq = static_cast<long long>(RR) * sh.P * c.dst_row;
+  return c;
+}
+
+kta_status ring_put(const RingPutParams& rp, int ncopies, cudaStream_t st) {
+  if (ncopies == 0) return KTA_OK;
+  const long long per = static_cast<long long>(rp.B) * rp.P * rp.chunks;
+  const unsigned gx = static_cast<unsigned>(std::max<long long>(1, std::min<long long>((per + 255) / 256, 2 * sm_count())));
+  TraceScope ts("ring_put", st);
+  ring_put_kernel<<<dim3(gx, static_cast<unsigned>(ncopies)), 256, 0, st>>>(rp);
+  KTA_CUDA(cudaGetLastError());
   return KTA_OK;
 }
 
@@ -1503,22 +1540,34 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
   char* swa_v = s->arena + s->off_swa_v;
   char* dswa_k = s->arena + s->off_dswa_k;
   char* dswa_v = s->arena + s->off_dswa_v;
-  // 1. append this frame's keys and values to the rings
-  if (c.n_swa) {
-    const int slot = f % s->R_swa;
-    if ((r = ring_put(s, k_f, swa_k, 0, c.n_swa, 2 * s->R_swa, slot, st)) ||
-        (r = ring_put(s, k_f, swa_k, 0, c.n_swa, 2 * s->R_swa, slot + s->R_swa, st)) ||
-        (r = ring_put(s, v_f, swa_v, 0, c.n_swa, 2 * s->R_swa, slot, st)) ||
-        (r = ring_put(s, v_f, swa_v, 0, c.n_swa, 2 * s->R_swa, slot + s->R_swa, st)))
-      return r;
-  }
-  if (c.n_dswa) {
-    const int slot = f % s->R_dswa;
-    if ((r = ring_put(s, k_f, dswa_k, c.n_swa, c.n_dswa, s->R_dswa, slot, st)) ||
-        (r = ring_put(s, v_f, dswa_v, c.n_swa, c.n_dswa, s->R_dswa, slot, st)))
-      return r;
+  // 1. append this frame's keys and values to the rings (one gather launch; every ring row holds
+  // a whole number of 16-byte pieces since d is 64 or 128)
+  {
+    RingPutParams rp;
+    rp.B = sh.B;
+    rp.P = sh.P;
+    int nc = 0;
+    if (c.n_swa) {
+      const int slot = f % s->R_swa, RR = 2 * s->R_swa;
+      rp.c[nc++] = ring_copy(s, k_f, swa_k, 0, c.n_swa, RR, slot);
+      rp.c[nc++] = ring_copy(s, k_f, swa_k, 0, c.n_swa, RR, slot + s->R_swa);
+      rp.c[nc++] = ring_copy(s, v_f, swa_v, 0, c.n_swa, RR, slot);
+      rp.c[nc++] = ring_copy(s, v_f, swa_v, 0, c.n_swa, RR, slot + s->R_swa);
+      rp.chunks = static_cast<int>(static_cast<size_t>(c.n_swa) * sh.d * s->es / 16);
+      if ((r = ring_put(rp, nc, st))) return r;
+      nc = 0;
+    }
+    if (c.n_dswa) {
+      const int slot = f % s->R_dswa;
+      rp.c[nc++] = ring_copy(s, k_f, dswa_k, c.n_swa, c.n_dswa, s->R_dswa, slot);
+      rp.c[nc++] = ring_copy(s, v_f, dswa_v, c.n_swa, c.n_dswa, s->R_dswa, slot);
+      rp.chunks = static_cast<int>(static_cast<size_t>(c.n_dswa) * sh.d * s->es / 16);
+      if ((r = ring_put(rp, nc, st))) return r;
+    }
   }
   // 2. softmax heads: queries of this frame against the rings
+  ThreadStreams* ts = nullptr;
+  int gla_budget = 0;
   if (c.n_swa + c.n_dswa > 0) {
     WinLaunch L;
     L.B = sh.B;
@@ -1562,6 +1611,17 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
       g.kb_frames = s->R_dswa;
       g.kmod = s->R_dswa;
     }
+    if (c.n_gla) {
+      // The GLA heads run beside the softmax heads on the thread's side stream, planned for the
+      // SMs that the softmax launch leaves free (its last wave's remainder).
+      const long long units = static_cast<long long>(c.n_swa + c.n_dswa) * sh.B;
+      const long long n_qt = (sh.P + 127) / 128;
+      const long long nblk = units * (units * ((n_qt + 1) / 2) >= 2 * 148 ? (n_qt + 1) / 2 : n_qt);
+      const long long sm = sm_count(), rem = nblk % sm;
+      gla_budget = static_cast<int>(nblk < sm ? sm - nblk : (rem ? sm - rem : sm));
+      if ((r = thread_streams(&ts))) return r;
+      KTA_CUDA(cudaEventRecord(ts->fork, st));
+    }
     if ((r = launch_win(L, st))) return r;
   }
   // 3. GLA heads: this frame's tokens from the carried state (ping-pong state buffers)
@@ -1587,7 +1647,16 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
     L.scale = c.scale_gla;
     L.delta = c.gla_delta != 0;
     L.erase_decayed = c.gla_delta == 2;
-    if ((r = launch_lin(L, st))) return r;
+    L.cta_budget = gla_budget;
+    if (ts) {
+      KTA_CUDA(cudaStreamWaitEvent(ts->side, ts->fork, 0));
+      r = launch_lin(L, ts->side);
+      KTA_CUDA(cudaEventRecord(ts->join, ts->side));
+      KTA_CUDA(cudaStreamWaitEvent(st, ts->join, 0));
+      if (r) return r;
+    } else if ((r = launch_lin(L, st))) {
+      return r;
+    }
     s->cur = 1 - s->cur;
   }
   s->frame += 1;
