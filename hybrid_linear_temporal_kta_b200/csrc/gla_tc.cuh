@@ -113,6 +113,18 @@ __device__ __forceinline__ float gt_lds_f32(uint32_t a) {
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
   return v;
 }
+__device__ __forceinline__ uint4 gt_lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void gt_sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
 // All-of / any-of over the 128 gate threads (named barrier 1).
 __device__ __forceinline__ bool gt_all(bool v) {
   uint32_t r;
@@ -263,22 +275,23 @@ __global__ void __launch_bounds__(384, 1)
       const int n = min(GT_C, t_end - t_begin - c * GT_C);
       if (!gt_all(!*abort_flag && mbar_wait(&sm.full[s], (c >> 1) & 1))) { ok = false; break; }
       // cumulative log2 gate of this key dim over the chunk, written over its alpha column (the
-      // stage stays untouched by the producer until the chunk's MMAs are done); rows >= n: alpha = 1
+      // stage stays untouched by the producer until the chunk's MMAs are done); rows >= n: alpha = 1.
+      // Each log2 gate is clamped to [-200, 0], so b_t never increases with t.
       const uint32_t bcol = smem_u32(&sm.alpha[s][0][kd]);
       float acc = 0.f;
       for (int t = 0; t < GT_C; ++t) {
         const uint32_t a = bcol + t * GT_D * 4;
-        acc += fmaxf(__log2f(t < n ? gt_lds_f32(a) : 1.f), -200.f);
+        acc += fmaxf(fminf(__log2f(t < n ? gt_lds_f32(a) : 1.f), 0.f), -200.f);
         asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(acc) : "memory");
       }
       ltot += acc;
       auto bt = [&](int t) { return gt_lds_f32(bcol + t * GT_D * 4); };
-      // span plan: the whole chunk, 16-token spans, or single tokens
+      // span plan: the whole chunk, 16-token spans, or single tokens. A span [lo, hi) with middle
+      // m = lo + (hi - lo) / 2 passes when every |b_t - b_m| <= KTA_GLA_LIM; b is monotone, so the
+      // largest deviation is at one of the span's ends.
       auto dev_ok = [&](int lo, int hi) {
         const float bm = bt(lo + ((hi - lo) >> 1));
-        float dv = 0.f;
-        for (int t = lo; t < hi; ++t) dv = fmaxf(dv, fabsf(bt(t) - bm));
-        return !(dv > KTA_GLA_LIM);
+        return !(fmaxf(bt(lo) - bm, bm - bt(hi - 1)) > KTA_GLA_LIM);
       };
       int span = GT_C;
       if (!gt_all(dev_ok(0, n))) {
@@ -315,44 +328,68 @@ __global__ void __launch_bounds__(384, 1)
         sm.bmv[kd] = bm;
         asm volatile("bar.sync 2, 128;" ::: "memory");
         {
+          // thread i takes the 8 key dims of 16-byte chunk i % 16 in rows i / 16 + 8 j; the
+          // inputs of four rows are read before any of them is written, so that the reads overlap
           const int cc = kd & 15, r0t = kd >> 4;
-          const float4 bm0 = *reinterpret_cast<const float4*>(&sm.bmv[cc * 8]);
-          const float4 bm1 = *reinterpret_cast<const float4*>(&sm.bmv[cc * 8 + 4]);
-          const float bmc[8] = {bm0.x, bm0.y, bm0.z, bm0.w, bm1.x, bm1.y, bm1.z, bm1.w};
+          const uint4 bm0 = gt_lds128(smem_u32(&sm.bmv[cc * 8]));
+          const uint4 bm1 = gt_lds128(smem_u32(&sm.bmv[cc * 8 + 4]));
+          const float bmc[8] = {__uint_as_float(bm0.x), __uint_as_float(bm0.y), __uint_as_float(bm0.z),
+                                __uint_as_float(bm0.w), __uint_as_float(bm1.x), __uint_as_float(bm1.y),
+                                __uint_as_float(bm1.z), __uint_as_float(bm1.w)};
+          const uint32_t a_base = smem_u32(&sm.alpha[s][0][cc * 8]);
+          const uint32_t k_base = smem_u32(sm.k[s]), q_base = smem_u32(sm.q[s]);
+          const uint32_t ks_base = smem_u32(sm.ks), qs_base = smem_u32(sm.qs);
 #pragma unroll
-          for (int j = 0; j < GT_C / 8; ++j) {
-            const int t = r0t + 8 * j;
-            const bool in = t >= lo && t < hi;
-            if (!in && !(t >= plo && t < phi)) continue;
-            const uint32_t off = gt_sw(t, cc * 8);
-            uint4 kw = make_uint4(0, 0, 0, 0), qw = kw;
-            if (in) {
-              const float4 b0 = *reinterpret_cast<const float4*>(&sm.alpha[s][t][cc * 8]);
-              const float4 b1 = *reinterpret_cast<const float4*>(&sm.alpha[s][t][cc * 8 + 4]);
-              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-              const uint4 kr = *reinterpret_cast<const uint4*>(sm.k[s] + off);
-              const uint32_t* kp = &kr.x;
-              uint32_t* ko = &kw.x;
+          for (int j0 = 0; j0 < GT_C / 8; j0 += 4) {
+            uint4 ga[4], gb[4], kr[4], qr[4];
+            bool in[4], touch[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float d0 = bb[2 * e] - bmc[2 * e], d1 = bb[2 * e + 1] - bmc[2 * e + 1];
-                ko[e] = pack_bf16x2(__uint_as_float(kp[e] << 16) * ex2_approx(-d0),
-                                    __uint_as_float(kp[e] & 0xffff0000u) * ex2_approx(-d1));
+            for (int jj = 0; jj < 4; ++jj) {
+              const int t = r0t + 8 * (j0 + jj);
+              in[jj] = t >= lo && t < hi;
+              touch[jj] = in[jj] || (t >= plo && t < phi);
+              ga[jj] = gb[jj] = kr[jj] = qr[jj] = make_uint4(0, 0, 0, 0);
+              if (in[jj]) {
+                const uint32_t off = gt_sw(t, cc * 8);
+                ga[jj] = gt_lds128(a_base + t * GT_D * 4);
+                gb[jj] = gt_lds128(a_base + t * GT_D * 4 + 16);
+                kr[jj] = gt_lds128(k_base + off);
+                if (OUTPUT) qr[jj] = gt_lds128(q_base + off);
               }
-              if (OUTPUT) {
-                const uint4 qr = *reinterpret_cast<const uint4*>(sm.q[s] + off);
-                const uint32_t* qp = &qr.x;
-                uint32_t* qo = &qw.x;
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              if (!touch[jj]) continue;
+              const int t = r0t + 8 * (j0 + jj);
+              const uint32_t off = gt_sw(t, cc * 8);
+              uint4 kw = make_uint4(0, 0, 0, 0), qw = kw;
+              if (in[jj]) {
+                const float bb[8] = {__uint_as_float(ga[jj].x), __uint_as_float(ga[jj].y),
+                                     __uint_as_float(ga[jj].z), __uint_as_float(ga[jj].w),
+                                     __uint_as_float(gb[jj].x), __uint_as_float(gb[jj].y),
+                                     __uint_as_float(gb[jj].z), __uint_as_float(gb[jj].w)};
+                const uint32_t* kp = &kr[jj].x;
+                uint32_t* ko = &kw.x;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const float d0 = bb[2 * e] - bmc[2 * e], d1 = bb[2 * e + 1] - bmc[2 * e + 1];
-                  qo[e] = pack_bf16x2(__uint_as_float(qp[e] << 16) * ex2_approx(d0),
-                                      __uint_as_float(qp[e] & 0xffff0000u) * ex2_approx(d1));
+                  ko[e] = pack_bf16x2(__uint_as_float(kp[e] << 16) * ex2_approx(-d0),
+                                      __uint_as_float(kp[e] & 0xffff0000u) * ex2_approx(-d1));
+                }
+                if (OUTPUT) {
+                  const uint32_t* qp = &qr[jj].x;
+                  uint32_t* qo = &qw.x;
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const float d0 = bb[2 * e] - bmc[2 * e], d1 = bb[2 * e + 1] - bmc[2 * e + 1];
+                    qo[e] = pack_bf16x2(__uint_as_float(qp[e] << 16) * ex2_approx(d0),
+                                        __uint_as_float(qp[e] & 0xffff0000u) * ex2_approx(d1));
+                  }
                 }
               }
+              gt_sts128(ks_base + off, kw);
+              if (OUTPUT) gt_sts128(qs_base + off, qw);
             }
-            *reinterpret_cast<uint4*>(sm.ks + off) = kw;
-            if (OUTPUT) *reinterpret_cast<uint4*>(sm.qs + off) = qw;
           }
         }
         plo = lo;

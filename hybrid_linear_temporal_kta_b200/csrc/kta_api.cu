@@ -147,9 +147,10 @@ DeviceRes& device_res(int dev) {
   return *it->second;
 }
 
-struct ThreadStreams {  // per host thread and device: side stream + events for the hybrid fork
-  cudaStream_t side = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+struct ThreadStreams {  // per host thread and device: the two streams of the hybrid fork
+  cudaStream_t hi = nullptr;    // softmax heads: the device's highest stream priority
+  cudaStream_t side = nullptr;  // linear heads: its lowest
+  cudaEvent_t fork = nullptr, join_hi = nullptr, join = nullptr;
 };
 
 kta_status thread_streams(ThreadStreams** out) {
@@ -158,8 +159,12 @@ kta_status thread_streams(ThreadStreams** out) {
   KTA_CUDA(cudaGetDevice(&dev));
   ThreadStreams& t = m[dev];
   if (!t.side) {
-    KTA_CUDA(cudaStreamCreateWithFlags(&t.side, cudaStreamNonBlocking));
+    int least = 0, greatest = 0;
+    KTA_CUDA(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    KTA_CUDA(cudaStreamCreateWithPriority(&t.hi, cudaStreamNonBlocking, greatest));
+    KTA_CUDA(cudaStreamCreateWithPriority(&t.side, cudaStreamNonBlocking, least));
     KTA_CUDA(cudaEventCreateWithFlags(&t.fork, cudaEventDisableTiming));
+    KTA_CUDA(cudaEventCreateWithFlags(&t.join_hi, cudaEventDisableTiming));
     KTA_CUDA(cudaEventCreateWithFlags(&t.join, cudaEventDisableTiming));
   }
   *out = &t;
@@ -900,6 +905,26 @@ static kta_status check_cfg(const kta_hybrid_cfg* c) {
   return check_heads(H, H, c->s);
 }
 
+// Softmax heads and linear heads of one hybrid call, forked from `st` onto the thread's two
+// streams and joined back into it. The softmax stream has the higher priority, so the block
+// scheduler dispatches every pending softmax CTA before a linear-head CTA: the linear heads fill
+// the SMs that the softmax launch leaves free (its last wave) instead of taking SMs from it.
+kta_status run_forked(const WinLaunch& W, const LinLaunch& L, cudaStream_t st) {
+  ThreadStreams* ts = nullptr;
+  kta_status r;
+  if ((r = thread_streams(&ts))) return r;
+  KTA_CUDA(cudaEventRecord(ts->fork, st));
+  KTA_CUDA(cudaStreamWaitEvent(ts->hi, ts->fork, 0));
+  KTA_CUDA(cudaStreamWaitEvent(ts->side, ts->fork, 0));
+  const kta_status r_win = launch_win(W, ts->hi);
+  const kta_status r_lin = launch_lin(L, ts->side);
+  KTA_CUDA(cudaEventRecord(ts->join_hi, ts->hi));
+  KTA_CUDA(cudaEventRecord(ts->join, ts->side));
+  KTA_CUDA(cudaStreamWaitEvent(st, ts->join_hi, 0));
+  KTA_CUDA(cudaStreamWaitEvent(st, ts->join, 0));
+  return r_win ? r_win : r_lin;
+}
+
 static kta_status hybrid_common(const kta_hybrid_cfg* cfg, int f0, const void* q, const void* k,
                                 const void* v, const float* alpha, const float* beta,
                                 const float* S0, float* S_out, void* o, void* stream) {
@@ -957,18 +982,7 @@ static kta_status hybrid_common(const kta_hybrid_cfg* cfg, int f0, const void* q
     if ((r = launch_win(W, st))) return r;
     return launch_lin(L, st);
   }
-  // The persistent softmax kernel is launched first and takes every SM; the GLA kernels, forked
-  // onto a side stream, fill SMs as soon as softmax CTAs retire (the tail of the softmax pass).
-  ThreadStreams* ts = nullptr;
-  if ((r = thread_streams(&ts))) return r;
-  KTA_CUDA(cudaEventRecord(ts->fork, st));
-  kta_status r_win = launch_win(W, st);
-  KTA_CUDA(cudaStreamWaitEvent(ts->side, ts->fork, 0));
-  kta_status r_lin = launch_lin(L, ts->side);
-  KTA_CUDA(cudaEventRecord(ts->join, ts->side));
-  KTA_CUDA(cudaStreamWaitEvent(st, ts->join, 0));
-  if (r_win) return r_win;
-  return r_lin;
+  return run_forked(W, L, st);
 }
 
 kta_status kta_hybrid_fwd(const kta_hybrid_cfg* cfg, const void* q, const void* k, const void* v,
@@ -1566,10 +1580,10 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
     }
   }
   // 2. softmax heads: queries of this frame against the rings
-  ThreadStreams* ts = nullptr;
-  int gla_budget = 0;
-  if (c.n_swa + c.n_dswa > 0) {
-    WinLaunch L;
+  const bool has_win = c.n_swa + c.n_dswa > 0;
+  WinLaunch W;
+  if (has_win) {
+    WinLaunch& L = W;
     L.B = sh.B;
     L.P = sh.P;
     L.Fq = 1;
@@ -1611,22 +1625,11 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
       g.kb_frames = s->R_dswa;
       g.kmod = s->R_dswa;
     }
-    if (c.n_gla) {
-      // The GLA heads run beside the softmax heads on the thread's side stream, planned for the
-      // SMs that the softmax launch leaves free (its last wave's remainder).
-      const long long units = static_cast<long long>(c.n_swa + c.n_dswa) * sh.B;
-      const long long n_qt = (sh.P + 127) / 128;
-      const long long nblk = units * (units * ((n_qt + 1) / 2) >= 2 * 148 ? (n_qt + 1) / 2 : n_qt);
-      const long long sm = sm_count(), rem = nblk % sm;
-      gla_budget = static_cast<int>(nblk < sm ? sm - nblk : (rem ? sm - rem : sm));
-      if ((r = thread_streams(&ts))) return r;
-      KTA_CUDA(cudaEventRecord(ts->fork, st));
-    }
-    if ((r = launch_win(L, st))) return r;
   }
   // 3. GLA heads: this frame's tokens from the carried state (ping-pong state buffers)
+  LinLaunch G;
   if (c.n_gla) {
-    LinLaunch L;
+    LinLaunch& L = G;
     L.B = sh.B;
     L.N = sh.P;
     L.H = c.n_gla;
@@ -1647,18 +1650,23 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
     L.scale = c.scale_gla;
     L.delta = c.gla_delta != 0;
     L.erase_decayed = c.gla_delta == 2;
-    L.cta_budget = gla_budget;
-    if (ts) {
-      KTA_CUDA(cudaStreamWaitEvent(ts->side, ts->fork, 0));
-      r = launch_lin(L, ts->side);
-      KTA_CUDA(cudaEventRecord(ts->join, ts->side));
-      KTA_CUDA(cudaStreamWaitEvent(st, ts->join, 0));
-      if (r) return r;
-    } else if ((r = launch_lin(L, st))) {
-      return r;
+    if (has_win) {
+      // planned for the SMs that the softmax launch leaves free (its last wave's remainder)
+      const long long units = static_cast<long long>(c.n_swa + c.n_dswa) * sh.B;
+      const long long n_qt = (sh.P + 127) / 128;
+      const long long nblk = units * (units * ((n_qt + 1) / 2) >= 2 * 148 ? (n_qt + 1) / 2 : n_qt);
+      const long long sm = sm_count(), rem = nblk % sm;
+      L.cta_budget = static_cast<int>(nblk < sm ? sm - nblk : (rem ? sm - rem : sm));
     }
-    s->cur = 1 - s->cur;
   }
+  if (has_win && c.n_gla)
+    r = run_forked(W, G, st);
+  else if (has_win)
+    r = launch_win(W, st);
+  else if (c.n_gla)
+    r = launch_lin(G, st);
+  if (r) return r;
+  if (c.n_gla) s->cur = 1 - s->cur;
   s->frame += 1;
   return KTA_OK;
 }

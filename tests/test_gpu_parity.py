@@ -249,44 +249,6 @@ def test_bf16_delta_matches_oracle(kta, d, N, B, H, with_s0):
     assert rel(S.cpu().numpy(), Sref) < BF16_TOL
 
 
-def small_gates(kind, shape, seed):
-    """Forget gates far below the usual range (all valid: alpha in [0, 1))."""
-    rng = np.random.default_rng(seed)
-    if kind == "sigmoid(N(-3,1))":
-        a = 1.0 / (1.0 + np.exp(-(rng.standard_normal(shape) - 3.0)))
-    elif kind == "uniform[1e-4,0.1]":
-        a = rng.uniform(1e-4, 0.1, size=shape)
-    else:  # ordinary gates with exact zeros, 1e-30 and 1e-12 sprinkled in
-        a = rng.uniform(0.3, 0.999, size=shape)
-        flat = a.reshape(-1)
-        idx = rng.choice(flat.size, size=flat.size // 20, replace=False)
-        flat[idx[0::3]], flat[idx[1::3]], flat[idx[2::3]] = 0.0, 1e-30, 1e-12
-    return torch.from_numpy(a.astype(np.float32))
-
-
-@pytest.mark.parametrize("kind", ["sigmoid(N(-3,1))", "uniform[1e-4,0.1]", "zeros-and-tiny"])
-@pytest.mark.parametrize("d,chunk,N", [(128, 64, 5 * 64 + 7), (128, 32, 4 * 32 + 19),
-                                       (128, 16, 4 * 16 + 5), (64, 64, 4 * 64 + 33),
-                                       (64, 32, 6 * 32), (64, 16, 5 * 16 + 1),
-                                       (128, 64, 9000)])
-def test_bf16_gla_small_gates_match_oracle(kta, kind, d, chunk, N):
-    """Gates near 0 (the GLA paragraph's forget gate ranges over (0, 1)): every output finite and
-    within the bf16 bound of the oracle, with a start state, several chunks, a ragged tail and
-    (N = 9000) several segments joined by the carry pass."""
-    B, H = 2, 2
-    w = synth.HYBRID_BF16.replace(d=d, n_swa=0, n_dswa=0, n_gla=H, chunk=chunk)
-    x = synth.make_inputs(w, N=N, B=B)
-    alpha = small_gates(kind, (B, N, H, d), seed=7 * d + chunk)
-    S0 = torch.from_numpy(np.random.default_rng(5).standard_normal((B, H, d, d)).astype(np.float32))
-    o, S = kta.gla_chunk_fwd(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(alpha), chunk=chunk,
-                             S0=dev(S0), return_state=True)
-    kta.device_status()
-    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
-    ref, Sref = oracle.gla(x["q"], x["k"], x["v"], alpha, S0=S0)
-    assert_heads_close(o, ref, range(H), BF16_TOL, what=f"gla {kind} d={d} C={chunk} N={N}")
-    assert rel(S.cpu().numpy(), Sref) < BF16_TOL
-
-
 @pytest.mark.parametrize("d,N,B,H,with_s0", [(128, 300, 2, 2, True), (64, 1000, 1, 3, False),
                                              (128, 50, 1, 1, True), (128, 4096, 1, 1, False)])
 def test_bf16_decayed_erase_delta_matches_oracle(kta, d, N, B, H, with_s0):
