@@ -68,7 +68,10 @@ struct GlaTcParams {
   float* S_out;            // [B][H][D][D], or null
   float* ws_S;             // [B*H][nseg][D][D] segment states (pass 1 writes, carry folds)
   float* ws_L;             // [B*H][nseg][D] segment total log2 decay
+  int fold;                // 1: pass 2 folds the segment end states itself (no carry kernel ran)
 };
+
+constexpr int GT_FOLD_MAX = 3;  // most predecessor segments a pass-2 CTA folds itself
 
 struct GlaTcSmem {
   alignas(1024) uint8_t q[2][GT_TILE];     // stage ring, TMA layout (two 64-column boxes)
@@ -459,15 +462,31 @@ __global__ void __launch_bounds__(384, 1)
     const int quad = warp & 3;
     const int vd = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    // start state: S0 for a single segment, else the carry kernel's start of this segment
+    // start state: S0 for a single segment, else the carry kernel's start of this segment, or
+    // (fold) S_start(s+1) = 2^{L_s} S_start(s) + S_loc(s) over the predecessors, as the carry
+    // kernel computes it
+    const bool fold = OUTPUT && p.fold && p.nseg > 1;
+    const float* S0b = p.S0 ? p.S0 + static_cast<long long>(bh) * GT_D * GT_D : nullptr;
     const float* Ss = !OUTPUT ? nullptr
-                      : p.nseg > 1 ? p.ws_S + (static_cast<long long>(bh) * p.nseg + seg) * GT_D * GT_D
-                                   : (p.S0 ? p.S0 + static_cast<long long>(bh) * GT_D * GT_D : nullptr);
+                      : p.nseg > 1 && !fold ? p.ws_S + (static_cast<long long>(bh) * p.nseg + seg) * GT_D * GT_D
+                                            : S0b;
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) {
       uint32_t r[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) r[j] = Ss ? __float_as_uint(Ss[(c4 * 32 + j) * GT_D + vd]) : 0u;
+      if (fold) {
+        for (int sp = 0; sp < seg && sp < GT_FOLD_MAX; ++sp) {
+          const float* E = p.ws_S + (static_cast<long long>(bh) * p.nseg + sp) * GT_D * GT_D;
+          const float* Lw = p.ws_L + (static_cast<long long>(bh) * p.nseg + sp) * GT_D;
+          float e[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) e[j] = E[(c4 * 32 + j) * GT_D + vd];
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            r[j] = __float_as_uint(fmaf(exp2f(Lw[c4 * 32 + j]), __uint_as_float(r[j]), e[j]));
+        }
+      }
       tmem_st32(tS + lane_off + 32 * c4, r);
     }
     tmem_wait_st();

@@ -470,6 +470,9 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
   p.ld = L.ld;
   p.S0 = L.S0;
   p.S_out = L.S_out;
+  // A few segments: each output-pass CTA folds its predecessors' end states itself (reading at
+  // most kta::GT_FOLD_MAX of them), which saves the carry launch.
+  p.fold = g.nseg > 1 && g.nseg <= kta::GT_FOLD_MAX + 1 ? 1 : 0;
   if (g.nseg > 1) {
     p.ws_S = static_cast<float*>(ws);
     p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * g.nseg * D * D;
@@ -485,16 +488,18 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
       kta::gla_tc_kernel<false><<<grid, 384, smem, st>>>(tq, tk, tv, ta, p);
     }
     KTA_CUDA(cudaGetLastError());
-    kta::GlaParams pc{};  // the carry kernel folds the same workspace layout
-    pc.S0 = L.S0;
-    pc.nseg = g.nseg;
-    pc.ws_S = p.ws_S;
-    pc.ws_L = p.ws_L;
-    {
-      TraceScope ts("gla_carry", st);
-      kta::gla_carry_kernel<D><<<dim3((D * D + 127) / 128, L.B * L.H), 128, 0, st>>>(pc);
+    if (!p.fold) {
+      kta::GlaParams pc{};  // the carry kernel folds the same workspace layout
+      pc.S0 = L.S0;
+      pc.nseg = g.nseg;
+      pc.ws_S = p.ws_S;
+      pc.ws_L = p.ws_L;
+      {
+        TraceScope ts("gla_carry", st);
+        kta::gla_carry_kernel<D><<<dim3((D * D + 127) / 128, L.B * L.H), 128, 0, st>>>(pc);
+      }
+      KTA_CUDA(cudaGetLastError());
     }
-    KTA_CUDA(cudaGetLastError());
   }
   {
     TraceScope ts("gla_tc_out", st);
@@ -1072,29 +1077,34 @@ kta_status valid_stream(kta_stream_t st) {
 }
 
 // One frame's keys and values into the rings: up to six row-block copies (SWA k and v into both
-// copies of their slot, DSWA k and v) in one launch, 16 bytes per thread. A copy takes heads
-// [h0, h0+nh) of a frame ([B][P][H][d]) into ring slot `slot` ([B][RR][P][nh][d]).
+// copies of their slot, DSWA k and v) in one launch, 16 bytes per thread and step. A copy takes
+// heads [h0, h0+nh) of a frame ([B][P][H][d]) into ring slot `slot` ([B][RR][P][nh][d]).
 struct RingCopy {
   const char* src = nullptr;
   char* dst = nullptr;
   long long src_seq = 0, dst_seq = 0;  // bytes between sequences
   int src_row = 0, dst_row = 0;        // bytes between rows
+  int chunks = 0;                      // 16-byte pieces per row (nh * d * element size / 16)
 };
+constexpr int kRingRows = 16;  // rows per block
 struct RingPutParams {
   RingCopy c[6];
-  int B = 0, P = 0, chunks = 0;  // chunks: 16-byte pieces per row (nh * d * element size / 16)
+  int B = 0, P = 0;
 };
 
+// Block (x, y): rows [16 x, 16 x + 16) of the frame batch (row = b * P + token) for copy y; 32-bit
+// index arithmetic only.
 __global__ void __launch_bounds__(256) ring_put_kernel(const RingPutParams p) {
   const RingCopy& c = p.c[blockIdx.y];
-  const long long n = static_cast<long long>(p.B) * p.P * p.chunks;
-  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n; i += static_cast<long long>(gridDim.x) * 256) {
-    const int ch = static_cast<int>(i % p.chunks);
-    const long long r = i / p.chunks;
-    const long long row = r % p.P, b = r / p.P;
-    const uint4 v =
-        *reinterpret_cast<const uint4*>(c.src + b * c.src_seq + row * c.src_row + ch * 16);
-    *reinterpret_cast<uint4*>(c.dst + b * c.dst_seq + row * c.dst_row + ch * 16) = v;
+  const int rows = p.B * p.P;
+  const int r0 = static_cast<int>(blockIdx.x) * kRingRows;
+  const int n = min(kRingRows, rows - r0) * c.chunks;
+  for (int i = threadIdx.x; i < n; i += 256) {
+    const int rr = i / c.chunks, ch = i - rr * c.chunks;
+    const int r = r0 + rr, b = r / p.P, row = r - b * p.P;
+    const uint4 v = *reinterpret_cast<const uint4*>(c.src + b * c.src_seq +
+                                                    static_cast<long long>(row) * c.src_row + ch * 16);
+    *reinterpret_cast<uint4*>(c.dst + b * c.dst_seq + static_cast<long long>(row) * c.dst_row + ch * 16) = v;
   }
 }
 
@@ -1109,14 +1119,16 @@ RingCopy ring_copy(const kta_stream_s* s, const void* src, char* ring, int h0, i
   c.dst = ring + static_cast<size_t>(slot) * sh.P * c.dst_row;
   c.src_seq = static_cast<long long>(sh.P) * c.src_row;
   c.dst_seq = static_cast<long long>(RR) * sh.P * c.dst_row;
+  c.chunks = c.dst_row / 16;
   return c;
 }
 
 kta_status ring_put(const RingPutParams& rp, int ncopies, cudaStream_t st) {
   if (ncopies == 0) return KTA_OK;
-  const long long per = static_cast<long long>(rp.B) * rp.P * rp.chunks;
-  const unsigned gx = static_cast<unsigned>(std::max<long long>(1, std::min<long long>((per + 255) / 256, 2 * sm_count())));
+  const long long rows = static_cast<long long>(rp.B) * rp.P;
+  if (rows * 1024 > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "too many rows per frame batch");
   TraceScope ts("ring_put", st);
+  const unsigned gx = static_cast<unsigned>((rows + kRingRows - 1) / kRingRows);
   ring_put_kernel<<<dim3(gx, static_cast<unsigned>(ncopies)), 256, 0, st>>>(rp);
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
@@ -1567,17 +1579,13 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
       rp.c[nc++] = ring_copy(s, k_f, swa_k, 0, c.n_swa, RR, slot + s->R_swa);
       rp.c[nc++] = ring_copy(s, v_f, swa_v, 0, c.n_swa, RR, slot);
       rp.c[nc++] = ring_copy(s, v_f, swa_v, 0, c.n_swa, RR, slot + s->R_swa);
-      rp.chunks = static_cast<int>(static_cast<size_t>(c.n_swa) * sh.d * s->es / 16);
-      if ((r = ring_put(rp, nc, st))) return r;
-      nc = 0;
     }
     if (c.n_dswa) {
       const int slot = f % s->R_dswa;
       rp.c[nc++] = ring_copy(s, k_f, dswa_k, c.n_swa, c.n_dswa, s->R_dswa, slot);
       rp.c[nc++] = ring_copy(s, v_f, dswa_v, c.n_swa, c.n_dswa, s->R_dswa, slot);
-      rp.chunks = static_cast<int>(static_cast<size_t>(c.n_dswa) * sh.d * s->es / 16);
-      if ((r = ring_put(rp, nc, st))) return r;
     }
+    if ((r = ring_put(rp, nc, st))) return r;
   }
   // 2. softmax heads: queries of this frame against the rings
   const bool has_win = c.n_swa + c.n_dswa > 0;

@@ -115,6 +115,8 @@ struct WinSmem {
   alignas(1024) uint8_t q[2][NBOX * BOX];
   alignas(1024) uint8_t kv[NSLOT][NBOX * BOX];
   uint64_t bar_q, full[NSLOT], empty[NSLOT], bar_s[2], bar_p[2], bar_o[2], bar_fin;
+  float part_m[128], part_l[128];  // key split: row max and row sum of the second key half
+  int part_ok[4];                  // key split: the second half's warps finished
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -158,6 +160,12 @@ __global__ void __launch_bounds__(384, 1)
   const CUtensorMap* tv = g ? &tv1 : &tv0;
   const int ntiles = win_num_tiles(f, p.P, W, dil);
   const bool has_b = p.pair == 2 && 2 * pr + 1 < p.n_qt;
+  // A CTA with one query tile and at least two key tiles splits the key range instead: tile slot 0
+  // takes key tiles [0, nA), slot 1 the rest for the same query rows, and the two partial softmax
+  // results are merged before the output is written.
+  const bool split = !has_b && ntiles >= 2;
+  const int nA = split ? (ntiles + 1) / 2 : ntiles;
+  const int nB = split ? ntiles - nA : (has_b ? ntiles : 0);
   const int q_row0 = b * p.q_rows_b + f_local * p.P + pr * p.pair * 128;  // tile A; B = +128
 
   if (threadIdx.x == 0) {
@@ -185,34 +193,50 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || (warp == 2 && split)) {
+    // ------------------------------------------------------------ TMA producer(s): warp 0 loads
+    // Q and the K / V ring; with a key split, warp 0 loads the first half's K / V and warp 2 the
+    // second's, so that neither half's next tiles wait behind the other's slot releases.
     if (lane == 0) {
-      prefetch_tmap(&tq);
+      const int half = warp == 2 ? 1 : 0;
       prefetch_tmap(tk);
       prefetch_tmap(tv);
-      mbar_arrive_expect_tx(&sm.bar_q, has_b ? 2 * TILE_BYTES : TILE_BYTES);
-      for (int x = 0; x < (has_b ? 2 : 1); ++x)
-        for (int c = 0; c < NBOX; ++c)
-          tma_load_3d(sm.q[x] + c * BOX, &tq, &sm.bar_q, c * 64, h, q_row0 + 128 * x);
-      int issued = 0;
-      for (int n = 0; n < 2 * ntiles; ++n) {  // load n: K_{n/2} (n even) or V_{n/2} (n odd)
-        if (*abort_flag) break;
-        const int slot = n % NSLOT, use = n / NSLOT;
+      if (half == 0) {
+        prefetch_tmap(&tq);
+        mbar_arrive_expect_tx(&sm.bar_q, has_b ? 2 * TILE_BYTES : TILE_BYTES);
+        for (int x = 0; x < (has_b ? 2 : 1); ++x)
+          for (int c = 0; c < NBOX; ++c)
+            tma_load_3d(sm.q[x] + c * BOX, &tq, &sm.bar_q, c * 64, h, q_row0 + 128 * x);
+      }
+      int uses[NSLOT] = {0, 0, 0, 0};
+      // load (key tile kt, V or K) into `slot` as that slot's next use
+      auto load = [&](int kt, bool is_v, int slot) {
         int fr0, off, nv;
-        win_tile(n >> 1, f, p.P, W, dil, fr0, off, nv);
+        win_tile(kt, f, p.P, W, dil, fr0, off, nv);
         const int krow = (b * kbf + fr0 % kmod) * p.P + off;
-        if (use > 0 && !mbar_wait(&sm.empty[slot], (use - 1) & 1)) { *abort_flag = 1; break; }
+        const int use = uses[slot];
+        if (use > 0 && !mbar_wait(&sm.empty[slot], (use - 1) & 1)) { *abort_flag = 1; return false; }
         mbar_arrive_expect_tx(&sm.full[slot], TILE_BYTES);
-        const CUtensorMap* tm = (n & 1) ? tv : tk;
+        const CUtensorMap* tm = is_v ? tv : tk;
         for (int c = 0; c < NBOX; ++c)
           tma_load_3d(sm.kv[slot] + c * BOX, tm, &sm.full[slot], c * 64, hk, krow);
-        ++issued;
+        uses[slot] = use + 1;
+        return true;
+      };
+      if (!split) {
+        // load n: K_{n/2} (n even) or V_{n/2} (n odd), slot n % NSLOT
+        for (int n = 0; n < 2 * ntiles; ++n)
+          if (*abort_flag || !load(n >> 1, n & 1, n % NSLOT)) break;
+      } else {
+        // this half's step i: K into slot `half`, V into slot 2 + `half`
+        const int nh = half ? nB : nA, kt0 = half ? nA : 0;
+        for (int i = 0; i < nh; ++i)
+          if (*abort_flag || !load(kt0 + i, false, half) || !load(kt0 + i, true, 2 + half)) break;
       }
       // Let the copies this thread started land before the CTA can exit (bounded waits).
-      mbar_wait(&sm.bar_q, 0);
-      for (int n = issued - NSLOT > 0 ? issued - NSLOT : 0; n < issued; ++n)
-        mbar_wait(&sm.full[n % NSLOT], (n / NSLOT) & 1);
+      if (half == 0) mbar_wait(&sm.bar_q, 0);
+      for (int sl = 0; sl < NSLOT; ++sl)
+        if (uses[sl] > 0) mbar_wait(&sm.full[sl], (uses[sl] - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -223,10 +247,11 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t q_base[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
       auto issue_s = [&](int x, int slot) {
         const uint32_t k_base = smem_u32(sm.kv[slot]);
+        const uint32_t qx = split ? q_base[0] : q_base[x];
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
-          mma_ss(tbase + 128 * x, smem_desc_sw128(q_base[x] + off, 16, 1024),
+          mma_ss(tbase + 128 * x, smem_desc_sw128(qx + off, 16, 1024),
                  smem_desc_sw128(k_base + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
         }
         mma_commit(&sm.bar_s[x]);
@@ -241,42 +266,81 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(&sm.bar_o[x]);
       };
       bool ok = mbar_wait(&sm.bar_q, 0) && ntiles > 0;
-      if (ok && !mbar_wait(&sm.full[0], 0)) ok = false;
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        if (has_b) issue_s(1, 0);
-        mma_commit(&sm.empty[0]);
-      }
-      for (int i = 0; ok && i < ntiles; ++i) {
-        const int vs = (2 * i + 1) % NSLOT;
-        const uint32_t ph = (i >> 1) & 1;  // phase of both slots of tile i
-        const bool more = i + 1 < ntiles;
-        const int ks1 = (2 * i + 2) % NSLOT;
-        const uint32_t ph1 = ((i + 1) >> 1) & 1;
-        if (*abort_flag) { ok = false; break; }
-        // The V tile of step i and the K tile of step i+1 landed long before P: check them first,
-        // so that only the P handoff (an mbarrier wait costs ~200 cycles even when complete)
-        // separates the softmax from the next MMAs.
-        if (!mbar_wait(&sm.full[vs], ph) || (more && !mbar_wait(&sm.full[ks1], ph1))) {
-          ok = false;
-          break;
-        }
-        // tile A: PV_A(i), then S_A(i+1)
-        if (!mbar_spin(&sm.bar_p[0], i & 1)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(0, vs, i == 0);
-        if (more) issue_s(0, ks1);
-        // tile B: PV_B(i), then S_B(i+1)
-        if (has_b) {
-          if (!mbar_spin(&sm.bar_p[1], i & 1)) { ok = false; break; }
+      if (!split) {
+        if (ok && !mbar_wait(&sm.full[0], 0)) ok = false;
+        if (ok) {
           tc_fence_after();
-          issue_pv(1, vs, i == 0);
+          issue_s(0, 0);
+          if (has_b) issue_s(1, 0);
+          mma_commit(&sm.empty[0]);
         }
-        mma_commit(&sm.empty[vs]);
-        if (more) {
-          if (has_b) issue_s(1, ks1);
-          mma_commit(&sm.empty[ks1]);
+        for (int i = 0; ok && i < ntiles; ++i) {
+          const int vs = (2 * i + 1) % NSLOT;
+          const uint32_t ph = (i >> 1) & 1;  // phase of both slots of tile i
+          const bool more = i + 1 < ntiles;
+          const int ks1 = (2 * i + 2) % NSLOT;
+          const uint32_t ph1 = ((i + 1) >> 1) & 1;
+          if (*abort_flag) { ok = false; break; }
+          // The V tile of step i and the K tile of step i+1 landed long before P: check them first,
+          // so that only the P handoff (an mbarrier wait costs ~200 cycles even when complete)
+          // separates the softmax from the next MMAs.
+          if (!mbar_wait(&sm.full[vs], ph) || (more && !mbar_wait(&sm.full[ks1], ph1))) {
+            ok = false;
+            break;
+          }
+          // tile A: PV_A(i), then S_A(i+1)
+          if (!mbar_spin(&sm.bar_p[0], i & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, vs, i == 0);
+          if (more) issue_s(0, ks1);
+          // tile B: PV_B(i), then S_B(i+1)
+          if (has_b) {
+            if (!mbar_spin(&sm.bar_p[1], i & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(1, vs, i == 0);
+          }
+          mma_commit(&sm.empty[vs]);
+          if (more) {
+            if (has_b) issue_s(1, ks1);
+            mma_commit(&sm.empty[ks1]);
+          }
+        }
+      } else {
+        // key split; slots: 0 = K of the first half, 1 = K of the second, 2 / 3 = their V
+        if (ok && !(mbar_wait(&sm.full[0], 0) && mbar_wait(&sm.full[1], 0))) ok = false;
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          mma_commit(&sm.empty[0]);
+          issue_s(1, 1);
+          mma_commit(&sm.empty[1]);
+        }
+        for (int i = 0; ok && i < nA; ++i) {
+          const uint32_t ph = i & 1, ph1 = (i + 1) & 1;
+          const bool act_b = i < nB, more_a = i + 1 < nA, more_b = i + 1 < nB;
+          if (*abort_flag) { ok = false; break; }
+          // each operand is checked right before its own MMAs: the halves' loads run
+          // independently, and a late K of one half must not hold back the other's PV
+          if (!mbar_wait(&sm.full[2], ph) || !mbar_spin(&sm.bar_p[0], ph)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, 2, i == 0);
+          mma_commit(&sm.empty[2]);
+          if (more_a) {
+            if (!mbar_wait(&sm.full[0], ph1)) { ok = false; break; }
+            issue_s(0, 0);
+            mma_commit(&sm.empty[0]);
+          }
+          if (act_b) {
+            if (!mbar_wait(&sm.full[3], ph) || !mbar_spin(&sm.bar_p[1], ph)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(1, 3, i == 0);
+            mma_commit(&sm.empty[3]);
+            if (more_b) {
+              if (!mbar_wait(&sm.full[1], ph1)) { ok = false; break; }
+              issue_s(1, 1);
+              mma_commit(&sm.empty[1]);
+            }
+          }
         }
       }
       if (!ok) *abort_flag = 1;
@@ -289,16 +353,19 @@ __global__ void __launch_bounds__(384, 1)
     const int x = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int nq = min(128, p.P - (p.pair * pr + x) * 128);  // rows of this tile in the frame
+    const int xq = split ? 0 : x;                              // query tile of this slot
+    const int nq = min(128, p.P - (p.pair * pr + xq) * 128);  // rows of this tile in the frame
+    const int n_x = x ? nB : nA;                               // key tiles of this slot
+    const int kt0 = split && x ? nA : 0;                       // its first key tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = sm.tmem_base + 128 * x;
     const uint32_t tO = sm.tmem_base + 256 + 128 * x;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    bool ok = x == 0 || has_b;
-    for (int i = 0; ok && i < ntiles; ++i) {
+    bool ok = n_x > 0;
+    for (int i = 0; ok && i < n_x; ++i) {
       int fr0, off, nv;
-      win_tile(i, f, p.P, W, dil, fr0, off, nv);
+      win_tile(kt0 + i, f, p.P, W, dil, fr0, off, nv);
       const bool got = !*abort_flag && mbar_wait(&sm.bar_s[x], i & 1);
       if (!__all_sync(0xffffffffu, got)) { *abort_flag = 1; ok = false; break; }
       tc_fence_after();
@@ -409,16 +476,42 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar_p[x]);
     }
-    // epilogue: O / l -> bf16 -> global (rows of this frame only)
-    const bool active = x == 0 || has_b;
+    // epilogue: O / l -> bf16 -> global (rows of this frame only). With a key split the second
+    // half hands its row max and row sum over through shared memory; its O stays in TMEM, where
+    // the first half's thread of the same row (same TMEM lane quarter) reads it and merges.
+    const bool active = x == 0 || has_b || split;
     if (active) {
-      const bool fin = ok && ntiles > 0 && mbar_wait(&sm.bar_o[x], (ntiles - 1) & 1);
-      if (__all_sync(0xffffffffu, fin)) {
+      bool fin = ok && n_x > 0 && mbar_wait(&sm.bar_o[x], (n_x - 1) & 1);
+      fin = __all_sync(0xffffffffu, fin);
+      float mb = -INFINITY, lb = 0.f;
+      if (split) {
+        if (x == 1) {
+          sm.part_m[row] = m;
+          sm.part_l[row] = l;
+          if (lane == 0) sm.part_ok[quad] = fin ? 1 : 0;
+        }
+        tc_fence_before();
+        asm volatile("bar.sync 3, 256;" ::: "memory");
+        if (x == 0) {
+          fin = fin && sm.part_ok[quad] != 0;
+          mb = sm.part_m[row];
+          lb = sm.part_l[row];
+        }
+      }
+      if (!fin) {
+        *abort_flag = 1;
+      } else if (!split || x == 0) {
         tc_fence_after();
-        const float inv = 1.0f / l;
+        // merge factors of the two halves (fa = 1, fb = 0 without a split)
+        const float mm = split ? fmaxf(m, mb) : m;
+        const float fa = split ? ex2_approx(m - mm) : 1.f;
+        const float fb = split ? ex2_approx(mb - mm) : 0.f;
+        const float lt = split ? fa * l + fb * lb : l;
+        const float inv = 1.0f / lt;
+        const float ia = fa * inv, ib = fb * inv;
         if (LSE && row < nq)
           p.lse[(static_cast<long long>(b) * p.Htot + h) * p.q_rows_b + f_local * p.P +
-                (p.pair * pr + x) * 128 + row] = m + __log2f(l);
+                (p.pair * pr + x) * 128 + row] = mm + __log2f(lt);
         __nv_bfloat16* orow =
             p.o + static_cast<long long>(q_row0 + 128 * x + row) * p.o_ld + h * D;
 #pragma unroll
@@ -427,18 +520,28 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld32(tO + lane_off + 32 * c, rr);
           tmem_wait_ld();
           tmem_ld_fence(rr);
+          if (split) {
+            uint32_t rb[32];
+            tmem_ld32(tO + 128 + lane_off + 32 * c, rb);
+            tmem_wait_ld();
+            tmem_ld_fence(rb);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              rr[j] = __float_as_uint(__uint_as_float(rr[j]) * ia + __uint_as_float(rb[j]) * ib);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * inv);
+          }
           if (row < nq) {
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * inv, __uint_as_float(rr[2 * j + 1]) * inv);
+              w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]), __uint_as_float(rr[2 * j + 1]));
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
             for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
           }
         }
-      } else {
-        *abort_flag = 1;
       }
     }
     tc_fence_before();

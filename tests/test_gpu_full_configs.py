@@ -87,8 +87,16 @@ def test_stream_rollout_full_size(kta):
     assert st.frame == w.F
     st.close()
     ns = w.n_swa + w.n_dswa
-    # softmax heads: identical key tiles in the same order -> bit-identical
-    assert torch.equal(roll[:, :, :ns], full[:, :, :ns])
+    # softmax heads: a one-frame launch splits each query tile's key range over the CTA's two
+    # accumulators, the full pass pairs query tiles instead, so the two agree to bf16 rounding;
+    # the last (ragged) tile of every frame is split in both, so its rows are bit-identical
+    for h in range(ns):
+        e = rel(roll[:, :, h].float().cpu().numpy(), full[:, :, h].float().cpu().numpy())
+        assert e <= BF16_TOL, f"stream vs full, softmax head {h}: {e:.3e}"
+    last = (P - 1) // 128 * 128
+    r_roll = roll[:, :, :ns].reshape(roll.shape[0], w.F, P, ns, -1)[:, :, last:]
+    r_full = full[:, :, :ns].reshape(full.shape[0], w.F, P, ns, -1)[:, :, last:]
+    assert torch.equal(r_roll, r_full)
     for h in range(ns, w.H):
         e = rel(roll[:, :, h].float().cpu().numpy(), full[:, :, h].float().cpu().numpy())
         assert e <= BF16_TOL, f"stream vs full, head {h}: {e:.3e}"

@@ -182,7 +182,10 @@ def test_bf16_dswa_equals_swa_on_page_reshape(kta):
 
 @pytest.mark.parametrize("d,chunk,N,B,H", [(128, 64, 1000, 2, 2), (128, 32, 777, 1, 3),
                                            (64, 16, 333, 2, 1), (128, 64, 20000, 1, 1),
-                                           (64, 64, 64, 1, 2)])
+                                           (64, 64, 64, 1, 2),
+                                           # 40 sequence-heads: three segments, folded by the
+                                           # output pass itself (no carry launch)
+                                           (128, 64, 700, 2, 20)])
 def test_bf16_gla_matches_oracle(kta, d, chunk, N, B, H):
     w = synth.HYBRID_BF16.replace(d=d, n_swa=0, n_dswa=0, n_gla=H, chunk=chunk)
     x = synth.make_inputs(w, N=N, B=B)
