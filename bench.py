@@ -460,6 +460,9 @@ def run_kta(args):
     achieved = flops / t_launch / 1e12
     peak = float(peaks["bf16_tflops"])
     traffic = recorded_traffic("win_attn_tc")
+    # DRAM bytes of one GLA call (state pass + output pass) from the committed ncu summary
+    gla_parts = [recorded_traffic(k) for k in ("gla_tc_state", "gla_tc_out")]
+    gla_traffic = sum(gla_parts) if all(x is not None for x in gla_parts) else None
     t_gla = sum(v["ms"] for v in kern_gla.values()) / args.steps / 1e3
     launches = sum(v["launches"] for v in kern.values()) // args.steps * args.steps
 
@@ -486,7 +489,8 @@ def run_kta(args):
                          "ms_per_call": t_gla * 1e3,
                          "bound": "hbm", "achieved": gla_bytes(w) / t_gla / 1e9 if t_gla > 0 else None,
                          "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                         "frac": gla_bytes(w) / t_gla / 1e9 / float(peaks["hbm_gbs"]) if t_gla > 0 else None},
+                         "frac": gla_bytes(w) / t_gla / 1e9 / float(peaks["hbm_gbs"]) if t_gla > 0 else None,
+                         "algorithmic_bytes": gla_bytes(w), "traffic": gla_traffic},
         "e2e": {"value": whole_job_rate(ws, w.B * w.N, args.steps, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,

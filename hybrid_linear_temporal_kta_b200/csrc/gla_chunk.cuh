@@ -58,6 +58,7 @@ struct GlaParams {
   float* S_out;            // [B][H][D][D], or null
   float* ws_S;             // [B*H][nseg][D][D] segment end states (pass 1)
   float* ws_L;             // [B*H][nseg][D] segment total log2 decay (pass 1)
+  float* S_fold;           // carry kernel: also write the state after the last segment here
 };
 
 template <int D, int C>
@@ -383,6 +384,7 @@ __global__ void __launch_bounds__(128) gla_carry_kernel(const GlaParams p) {
       }
     }
   }
+  if (p.S_fold) p.S_fold[static_cast<long long>(bh) * D * D + e] = cur;
 }
 
 }  // namespace kta

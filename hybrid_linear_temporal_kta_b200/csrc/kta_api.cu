@@ -398,6 +398,7 @@ struct LinLaunch {
   bool erase_decayed = false;  // delta rule: decayed erase (GatedDeltaNet form)
   bool allow_segments = true;
   int cta_budget = 0;  // SMs the segment plan may fill (0: all of them)
+  bool state_only = false;  // GLA: the end state only (state pass + carry fold, no outputs)
 };
 
 // Segment plan of the chunked GLA kernels: enough (segment, value slice, sequence-head) CTAs for
@@ -442,7 +443,9 @@ GlaPlan gla_plan(const LinLaunch& L) {
   const int seg_chunks = (nchunks + nseg - 1) / nseg;
   g.seg_len = seg_chunks * C;
   g.nseg = (L.N + g.seg_len - 1) / g.seg_len;
-  g.ws_bytes = g.nseg > 1 ? static_cast<size_t>(L.B) * L.H * g.nseg * (size_t(D) * D + D) * 4 : 0;
+  g.ws_bytes = g.nseg > 1 || L.state_only
+                   ? static_cast<size_t>(L.B) * L.H * g.nseg * (size_t(D) * D + D) * 4
+                   : 0;
   return g;
 }
 
@@ -453,7 +456,7 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
   CUtensorMap tq, tk, tv, ta;
   const long long rows = static_cast<long long>(L.B) * L.rows_b;
   kta_status r;
-  if ((r = make_map_box(&tq, L.q, false, D, L.H, rows, L.ld, 64, kta::GT_C)) ||
+  if ((r = make_map_box(&tq, L.q ? L.q : L.k, false, D, L.H, rows, L.ld, 64, kta::GT_C)) ||
       (r = make_map_box(&tk, L.k, false, D, L.H, rows, L.ld, 64, kta::GT_C)) ||
       (r = make_map_box(&tv, L.v, false, D, L.H, rows, L.ld, 64, kta::GT_C)) ||
       (r = make_map_box(&ta, L.alpha, true, D, L.H, rows, static_cast<long long>(L.H) * D, D,
@@ -472,8 +475,8 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
   p.S_out = L.S_out;
   // A few segments: each output-pass CTA folds its predecessors' end states itself (reading at
   // most kta::GT_FOLD_MAX of them), which saves the carry launch.
-  p.fold = g.nseg > 1 && g.nseg <= kta::GT_FOLD_MAX + 1 ? 1 : 0;
-  if (g.nseg > 1) {
+  p.fold = g.nseg > 1 && g.nseg <= kta::GT_FOLD_MAX + 1 && !L.state_only ? 1 : 0;
+  if (g.nseg > 1 || L.state_only) {
     p.ws_S = static_cast<float*>(ws);
     p.ws_L = p.ws_S + static_cast<size_t>(L.B) * L.H * g.nseg * D * D;
   }
@@ -482,7 +485,7 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
       (r = set_smem_attr(kta::gla_tc_kernel<true>, smem)))
     return r;
   const dim3 grid(g.nseg, L.B * L.H);
-  if (g.nseg > 1) {
+  if (g.nseg > 1 || L.state_only) {
     {
       TraceScope ts("gla_tc_state", st);
       kta::gla_tc_kernel<false><<<grid, 384, smem, st>>>(tq, tk, tv, ta, p);
@@ -494,6 +497,7 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
       pc.nseg = g.nseg;
       pc.ws_S = p.ws_S;
       pc.ws_L = p.ws_L;
+      pc.S_fold = L.state_only ? L.S_out : nullptr;
       {
         TraceScope ts("gla_carry", st);
         kta::gla_carry_kernel<D><<<dim3((D * D + 127) / 128, L.B * L.H), 128, 0, st>>>(pc);
@@ -501,6 +505,7 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
       KTA_CUDA(cudaGetLastError());
     }
   }
+  if (L.state_only) return KTA_OK;
   {
     TraceScope ts("gla_tc_out", st);
     kta::gla_tc_kernel<true><<<grid, 384, smem, st>>>(tq, tk, tv, ta, p);
@@ -530,8 +535,9 @@ kta_status launch_gla_planned(const LinLaunch& L, const GlaPlan& g, void* ws, cu
   p.nseg = g.nseg;
   p.scale = L.scale;
   p.S0 = L.S0;
-  p.S_out = L.S_out;
-  if (g.nseg > 1) {
+  p.S_out = L.state_only ? nullptr : L.S_out;
+  p.S_fold = L.state_only ? L.S_out : nullptr;
+  if (g.nseg > 1 || L.state_only) {
     // Every word the kernels read from the workspace is written earlier in the same call (the
     // state pass writes all segment states and decays, the carry pass rewrites them in place),
     // so nothing has to be cleared.
@@ -544,7 +550,7 @@ kta_status launch_gla_planned(const LinLaunch& L, const GlaPlan& g, void* ws, cu
       (sa = set_smem_attr(kta::gla_chunk_kernel<D, C, true>, smem)))
     return sa;
   dim3 grid(g.nseg, g.slices, L.B * L.H);
-  if (g.nseg > 1) {
+  if (g.nseg > 1 || L.state_only) {
     {
       TraceScope ts("gla_chunk_state", st);
       kta::gla_chunk_kernel<D, C, false><<<grid, 128, smem, st>>>(p);
@@ -556,6 +562,7 @@ kta_status launch_gla_planned(const LinLaunch& L, const GlaPlan& g, void* ws, cu
     }
   }
   KTA_CUDA(cudaGetLastError());
+  if (L.state_only) return KTA_OK;
   {
     TraceScope ts("gla_chunk_out", st);
     kta::gla_chunk_kernel<D, C, true><<<grid, 128, smem, st>>>(p);
@@ -870,6 +877,36 @@ kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const 
                     false, stream);
 }
 
+kta_status kta_gla_chunk_state(const void* k, const void* v, const float* alpha, const float* S0,
+                               float* S_out, kta_shape s, int H, int ld_heads, int chunk,
+                               void* stream) {
+  kta_status r;
+  if ((r = check_shape(s)) || (r = check_heads(H, ld_heads, s)) || (r = check_ptrs({k, v})))
+    return r;
+  if (s.dtype != KTA_BF16) return fail(KTA_ERR_UNSUPPORTED, "the end-state pass is built for bf16 only");
+  if (!alpha || !S_out) return fail(KTA_ERR_INVALID_ARG, "null alpha or S_out");
+  if (!aligned16(alpha) || (S0 && !aligned16(S0)) || !aligned16(S_out))
+    return fail(KTA_ERR_ALIGNMENT, "gate / state pointers must be 16-byte aligned");
+  if (chunk != 16 && chunk != 32 && chunk != 64)
+    return fail(KTA_ERR_INVALID_ARG, "chunk must be 16, 32 or 64");
+  LinLaunch L;
+  L.B = s.B;
+  L.N = s.F * s.P;
+  L.H = H;
+  L.d = s.d;
+  L.rows_b = L.N;
+  L.chunk = chunk;
+  L.dt = s.dtype;
+  L.k = k;
+  L.v = v;
+  L.ld = static_cast<long long>(ld_heads) * s.d;
+  L.alpha = alpha;
+  L.S0 = S0;
+  L.S_out = S_out;
+  L.state_only = true;
+  return launch_lin(L, as_stream(stream));
+}
+
 kta_status kta_gla_delta_fwd(const void* q, const void* k, const void* v, const float* alpha,
                              const float* beta, const float* S0, float* S_out, void* o,
                              kta_shape s, int H, int ld_heads, int chunk, float scale,
@@ -1010,14 +1047,28 @@ kta_status kta_gla_transition(const float* alpha, float* T, int B, int N, int H,
   if (static_cast<long long>(B) * H > 0x7fffffffLL)
     return fail(KTA_ERR_UNSUPPORTED, "too many sequences x heads");
   if (!aligned16(alpha) || !aligned16(T)) return fail(KTA_ERR_ALIGNMENT, "pointers not 16-byte aligned");
+  if (d != 128 && d != 64 && d != 32) return fail(KTA_ERR_UNSUPPORTED, "d must be 32, 64 or 128 (got %d)", d);
   cudaStream_t st = as_stream(stream);
-  const unsigned grid = static_cast<unsigned>(B * H);
+  // token blocks per (sequence, head): enough CTAs for every SM, at least ~32 tokens each
+  const int G = static_cast<int>(std::max(1LL, std::min<long long>(
+      (2LL * sm_count() + B * H - 1) / (static_cast<long long>(B) * H), (N + 31) / 32)));
+  void* part = nullptr;
+  kta_status r;
+  if ((r = workspace(static_cast<size_t>(B) * H * G * d * sizeof(float), st, &part))) return r;
+  const dim3 grid(static_cast<unsigned>(B * H), static_cast<unsigned>(G));
+  float* pf = static_cast<float*>(part);
   {
     TraceScope ts("gla_transition", st);
-    if (d == 128) kta::gla_transition_kernel<128><<<grid, 1024, 0, st>>>(alpha, T, N, H);
-    else if (d == 64) kta::gla_transition_kernel<64><<<grid, 512, 0, st>>>(alpha, T, N, H);
-    else if (d == 32) kta::gla_transition_kernel<32><<<grid, 256, 0, st>>>(alpha, T, N, H);
-    else return fail(KTA_ERR_UNSUPPORTED, "d must be 32, 64 or 128 (got %d)", d);
+    if (d == 128) {
+      kta::gla_transition_part_kernel<128><<<grid, 512, 0, st>>>(alpha, pf, N, H, G);
+      kta::gla_transition_finish_kernel<128><<<grid.x, 256, 0, st>>>(pf, T, G);
+    } else if (d == 64) {
+      kta::gla_transition_part_kernel<64><<<grid, 256, 0, st>>>(alpha, pf, N, H, G);
+      kta::gla_transition_finish_kernel<64><<<grid.x, 256, 0, st>>>(pf, T, G);
+    } else {
+      kta::gla_transition_part_kernel<32><<<grid, 128, 0, st>>>(alpha, pf, N, H, G);
+      kta::gla_transition_finish_kernel<32><<<grid.x, 256, 0, st>>>(pf, T, G);
+    }
   }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;

@@ -230,33 +230,45 @@ __global__ void __launch_bounds__(256) state_affine_kernel(const float* __restri
 
 // T = diag(prod_t alpha_t) per (sequence, head): the transition of a vector-gated GLA run, whose
 // end state is S_end = diag(prod_t alpha_t) S_start + S_loc (GLA paragraph: the gate scales the
-// state row of each key dim once per token). alpha: [B][N][H][D] fp32; T: [B][H][D][D]. Eight
-// token groups per key dim sum log2(alpha) (clamped at -200, so a zero gate gives 0), combined
-// in shared memory; the whole D x D matrix is written, zeros off the diagonal.
+// state row of each key dim once per token). alpha: [B][N][H][D] fp32; T: [B][H][D][D]. G token
+// blocks per (sequence, head) each sum log2(alpha) per key dim into `part` ([B*H][G][D]); a
+// second kernel adds the G partial sums in order and writes exp2 of the total on the diagonal.
 template <int D>
-__global__ void __launch_bounds__(D * 8) gla_transition_kernel(const float* __restrict__ alpha,
-                                                               float* __restrict__ T, int N,
-                                                               int H) {
-  __shared__ float part[8][D];
-  __shared__ float diag[D];
-  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+__global__ void __launch_bounds__(D * 4) gla_transition_part_kernel(const float* __restrict__ alpha,
+                                                                    float* __restrict__ part,
+                                                                    int N, int H, int G) {
+  // block (bh, blk): sum over its token block of log2(alpha) per key dim, clamped at -200
+  // (a zero gate gives 0); four token groups per key dim, combined in a fixed order
+  __shared__ float s[4][D];
+  const int bh = blockIdx.x, blk = blockIdx.y, b = bh / H, h = bh % H;
   const int i = threadIdx.x % D, g = threadIdx.x / D;
+  const int per = (N + G - 1) / G, t0 = blk * per, t1 = min(N, t0 + per);
   float acc = 0.f;
-  for (int t = g; t < N; t += 8)
+  for (int t = t0 + g; t < t1; t += 4)
     acc += fmaxf(__log2f(alpha[((static_cast<long long>(b) * N + t) * H + h) * D + i]), -200.f);
-  part[g][i] = acc;
+  s[g][i] = acc;
   __syncthreads();
-  if (g == 0) {
-    float s = 0.f;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) s += part[u][i];
-    diag[i] = exp2f(s);
+  if (g == 0) part[(static_cast<long long>(bh) * G + blk) * D + i] = (s[0][i] + s[1][i]) + (s[2][i] + s[3][i]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) gla_transition_finish_kernel(const float* __restrict__ part,
+                                                                    float* __restrict__ T, int G) {
+  // the blocks' sums in block order, then the whole D x D matrix, zeros off the diagonal
+  __shared__ float diag[D];
+  const int bh = blockIdx.x;
+  for (int i = threadIdx.x; i < D; i += 256) {
+    float sum = 0.f;
+    for (int u = 0; u < G; ++u) sum += part[(static_cast<long long>(bh) * G + u) * D + i];
+    diag[i] = exp2f(sum);
   }
   __syncthreads();
-  float* Tb = T + static_cast<long long>(bh) * D * D;
-  for (int e = threadIdx.x; e < D * D; e += D * 8) {
-    const int r = e / D, c = e % D;
-    Tb[e] = r == c ? diag[r] : 0.f;
+  float4* Tb = reinterpret_cast<float4*>(T + static_cast<long long>(bh) * D * D);
+  for (int e = threadIdx.x; e < D * D / 4; e += 256) {
+    const int r = (4 * e) / D, c = (4 * e) % D;
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r >= c && r < c + 4) (&w.x)[r - c] = diag[r];
+    Tb[e] = w;
   }
 }
 

@@ -60,6 +60,7 @@ _SIGS = {
                           _st),
     "kta_gla_gdn_fwd": ([_vp, _vp, _vp, _fp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
                         _st),
+    "kta_gla_chunk_state": ([_vp, _vp, _fp, _fp, _fp, Shape, _i, _i, _i, _vp], _st),
     "kta_gla_chunk_fwd_noalloc": ([_vp, _vp, _vp, _fp, _fp, _fp, _vp, Shape, _i, _i, _i, _f, _vp],
                                   _st),
     "kta_hybrid_fwd": ([ctypes.POINTER(HybridCfg), _vp, _vp, _vp, _fp, _fp, _vp, _vp], _st),
@@ -200,6 +201,24 @@ def gla_chunk_fwd(q, k, v, alpha, *, chunk: int = 64, scale: float = 1.0, S0=Non
                   return_state: bool = False, heads=None, out=None, stream=None):
     """Vector-gated GLA; alpha [B, N, H, d] fp32. Returns o (and the final state)."""
     return _linear(False, q, k, v, alpha, None, chunk, scale, S0, return_state, heads, out, stream)
+
+
+def gla_chunk_state(k, v, alpha, *, chunk: int = 64, S0=None, heads=None, stream=None):
+    """End state [B, H, d, d] fp32 of a vector-gated GLA run (no outputs); k, v bf16."""
+    for n, t in (("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16)
+    _need(alpha, "alpha", torch.float32)
+    B, N, Htot, d = k.shape
+    h0, h1 = heads if heads is not None else (0, Htot)
+    H = h1 - h0
+    if S0 is not None:
+        _need(S0, "S0", torch.float32)
+    S_out = torch.empty((B, H, d, d), device=k.device, dtype=torch.float32)
+    s = Shape(B, 1, N, d, _DT[k.dtype])
+    _check(_lib.kta_gla_chunk_state(_ptr(k, h0 * d), _ptr(v, h0 * d), _ptr(alpha), _ptr(S0),
+                                    _ptr(S_out), s, H, Htot, chunk, _stream(stream)),
+           "kta_gla_chunk_state")
+    return S_out
 
 
 def gla_delta_fwd(q, k, v, alpha, beta, *, chunk: int = 64, scale: float = 1.0, S0=None,

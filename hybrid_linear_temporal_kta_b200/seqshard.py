@@ -236,6 +236,9 @@ class KtaOps:
 
     def lin_state(self, c: ShardCfg, q, k, v, alpha, beta, S0):
         heads = (c.n_swa + c.n_dswa, c.H)
+        if not c.gla_delta and q.dtype == torch.bfloat16:
+            # the end state alone: state pass and segment fold, no output pass
+            return self.kta.gla_chunk_state(k, v, alpha, chunk=c.chunk, S0=S0, heads=heads)
         scratch = torch.empty_like(q)
         if c.gla_delta:
             _, S = self.kta.gla_delta_fwd(q, k, v, alpha, beta, chunk=c.chunk, scale=c.scale_gla,

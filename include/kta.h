@@ -120,6 +120,22 @@ kta_status kta_gla_chunk_fwd(const void* q, const void* k, const void* v, const 
                              int ld_heads, int chunk, float scale, void* stream);
 
 /*
+ * End state of a vector-gated GLA run, without its outputs -- the same recurrence as
+ * kta_gla_chunk_fwd (paper-read, section 2, second pillar, GLA paragraph):
+ *     S_end = diag(prod_t alpha_t) S0 + sum_t diag(prod_{u>t} alpha_u) k_t^T v_t.
+ * k, v: [B][N][ld_heads][d] bf16 rows as in kta_gla_chunk_fwd (N = F * P, first of H heads at the
+ * pointer); alpha [B][N][H][d] fp32; S0 (NULL = zero) and S_out [B][H][d][d] fp32 key-major.
+ * Runs the chunked state pass and the segment fold only (no output pass), for callers that need
+ * a run's state map and not its outputs (a sequence split's per-rank end state from zero).
+ *  - bf16 only, d in {64, 128}, chunk in {16, 32, 64}; KTA_F32 returns KTA_ERR_UNSUPPORTED.
+ *  - S_out must not be NULL; k, v, alpha, S0, S_out 16-byte aligned.
+ *  - Same gate range, workspace and concurrency rules as kta_gla_chunk_fwd.
+ */
+kta_status kta_gla_chunk_state(const void* k, const void* v, const float* alpha, const float* S0,
+                               float* S_out, kta_shape s, int H, int ld_heads, int chunk,
+                               void* stream);
+
+/*
  * kta_gla_chunk_fwd without any device allocation. The pages have no counterpart: this is a
  * service for callers that cannot allocate device memory while they run -- a real-time rollout
  * loop that forbids allocation once started, or a process whose device memory is entirely held

@@ -198,6 +198,25 @@ def test_bf16_gla_matches_oracle(kta, d, chunk, N, B, H):
     assert rel(S.cpu().numpy(), Sref) < BF16_TOL
 
 
+@pytest.mark.parametrize("d,chunk,N,B,H", [(128, 64, 1000, 2, 2), (128, 64, 50, 1, 3),
+                                           (128, 64, 9000, 1, 2), (64, 32, 777, 2, 1),
+                                           (128, 16, 300, 1, 2)])
+def test_bf16_gla_end_state_only_matches_full_forward(kta, d, chunk, N, B, H):
+    """kta_gla_chunk_state (state pass + segment fold, no outputs) against the full forward's
+    S_out and the oracle, with a start state; one segment (N = 50) and many (N = 9000)."""
+    w = synth.HYBRID_BF16.replace(d=d, n_swa=0, n_dswa=0, n_gla=H, chunk=chunk)
+    x = synth.make_inputs(w, N=N, B=B)
+    S0 = torch.from_numpy(np.random.default_rng(4).standard_normal((B, H, d, d)).astype(np.float32))
+    q, k, v, a = dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["alpha"])
+    S = kta.gla_chunk_state(k, v, a, chunk=chunk, S0=dev(S0))
+    _, S_full = kta.gla_chunk_fwd(q, k, v, a, chunk=chunk, S0=dev(S0), return_state=True)
+    kta.device_status()
+    assert torch.isfinite(S).all()
+    assert rel(S.cpu().numpy(), S_full.cpu().numpy()) < 1e-5
+    _, Sref = oracle.gla(x["q"], x["k"], x["v"], x["alpha"], S0=S0)
+    assert rel(S.cpu().numpy(), Sref) < BF16_TOL
+
+
 def small_gates(kind, shape, seed):
     """Forget gates far below the usual range (all valid: alpha in [0, 1))."""
     rng = np.random.default_rng(seed)
