@@ -588,6 +588,18 @@ def run_other(args):
                 st.step(q, k, v, a, out=of)
         ms = _device_ms(rollout, args.steps, args.warmup)
         kern = _traced(rollout, args.steps)
+        # the same rollout captured once as a CUDA graph (240 steps' launches replayed together)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            rollout()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            rollout()
+        ms_graph = _device_ms(graph.replay, args.steps, args.warmup)
+        del graph
         flops = softmax_flops(w)
         t_star = max(flops / (tc * 1e12), (8.0 * w.d * w.B * w.N * (w.n_swa + w.n_dswa) +
                                           gla_bytes(w)) / (hbm * 1e9))
@@ -595,6 +607,9 @@ def run_other(args):
             "workload": w.name, "metric": "streaming rollout tokens/s (one frame per call)",
             "unit": "tokens/s", "value": w.B * w.N / (ms / 1e3), "ms_per_rollout": ms,
             "us_per_frame": ms * 1e3 / w.F, "steps": args.steps,
+            "graph": {"value": w.B * w.N / (ms_graph / 1e3), "ms_per_rollout": ms_graph,
+                      "us_per_frame": ms_graph * 1e3 / w.F,
+                      "note": "the rollout captured once with torch.cuda.graph and replayed"},
             "config": {"B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d,
                        "state_bytes": st.state_bytes},
             "roofline": {"bound": "tensor", "t_star_ms": t_star * 1e3, "frac": t_star / (ms / 1e3),
