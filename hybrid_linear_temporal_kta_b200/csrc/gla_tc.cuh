@@ -86,7 +86,9 @@ struct GlaTcSmem {
   alignas(16) float bmv[GT_D];             // b_m of the current span, per key dim
   int rinfo[2][8];                         // per span parity: lo, hi, flags, stage, chunk
   alignas(16) __nv_bfloat16 otr[4][8][32]; // per state warp: 8 output rows x 32 values (transpose)
+  alignas(128) __nv_bfloat16 ostage[GT_C][GT_D]; // a whole chunk's output rows for one TMA store
   uint64_t full[2], sfree[2], facrdy, opnd, opfree, sready, sdone, odone[2], ofree[2], fin;
+  uint64_t gready;                         // a chunk's cumulative gates are in its alpha stage
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -144,7 +146,7 @@ template <bool OUTPUT>
 __global__ void __launch_bounds__(384, 1)
     gla_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap ta,
-                  const GlaTcParams p) {
+                  const __grid_constant__ CUtensorMap to, const GlaTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   GlaTcSmem& sm = *reinterpret_cast<GlaTcSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&sm.sready, 4);
     mbar_init(&sm.sdone, 1);
     mbar_init(&sm.fin, 1);
+    mbar_init(&sm.gready, 4);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------------ gate warps (key dim kd)
     const int kd = threadIdx.x - 128;
     const int gw = warp - 4;
-    float ltot = 0.f, cend_prev = 1.f;
+    float cend_prev = 1.f;
     int plo = 0, phi = 0;  // rows of the previous span in qs / ks
     int R = 0;
     bool ok = true;
@@ -277,17 +280,9 @@ __global__ void __launch_bounds__(384, 1)
       const int s = c & 1;
       const int n = min(GT_C, t_end - t_begin - c * GT_C);
       if (!gt_all(!*abort_flag && mbar_wait(&sm.full[s], (c >> 1) & 1))) { ok = false; break; }
-      // cumulative log2 gate of this key dim over the chunk, written over its alpha column (the
-      // stage stays untouched by the producer until the chunk's MMAs are done); rows >= n: alpha = 1.
-      // Each log2 gate is clamped to [-200, 0], so b_t never increases with t.
+      // the state warps have replaced this chunk's alpha columns by the cumulative log2 gates
+      if (!gt_all(!*abort_flag && mbar_wait(&sm.gready, c & 1))) { ok = false; break; }
       const uint32_t bcol = smem_u32(&sm.alpha[s][0][kd]);
-      float acc = 0.f;
-      for (int t = 0; t < GT_C; ++t) {
-        const uint32_t a = bcol + t * GT_D * 4;
-        acc += fmaxf(fminf(__log2f(t < n ? gt_lds_f32(a) : 1.f), 0.f), -200.f);
-        asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(acc) : "memory");
-      }
-      ltot += acc;
       auto bt = [&](int t) { return gt_lds_f32(bcol + t * GT_D * 4); };
       // span plan: the whole chunk, 16-token spans, or single tokens. A span [lo, hi) with middle
       // m = lo + (hi - lo) / 2 passes when every |b_t - b_m| <= KTA_GLA_LIM; b is monotone, so the
@@ -454,14 +449,37 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(&sm.facrdy);
         mbar_arrive(&sm.opnd);
       }
-    } else if (!OUTPUT) {
-      p.ws_L[(static_cast<long long>(bh) * p.nseg + seg) * GT_D + kd] = ltot;
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------------ state warps (value vd)
     const int quad = warp & 3;
     const int vd = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    // Cumulative log2 gate of key dim vd over chunk cc, written over its alpha column (the stage
+    // stays untouched by the producer until the chunk's MMAs are done); rows >= n: alpha = 1. Each
+    // log2 gate is clamped to [-200, 0], so b_t never increases with t. The state warps do this
+    // one chunk ahead of the gate warps, which wait for it on `gready`.
+    float ltot = 0.f;
+    auto cumsum = [&](int cc) {
+      const int sc = cc & 1;
+      const int n = min(GT_C, t_end - t_begin - cc * GT_C);
+      const bool got = !*abort_flag && mbar_wait(&sm.full[sc], (cc >> 1) & 1);
+      if (!__all_sync(0xffffffffu, got)) return false;
+      const uint32_t bcol = smem_u32(&sm.alpha[sc][0][vd]);
+      float acc = 0.f;
+      for (int t = 0; t < GT_C; ++t) {
+        const uint32_t a = bcol + t * GT_D * 4;
+        acc += fmaxf(fminf(__log2f(t < n ? gt_lds_f32(a) : 1.f), 0.f), -200.f);
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(acc) : "memory");
+      }
+      ltot += acc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.gready);
+      return true;
+    };
+    int next_cum = 1;  // the next chunk whose gates are still raw
+    bool ok = cumsum(0);
+    if (!ok) *abort_flag = 1;
     // start state: S0 for a single segment, else the carry kernel's start of this segment, or
     // (fold) S_start(s+1) = 2^{L_s} S_start(s) + S_loc(s) over the predecessors, as the carry
     // kernel computes it
@@ -490,12 +508,23 @@ __global__ void __launch_bounds__(384, 1)
       tmem_st32(tS + lane_off + 32 * c4, r);
     }
     tmem_wait_st();
-    bool ok = true;
     int R = 0, lo_prev = 0, hi_prev = 0, c_prev = 0;
+    // All-of over the four state warps (named barrier 3), so that they take the same path.
+    auto st_all = [&](bool v) {
+      uint32_t r;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+          "bar.red.and.pred q, 3, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(r)
+          : "r"(static_cast<uint32_t>(v))
+          : "memory");
+      return r != 0;
+    };
+    const bool store_lead = warp == 8 && lane == 0;  // issues the output TMA stores
     auto epilogue = [&](int Rq, int lo, int hi, int c) -> bool {
       const int ob = Rq & 1;
       const bool got = mbar_wait(&sm.odone[ob], (Rq >> 1) & 1);
-      if (!__all_sync(0xffffffffu, got)) return false;
+      if (!st_all(got)) return false;
       tc_fence_after();
       uint32_t r[64];
       tmem_ld32(tO0 + 64 * ob + lane_off, *reinterpret_cast<uint32_t(*)[32]>(r));
@@ -505,8 +534,31 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.ofree[ob]);
-      // rows [lo, hi) of this warp's 32 value columns, eight rows at a time through a small
-      // transpose buffer: each thread then stores 16 bytes (8 values of one row)
+      const int n = min(GT_C, t_end - t_begin - c * GT_C);
+      if (lo == 0 && hi == n) {
+        // the whole chunk: thread vd writes its value column of the 64 rows into the staging tile
+        // (row-major, 256 bytes a row), then one thread stores the tile with the TMA unit (rows
+        // past the sequence's end are outside the map and not written)
+        if (store_lead) bulk_wait_read_all();  // the previous store has read the tile
+        asm volatile("bar.sync 3, 128;" ::: "memory");
+        const uint32_t col = smem_u32(&sm.ostage[0][vd]);
+#pragma unroll
+        for (int t = 0; t < GT_C; ++t) {
+          const __nv_bfloat16 x = __float2bfloat16_rn(__uint_as_float(r[t]) * p.scale);
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(col + t * GT_D * 2),
+                       "h"(*reinterpret_cast<const uint16_t*>(&x))
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 3, 128;" ::: "memory");
+        if (store_lead) {
+          tma_store_4d(&to, &sm.ostage[0][0], 0, h, t_begin + c * GT_C, b);
+          bulk_commit();
+        }
+        return true;
+      }
+      // a span inside the chunk: rows [lo, hi) of this warp's 32 value columns, eight rows at a
+      // time through a small transpose buffer (each thread then stores 16 bytes of one row)
       __nv_bfloat16 (*tb)[32] = sm.otr[quad];
       const int tr = lane >> 2, tc = (lane & 3) * 8;
       __nv_bfloat16* obase = p.o + (row_b + t_begin + c * GT_C) * p.ld +
@@ -525,7 +577,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       return true;
     };
-    for (;; ++R) {
+    for (; ok; ++R) {
       const bool got = !*abort_flag && (R == 0 || mbar_wait(&sm.sdone, (R - 1) & 1)) &&
                        mbar_wait(&sm.facrdy, R & 1);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -555,6 +607,11 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.sready);
+      // the next chunk's gates, before this warp's output rows, so that the gate warps can start it
+      if (next_cum == c + 1 && next_cum < nchunk) {
+        if (!cumsum(next_cum)) { ok = false; break; }
+        ++next_cum;
+      }
       if (OUTPUT && R > 0 && !epilogue(R - 1, lo_prev, hi_prev, c_prev)) { ok = false; break; }
       lo_prev = lo;
       hi_prev = hi;
@@ -562,6 +619,8 @@ __global__ void __launch_bounds__(384, 1)
       if (flags & GT_LAST_OF_SEG) break;
     }
     if (ok && OUTPUT && !epilogue(R, lo_prev, hi_prev, c_prev)) ok = false;
+    if (OUTPUT && store_lead) bulk_wait_all();  // the output stores are complete before exit
+    if (ok && !OUTPUT) p.ws_L[(static_cast<long long>(bh) * p.nseg + seg) * GT_D + vd] = ltot;
     // end state of the segment: S^T diag(cend of the last span), written key-major
     const bool fin = ok && mbar_wait(&sm.sdone, R & 1);
     if (__all_sync(0xffffffffu, fin)) {

@@ -462,6 +462,17 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
       (r = make_map_box(&ta, L.alpha, true, D, L.H, rows, static_cast<long long>(L.H) * D, D,
                         kta::GT_C)))
     return r;
+  // o: stores of whole 64-token chunks, [64 rows][128 values] unswizzled, per (head, sequence);
+  // rows past N are outside the map
+  CUtensorMap to = tq;
+  if (!L.state_only) {
+    const cuuint64_t dO[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L.H),
+                              static_cast<cuuint64_t>(L.N), static_cast<cuuint64_t>(L.B)};
+    const cuuint64_t sO[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L.ld) * 2,
+                              static_cast<cuuint64_t>(L.rows_b) * L.ld * 2};
+    const cuuint32_t bO[4] = {static_cast<cuuint32_t>(D), 1, static_cast<cuuint32_t>(kta::GT_C), 1};
+    if ((r = make_map_nd(&to, L.o, 4, dO, sO, bO, CU_TENSOR_MAP_SWIZZLE_NONE))) return r;
+  }
   kta::GlaTcParams p{};
   p.N = L.N;
   p.H = L.H;
@@ -488,7 +499,7 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
   if (g.nseg > 1 || L.state_only) {
     {
       TraceScope ts("gla_tc_state", st);
-      kta::gla_tc_kernel<false><<<grid, 384, smem, st>>>(tq, tk, tv, ta, p);
+      kta::gla_tc_kernel<false><<<grid, 384, smem, st>>>(tq, tk, tv, ta, to, p);
     }
     KTA_CUDA(cudaGetLastError());
     if (!p.fold) {
@@ -508,7 +519,7 @@ kta_status launch_gla_tc(const LinLaunch& L, const GlaPlan& g, void* ws, cudaStr
   if (L.state_only) return KTA_OK;
   {
     TraceScope ts("gla_tc_out", st);
-    kta::gla_tc_kernel<true><<<grid, 384, smem, st>>>(tq, tk, tv, ta, p);
+    kta::gla_tc_kernel<true><<<grid, 384, smem, st>>>(tq, tk, tv, ta, to, p);
   }
   KTA_CUDA(cudaGetLastError());
   return KTA_OK;
