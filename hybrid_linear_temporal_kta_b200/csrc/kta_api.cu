@@ -78,13 +78,13 @@ EncodeTiledFn encode_fn() {
 // dim2 = rows (stride ld elements); box = 64 columns x 1 head x 128 rows, 128-byte swizzle,
 // zero fill outside the tensor.
 kta_status make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows,
-                    long long ld) {
+                    long long ld, int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(KTA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
                         static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -283,6 +283,17 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   if ((s = make_map(&tv0, g0.v, D, g0.k_heads, g0.k_rows, g0.k_ld))) return s;
   if ((s = make_map(&tk1, g1.k, D, g1.k_heads, g1.k_rows, g1.k_ld))) return s;
   if ((s = make_map(&tv1, g1.v, D, g1.k_heads, g1.k_rows, g1.k_ld))) return s;
+  // 8-row boxes for the key tiles that span two frames of a dilated window (packed tiling)
+  CUtensorMap tk0s = tk0, tv0s = tv0, tk1s = tk1, tv1s = tv1;
+  const bool pk = L.P % 8 == 0;
+  if (pk && g0.dil > 1 &&
+      ((s = make_map(&tk0s, g0.k, D, g0.k_heads, g0.k_rows, g0.k_ld, 8)) ||
+       (s = make_map(&tv0s, g0.v, D, g0.k_heads, g0.k_rows, g0.k_ld, 8))))
+    return s;
+  if (pk && g1.dil > 1 &&
+      ((s = make_map(&tk1s, g1.k, D, g1.k_heads, g1.k_rows, g1.k_ld, 8)) ||
+       (s = make_map(&tv1s, g1.v, D, g1.k_heads, g1.k_rows, g1.k_ld, 8))))
+    return s;
   WinParams p{};
   p.B = L.B;
   p.P = L.P;
@@ -319,10 +330,10 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
     TraceScope ts("win_attn_tc", st);
     if (L.lse)
       kta::win_attn_tc_kernel<D, true><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
-          tq, tk0, tv0, tk1, tv1, p);
+          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, p);
     else
       kta::win_attn_tc_kernel<D, false><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
-          tq, tk0, tv0, tk1, tv1, p);
+          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, p);
   }
   const cudaError_t le = cudaGetLastError();
   if (le != cudaSuccess) {

@@ -6,8 +6,10 @@
 //
 // Query tiles of up to 128 rows lie in ONE frame (tiles restart at every frame start), so every
 // row of a tile sees the same key frames and the only mask is a column bound on the last key tile
-// of each key span. Key spans: for dil == 1 the W visible frames are adjacent and form one span;
-// for dil > 1 each visible frame is its own span.
+// of the window (or of each key span). For dil == 1 the W visible frames are adjacent and form
+// one span; for dil > 1 with P a multiple of 8 the visible frames are packed into one sequence of
+// keys whose tiles may straddle two frames (loaded as 8-row boxes from both), otherwise each
+// visible frame is its own span.
 //
 // One CTA (one per SM: it holds all 512 TMEM columns) computes a PAIR of query tiles A and B of
 // the same sequence, head and frame (launches too small to fill the GPU with pairs give each CTA
@@ -107,6 +109,43 @@ __device__ __forceinline__ void win_tile(int i, int f, int P, int W, int dil, in
   nvalid = min(128, P - off);
 }
 
+// Key tiles of the forward kernel. For dil > 1 with P a multiple of 8 the visible frames are
+// packed: they form one sequence of nsp * P keys cut into 128-key tiles, so only the window's last
+// tile is ragged (per-frame tiles would leave a ragged tile in every frame). A packed tile takes
+// rows_a rows (a multiple of 8) from frame fr_a at row off_a and the rest from the first rows of
+// frame fr_b; nv keys of it are visible. Otherwise the tiles are win_tile's.
+struct WinKTile {
+  int fr_a, off_a, rows_a, fr_b, nv;
+};
+// (packed only where it saves tiles: with P = 880 the per-frame tiles are already as few)
+__device__ __forceinline__ bool win_packed(int f, int P, int W, int dil) {
+  if (dil == 1 || (P & 7) != 0) return false;
+  const int nsp = min(W, f / dil + 1);
+  return (nsp * P + 127) / 128 < nsp * ((P + 127) / 128);
+}
+__device__ __forceinline__ int win_ktiles(int f, int P, int W, int dil) {
+  if (!win_packed(f, P, W, dil)) return win_num_tiles(f, P, W, dil);
+  return (min(W, f / dil + 1) * P + 127) / 128;
+}
+__device__ __forceinline__ WinKTile win_ktile(int i, int f, int P, int W, int dil) {
+  WinKTile t;
+  if (!win_packed(f, P, W, dil)) {
+    win_tile(i, f, P, W, dil, t.fr_a, t.off_a, t.nv);
+    t.rows_a = 128;
+    t.fr_b = t.fr_a;
+    return t;
+  }
+  const int nsp = min(W, f / dil + 1);
+  const int v0 = 128 * i, j = v0 / P, o1 = v0 - j * P;
+  t.fr_a = f - (nsp - 1 - j) * dil;
+  t.off_a = o1;
+  t.rows_a = min(128, P - o1);
+  // rows past the window's last key come from any visible frame (finite data, masked by nv)
+  t.fr_b = j + 1 < nsp ? t.fr_a + dil : t.fr_a;
+  t.nv = min(128, nsp * P - v0);
+  return t;
+}
+
 template <int D>
 struct WinSmem {
   static constexpr int BOX = 128 * 64 * 2;  // one 128-row x 64-column bf16 box, 16 KB
@@ -134,7 +173,11 @@ __global__ void __launch_bounds__(384, 1)
                        const __grid_constant__ CUtensorMap tk0,
                        const __grid_constant__ CUtensorMap tv0,
                        const __grid_constant__ CUtensorMap tk1,
-                       const __grid_constant__ CUtensorMap tv1, const WinParams p) {
+                       const __grid_constant__ CUtensorMap tv1,
+                       const __grid_constant__ CUtensorMap tk0s,
+                       const __grid_constant__ CUtensorMap tv0s,
+                       const __grid_constant__ CUtensorMap tk1s,
+                       const __grid_constant__ CUtensorMap tv1s, const WinParams p) {
   static_assert(D == 64 || D == 128, "head dim");
   extern __shared__ uint8_t smem_raw[];
   WinSmem<D>& sm = *reinterpret_cast<WinSmem<D>*>(
@@ -158,7 +201,9 @@ __global__ void __launch_bounds__(384, 1)
   const int kmod = g ? p.kmod[1] : p.kmod[0];
   const CUtensorMap* tk = g ? &tk1 : &tk0;
   const CUtensorMap* tv = g ? &tv1 : &tv0;
-  const int ntiles = win_num_tiles(f, p.P, W, dil);
+  const CUtensorMap* tks = g ? &tk1s : &tk0s;  // 8-row boxes, for tiles that span two frames
+  const CUtensorMap* tvs = g ? &tv1s : &tv0s;
+  const int ntiles = win_ktiles(f, p.P, W, dil);
   const bool has_b = p.pair == 2 && 2 * pr + 1 < p.n_qt;
   // A CTA with one query tile and at least two key tiles splits the key range instead: tile slot 0
   // takes key tiles [0, nA), slot 1 the rest for the same query rows, and the two partial softmax
@@ -211,15 +256,24 @@ __global__ void __launch_bounds__(384, 1)
       int uses[NSLOT] = {0, 0, 0, 0};
       // load (key tile kt, V or K) into `slot` as that slot's next use
       auto load = [&](int kt, bool is_v, int slot) {
-        int fr0, off, nv;
-        win_tile(kt, f, p.P, W, dil, fr0, off, nv);
-        const int krow = (b * kbf + fr0 % kmod) * p.P + off;
+        const WinKTile t = win_ktile(kt, f, p.P, W, dil);
+        const int krow = (b * kbf + t.fr_a % kmod) * p.P + t.off_a;
         const int use = uses[slot];
         if (use > 0 && !mbar_wait(&sm.empty[slot], (use - 1) & 1)) { *abort_flag = 1; return false; }
         mbar_arrive_expect_tx(&sm.full[slot], TILE_BYTES);
-        const CUtensorMap* tm = is_v ? tv : tk;
-        for (int c = 0; c < NBOX; ++c)
-          tma_load_3d(sm.kv[slot] + c * BOX, tm, &sm.full[slot], c * 64, hk, krow);
+        if (t.rows_a == 128) {
+          const CUtensorMap* tm = is_v ? tv : tk;
+          for (int c = 0; c < NBOX; ++c)
+            tma_load_3d(sm.kv[slot] + c * BOX, tm, &sm.full[slot], c * 64, hk, krow);
+        } else {
+          // a tile across two frames, in 8-row boxes (one 128-byte swizzle atom each)
+          const CUtensorMap* tm = is_v ? tvs : tks;
+          const int krow_b = (b * kbf + t.fr_b % kmod) * p.P - t.rows_a;
+          for (int c = 0; c < NBOX; ++c)
+            for (int r = 0; r < 128; r += 8)
+              tma_load_3d(sm.kv[slot] + c * BOX + r * 128, tm, &sm.full[slot], c * 64, hk,
+                          r < t.rows_a ? krow + r : krow_b + r);
+        }
         uses[slot] = use + 1;
         return true;
       };
@@ -364,8 +418,7 @@ __global__ void __launch_bounds__(384, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = n_x > 0;
     for (int i = 0; ok && i < n_x; ++i) {
-      int fr0, off, nv;
-      win_tile(kt0 + i, f, p.P, W, dil, fr0, off, nv);
+      const int nv = win_ktile(kt0 + i, f, p.P, W, dil).nv;
       const bool got = !*abort_flag && mbar_wait(&sm.bar_s[x], i & 1);
       if (!__all_sync(0xffffffffu, got)) { *abort_flag = 1; ok = false; break; }
       tc_fence_after();
