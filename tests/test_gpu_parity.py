@@ -470,3 +470,52 @@ def test_repeat_runs_are_bit_identical(kta):
     o1 = kta.hybrid_fwd(cfg, *args)
     o2 = kta.hybrid_fwd(cfg, *args)
     assert torch.equal(o1, o2)
+
+
+def test_hybrid_and_stream_replay_as_cuda_graphs(kta):
+    """The hybrid call (its fork onto two internal streams and join) and a streamed rollout
+    (ring gather, one-frame softmax, GLA beside it) captured with torch.cuda.graph and replayed:
+    bit-identical to the eager calls."""
+    w = synth.STREAM_BF16.replace(F=6, P=200, n_swa=2, n_dswa=2, n_gla=2)
+    x = synth.make_inputs(w, B=2)
+    cfg = kta.cfg_from_workload(w, B=2)
+    q, k, v, a = dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["alpha"])
+    ref = kta.hybrid_fwd(cfg, q, k, v, a)
+    st = kta.Stream(cfg)
+    P = w.P
+    frames = [tuple(t[:, f * P:(f + 1) * P].contiguous() for t in (q, k, v, a)) for f in range(w.F)]
+    outs = [torch.empty_like(fr[0]) for fr in frames]
+
+    def rollout():
+        st.reset()
+        for (qf, kf, vf, af), of in zip(frames, outs):
+            st.step(qf, kf, vf, af, out=of)
+
+    rollout()  # eager: allocates the library's workspaces and side streams before capture
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs]
+    o_graph = torch.empty_like(ref)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        kta.hybrid_fwd(cfg, q, k, v, a, out=o_graph)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1):
+        kta.hybrid_fwd(cfg, q, k, v, a, out=o_graph)
+    with torch.cuda.graph(g2):
+        rollout()
+    for o in outs:
+        o.zero_()
+    o_graph.zero_()
+    g1.replay()
+    g2.replay()
+    torch.cuda.synchronize()
+    kta.device_status()
+    assert torch.equal(o_graph, ref)
+    for o, e in zip(outs, eager):
+        assert torch.equal(o, e)
+    assert st.frame == w.F
+    del g1, g2
+    st.close()
