@@ -153,7 +153,7 @@ struct WinSmem {
   static constexpr int NSLOT = 4;           // K / V ring slots
   alignas(1024) uint8_t q[2][NBOX * BOX];
   alignas(1024) uint8_t kv[NSLOT][NBOX * BOX];
-  uint64_t bar_q, full[NSLOT], empty[NSLOT], bar_s[2], bar_p[2], bar_o[2], bar_fin;
+  uint64_t bar_q[2], full[NSLOT], empty[NSLOT], bar_s[2], bar_p[2], bar_o[2], bar_fin;
   float part_m[128], part_l[128];  // key split: row max and row sum of the second key half
   int part_ok[4];                  // key split: the second half's warps finished
   uint32_t tmem_base;
@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(384, 1)
   const int q_row0 = b * p.q_rows_b + f_local * p.P + pr * p.pair * 128;  // tile A; B = +128
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.bar_q, 1);
+    mbar_init(&sm.bar_q[0], 1);
+    mbar_init(&sm.bar_q[1], 1);
     for (int s = 0; s < NSLOT; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
@@ -248,11 +249,18 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tmap(tv);
       if (half == 0) {
         prefetch_tmap(&tq);
-        mbar_arrive_expect_tx(&sm.bar_q, has_b ? 2 * TILE_BYTES : TILE_BYTES);
-        for (int x = 0; x < (has_b ? 2 : 1); ++x)
-          for (int c = 0; c < NBOX; ++c)
-            tma_load_3d(sm.q[x] + c * BOX, &tq, &sm.bar_q, c * 64, h, q_row0 + 128 * x);
+        // Q_A first, then K_0 (below), then Q_B: the first product S_A(0) needs only Q_A and K_0
+        mbar_arrive_expect_tx(&sm.bar_q[0], TILE_BYTES);
+        for (int c = 0; c < NBOX; ++c)
+          tma_load_3d(sm.q[0] + c * BOX, &tq, &sm.bar_q[0], c * 64, h, q_row0);
       }
+      bool qb_issued = false;
+      auto load_qb = [&]() {
+        qb_issued = true;
+        mbar_arrive_expect_tx(&sm.bar_q[1], TILE_BYTES);
+        for (int c = 0; c < NBOX; ++c)
+          tma_load_3d(sm.q[1] + c * BOX, &tq, &sm.bar_q[1], c * 64, h, q_row0 + 128);
+      };
       int uses[NSLOT] = {0, 0, 0, 0};
       // load (key tile kt, V or K) into `slot` as that slot's next use
       auto load = [&](int kt, bool is_v, int slot) {
@@ -279,8 +287,10 @@ __global__ void __launch_bounds__(384, 1)
       };
       if (!split) {
         // load n: K_{n/2} (n even) or V_{n/2} (n odd), slot n % NSLOT
-        for (int n = 0; n < 2 * ntiles; ++n)
+        for (int n = 0; n < 2 * ntiles; ++n) {
           if (*abort_flag || !load(n >> 1, n & 1, n % NSLOT)) break;
+          if (n == 0 && has_b) load_qb();
+        }
       } else {
         // this half's step i: K into slot `half`, V into slot 2 + `half`
         const int nh = half ? nB : nA, kt0 = half ? nA : 0;
@@ -288,7 +298,10 @@ __global__ void __launch_bounds__(384, 1)
           if (*abort_flag || !load(kt0 + i, false, half) || !load(kt0 + i, true, 2 + half)) break;
       }
       // Let the copies this thread started land before the CTA can exit (bounded waits).
-      if (half == 0) mbar_wait(&sm.bar_q, 0);
+      if (half == 0) {
+        mbar_wait(&sm.bar_q[0], 0);
+        if (qb_issued) mbar_wait(&sm.bar_q[1], 0);
+      }
       for (int sl = 0; sl < NSLOT; ++sl)
         if (uses[sl] > 0) mbar_wait(&sm.full[sl], (uses[sl] - 1) & 1);
     }
@@ -319,13 +332,17 @@ __global__ void __launch_bounds__(384, 1)
                  (!first || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar_o[x]);
       };
-      bool ok = mbar_wait(&sm.bar_q, 0) && ntiles > 0;
+      bool ok = mbar_wait(&sm.bar_q[0], 0) && ntiles > 0;
       if (!split) {
         if (ok && !mbar_wait(&sm.full[0], 0)) ok = false;
         if (ok) {
           tc_fence_after();
           issue_s(0, 0);
-          if (has_b) issue_s(1, 0);
+          if (has_b) {
+            if (!mbar_wait(&sm.bar_q[1], 0)) ok = false;
+            tc_fence_after();
+            if (ok) issue_s(1, 0);
+          }
           mma_commit(&sm.empty[0]);
         }
         for (int i = 0; ok && i < ntiles; ++i) {
