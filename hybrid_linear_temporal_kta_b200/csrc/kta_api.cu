@@ -256,6 +256,7 @@ struct WinGroup {
   int k_heads = 0;           // heads in one row of the buffer addressed by the map
   int kh_off = 0;
   int kb_frames = 0, kmod = 1;
+  int span_mode = 0;         // 1: visible frames not adjacent in the buffer (a ring of W slots)
 };
 
 struct WinLaunch {
@@ -286,11 +287,11 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   // 8-row boxes for the key tiles that span two frames of a dilated window (packed tiling)
   CUtensorMap tk0s = tk0, tv0s = tv0, tk1s = tk1, tv1s = tv1;
   const bool pk = L.P % 8 == 0;
-  if (pk && g0.dil > 1 &&
+  if (pk && (g0.dil > 1 || g0.span_mode) &&
       ((s = make_map(&tk0s, g0.k, D, g0.k_heads, g0.k_rows, g0.k_ld, 8)) ||
        (s = make_map(&tv0s, g0.v, D, g0.k_heads, g0.k_rows, g0.k_ld, 8))))
     return s;
-  if (pk && g1.dil > 1 &&
+  if (pk && (g1.dil > 1 || g1.span_mode) &&
       ((s = make_map(&tk1s, g1.k, D, g1.k_heads, g1.k_rows, g1.k_ld, 8)) ||
        (s = make_map(&tv1s, g1.v, D, g1.k_heads, g1.k_rows, g1.k_ld, 8))))
     return s;
@@ -309,6 +310,7 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
     p.kh_off[i] = g.kh_off;
     p.kb_frames[i] = g.kb_frames;
     p.kmod[i] = g.kmod;
+    p.span_mode[i] = g.span_mode;
   }
   p.q_rows_b = L.q_rows_b;
   p.scale_log2 = L.scale * 1.4426950408889634f;
@@ -1117,7 +1119,7 @@ struct kta_stream_s {
   kta_hybrid_cfg cfg;
   int device = 0;
   int64_t frame = 0;
-  int R_swa = 0, R_dswa = 0;    // ring slots (SWA ring is stored twice: 2 * R_swa frames)
+  int R_swa = 0, R_dswa = 0;    // ring slots: a frame's keys and values go to slot f % R
   size_t es = 2;
   char* arena = nullptr;        // [header | swa k | swa v | dswa k | dswa v | state 0 | state 1]
   size_t arena_bytes = 0;
@@ -1149,9 +1151,9 @@ kta_status valid_stream(kta_stream_t st) {
   return KTA_OK;
 }
 
-// One frame's keys and values into the rings: up to six row-block copies (SWA k and v into both
-// copies of their slot, DSWA k and v) in one launch, 16 bytes per thread and step. A copy takes
-// heads [h0, h0+nh) of a frame ([B][P][H][d]) into ring slot `slot` ([B][RR][P][nh][d]).
+// One frame's keys and values into the rings: up to four row-block copies (SWA k and v, DSWA k
+// and v) in one launch, 16 bytes per thread and step. A copy takes heads [h0, h0+nh) of a frame
+// ([B][P][H][d]) into ring slot `slot` ([B][RR][P][nh][d]).
 struct RingCopy {
   const char* src = nullptr;
   char* dst = nullptr;
@@ -1161,7 +1163,7 @@ struct RingCopy {
 };
 constexpr int kRingRows = 16;  // rows per block
 struct RingPutParams {
-  RingCopy c[6];
+  RingCopy c[4];
   int B = 0, P = 0;
 };
 
@@ -1590,7 +1592,7 @@ kta_status kta_stream_create(const kta_hybrid_cfg* cfg, kta_stream_t* out) {
   s->R_dswa = c.n_dswa ? (c.W_dswa - 1) * c.dil + 1 : 0;
   const size_t frame_bytes_swa = static_cast<size_t>(c.s.P) * c.n_swa * c.s.d * s->es;
   const size_t frame_bytes_dswa = static_cast<size_t>(c.s.P) * c.n_dswa * c.s.d * s->es;
-  s->ring_swa_bytes = round_up(static_cast<size_t>(c.s.B) * 2 * s->R_swa * frame_bytes_swa, 256);
+  s->ring_swa_bytes = round_up(static_cast<size_t>(c.s.B) * s->R_swa * frame_bytes_swa, 256);
   s->ring_dswa_bytes = round_up(static_cast<size_t>(c.s.B) * s->R_dswa * frame_bytes_dswa, 256);
   s->state_bytes = round_up(static_cast<size_t>(c.s.B) * c.n_gla * c.s.d * c.s.d * 4, 256);
   size_t off = kHeader;
@@ -1647,11 +1649,9 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
     rp.P = sh.P;
     int nc = 0;
     if (c.n_swa) {
-      const int slot = f % s->R_swa, RR = 2 * s->R_swa;
-      rp.c[nc++] = ring_copy(s, k_f, swa_k, 0, c.n_swa, RR, slot);
-      rp.c[nc++] = ring_copy(s, k_f, swa_k, 0, c.n_swa, RR, slot + s->R_swa);
-      rp.c[nc++] = ring_copy(s, v_f, swa_v, 0, c.n_swa, RR, slot);
-      rp.c[nc++] = ring_copy(s, v_f, swa_v, 0, c.n_swa, RR, slot + s->R_swa);
+      const int slot = f % s->R_swa;
+      rp.c[nc++] = ring_copy(s, k_f, swa_k, 0, c.n_swa, s->R_swa, slot);
+      rp.c[nc++] = ring_copy(s, v_f, swa_v, 0, c.n_swa, s->R_swa, slot);
     }
     if (c.n_dswa) {
       const int slot = f % s->R_dswa;
@@ -1686,11 +1686,12 @@ kta_status kta_stream_step(kta_stream_t s, const void* q_f, const void* k_f, con
       g.k = swa_k;
       g.v = swa_v;
       g.k_ld = static_cast<long long>(c.n_swa) * sh.d;
-      g.k_rows = static_cast<long long>(sh.B) * 2 * s->R_swa * sh.P;
+      g.k_rows = static_cast<long long>(sh.B) * s->R_swa * sh.P;
       g.k_heads = c.n_swa;
       g.kh_off = 0;
-      g.kb_frames = 2 * s->R_swa;
+      g.kb_frames = s->R_swa;
       g.kmod = s->R_swa;
+      g.span_mode = 1;  // the window's frames wrap around the ring
     }
     if (c.n_dswa) {
       WinGroup& g = L.g[gi++];

@@ -54,6 +54,8 @@ struct WinParams {
   int kh_off[2];    // head coordinate in the group's K/V map = h - kh_off[g]
   int kb_frames[2]; // frames per sequence in the group's K/V buffer
   int kmod[2];      // frame index modulus in the K/V buffer (ring slots; = F for a sequence)
+  int span_mode[2]; // 1: the group's visible frames are not adjacent in its buffer (a ring of
+                    // W slots), so each frame is its own span even with dil == 1
   int q_rows_b;     // rows per sequence in the q / o buffers
   float scale_log2; // softmax scale * log2(e)
   __nv_bfloat16* o; // output, already offset to the launch's first head
@@ -117,25 +119,43 @@ __device__ __forceinline__ void win_tile(int i, int f, int P, int W, int dil, in
 struct WinKTile {
   int fr_a, off_a, rows_a, fr_b, nv;
 };
-// (packed only where it saves tiles: with P = 880 the per-frame tiles are already as few)
-__device__ __forceinline__ bool win_packed(int f, int P, int W, int dil) {
-  if (dil == 1 || (P & 7) != 0) return false;
+// (packed only where it saves tiles: with P = 880 the per-frame tiles are already as few). With
+// `spans` (a dil == 1 window whose frames sit in a ring, not side by side) each frame is its own
+// span as well, and the frames are packed whenever P is a multiple of 8: the packed tiles then
+// start at the same keys as the tiles of the adjacent-frame layout, so results agree bit for bit.
+__device__ __forceinline__ bool win_per_frame(int dil, bool spans) { return dil > 1 || spans; }
+__device__ __forceinline__ bool win_packed(int f, int P, int W, int dil, bool spans) {
+  if (!win_per_frame(dil, spans) || (P & 7) != 0) return false;
+  if (dil == 1) return true;
   const int nsp = min(W, f / dil + 1);
   return (nsp * P + 127) / 128 < nsp * ((P + 127) / 128);
 }
-__device__ __forceinline__ int win_ktiles(int f, int P, int W, int dil) {
-  if (!win_packed(f, P, W, dil)) return win_num_tiles(f, P, W, dil);
-  return (min(W, f / dil + 1) * P + 127) / 128;
+__device__ __forceinline__ int win_ktiles(int f, int P, int W, int dil, bool spans) {
+  if (!win_per_frame(dil, spans)) return win_num_tiles(f, P, W, dil);
+  const int nsp = min(W, f / dil + 1);
+  if (!win_packed(f, P, W, dil, spans)) return nsp * ((P + 127) / 128);
+  return (nsp * P + 127) / 128;
 }
-__device__ __forceinline__ WinKTile win_ktile(int i, int f, int P, int W, int dil) {
+__device__ __forceinline__ WinKTile win_ktile(int i, int f, int P, int W, int dil, bool spans) {
   WinKTile t;
-  if (!win_packed(f, P, W, dil)) {
+  if (!win_per_frame(dil, spans)) {
     win_tile(i, f, P, W, dil, t.fr_a, t.off_a, t.nv);
     t.rows_a = 128;
     t.fr_b = t.fr_a;
     return t;
   }
   const int nsp = min(W, f / dil + 1);
+  if (!win_packed(f, P, W, dil, spans)) {
+    // one frame per span, its own tiles
+    const int tp = (P + 127) / 128;
+    const int j = i / tp, tt = i % tp;
+    t.fr_a = f - (nsp - 1 - j) * dil;
+    t.off_a = 128 * tt;
+    t.nv = min(128, P - t.off_a);
+    t.rows_a = 128;
+    t.fr_b = t.fr_a;
+    return t;
+  }
   const int v0 = 128 * i, j = v0 / P, o1 = v0 - j * P;
   t.fr_a = f - (nsp - 1 - j) * dil;
   t.off_a = o1;
@@ -203,7 +223,8 @@ __global__ void __launch_bounds__(384, 1)
   const CUtensorMap* tv = g ? &tv1 : &tv0;
   const CUtensorMap* tks = g ? &tk1s : &tk0s;  // 8-row boxes, for tiles that span two frames
   const CUtensorMap* tvs = g ? &tv1s : &tv0s;
-  const int ntiles = win_ktiles(f, p.P, W, dil);
+  const bool spans = (g ? p.span_mode[1] : p.span_mode[0]) != 0;
+  const int ntiles = win_ktiles(f, p.P, W, dil, spans);
   const bool has_b = p.pair == 2 && 2 * pr + 1 < p.n_qt;
   // A CTA with one query tile and at least two key tiles splits the key range instead: tile slot 0
   // takes key tiles [0, nA), slot 1 the rest for the same query rows, and the two partial softmax
@@ -264,7 +285,7 @@ __global__ void __launch_bounds__(384, 1)
       int uses[NSLOT] = {0, 0, 0, 0};
       // load (key tile kt, V or K) into `slot` as that slot's next use
       auto load = [&](int kt, bool is_v, int slot) {
-        const WinKTile t = win_ktile(kt, f, p.P, W, dil);
+        const WinKTile t = win_ktile(kt, f, p.P, W, dil, spans);
         const int krow = (b * kbf + t.fr_a % kmod) * p.P + t.off_a;
         const int use = uses[slot];
         if (use > 0 && !mbar_wait(&sm.empty[slot], (use - 1) & 1)) { *abort_flag = 1; return false; }
@@ -435,7 +456,7 @@ __global__ void __launch_bounds__(384, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = n_x > 0;
     for (int i = 0; ok && i < n_x; ++i) {
-      const int nv = win_ktile(kt0 + i, f, p.P, W, dil).nv;
+      const int nv = win_ktile(kt0 + i, f, p.P, W, dil, spans).nv;
       const bool got = !*abort_flag && mbar_wait(&sm.bar_s[x], i & 1);
       if (!__all_sync(0xffffffffu, got)) { *abort_flag = 1; ok = false; break; }
       tc_fence_after();
