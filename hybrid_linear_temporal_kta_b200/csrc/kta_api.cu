@@ -1174,12 +1174,25 @@ __global__ void __launch_bounds__(256) ring_put_kernel(const RingPutParams p) {
   const int rows = p.B * p.P;
   const int r0 = static_cast<int>(blockIdx.x) * kRingRows;
   const int n = min(kRingRows, rows - r0) * c.chunks;
-  for (int i = threadIdx.x; i < n; i += 256) {
-    const int rr = i / c.chunks, ch = i - rr * c.chunks;
-    const int r = r0 + rr, b = r / p.P, row = r - b * p.P;
-    const uint4 v = *reinterpret_cast<const uint4*>(c.src + b * c.src_seq +
-                                                    static_cast<long long>(row) * c.src_row + ch * 16);
-    *reinterpret_cast<uint4*>(c.dst + b * c.dst_seq + static_cast<long long>(row) * c.dst_row + ch * 16) = v;
+  // eight pieces per thread in flight at once: all loads, then all stores
+  for (int i0 = 0; i0 < n; i0 += 8 * 256) {
+    uint4 v[8];
+    long long dst[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * 256 + threadIdx.x;
+      dst[u] = -1;
+      if (i < n) {
+        const int rr = i / c.chunks, ch = i - rr * c.chunks;
+        const int r = r0 + rr, b = r / p.P, row = r - b * p.P;
+        v[u] = *reinterpret_cast<const uint4*>(c.src + b * c.src_seq +
+                                               static_cast<long long>(row) * c.src_row + ch * 16);
+        dst[u] = b * c.dst_seq + static_cast<long long>(row) * c.dst_row + ch * 16;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (dst[u] >= 0) *reinterpret_cast<uint4*>(c.dst + dst[u]) = v[u];
   }
 }
 
