@@ -295,7 +295,22 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
       ((s = make_map(&tk1s, g1.k, D, g1.k_heads, g1.k_rows, g1.k_ld, 8)) ||
        (s = make_map(&tv1s, g1.v, D, g1.k_heads, g1.k_rows, g1.k_ld, 8))))
     return s;
+  // output map (cols, heads, token of the frame, frame, sequence): a tile's rows past the frame
+  // end lie outside the token extent P, so TMA stores of whole 32-row boxes never write them
+  CUtensorMap to = tq;
+  const bool o_tma = reinterpret_cast<uintptr_t>(L.o) % 16 == 0 && L.o_ld % 8 == 0;
+  if (o_tma) {
+    const cuuint64_t dO[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Htot),
+                              static_cast<cuuint64_t>(L.P), static_cast<cuuint64_t>(L.Fq),
+                              static_cast<cuuint64_t>(L.B)};
+    const cuuint64_t sO[4] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L.o_ld) * 2,
+                              static_cast<cuuint64_t>(L.P) * L.o_ld * 2,
+                              static_cast<cuuint64_t>(L.q_rows_b) * L.o_ld * 2};
+    const cuuint32_t bO[5] = {64, 1, 32, 1, 1};
+    if ((s = make_map_nd(&to, L.o, 5, dO, sO, bO))) return s;
+  }
   WinParams p{};
+  p.o_tma = o_tma ? 1 : 0;
   p.B = L.B;
   p.P = L.P;
   p.Fq = L.Fq;
@@ -332,10 +347,10 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
     TraceScope ts("win_attn_tc", st);
     if (L.lse)
       kta::win_attn_tc_kernel<D, true><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
-          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, p);
+          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, to, p);
     else
       kta::win_attn_tc_kernel<D, false><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
-          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, p);
+          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, to, p);
   }
   const cudaError_t le = cudaGetLastError();
   if (le != cudaSuccess) {

@@ -60,6 +60,7 @@ struct WinParams {
   float scale_log2; // softmax scale * log2(e)
   __nv_bfloat16* o; // output, already offset to the launch's first head
   long long o_ld;   // output row stride in elements
+  int o_tma;        // 1: rows leave through the tile's Q buffer and TMA stores (map `to`)
   float* lse;       // optional [B][Htot][q_rows_b]: m + log2(l), the base-2 log-sum-exp of
                     // scale * log2(e) * S over each row's visible keys (null = not written)
 };
@@ -197,7 +198,8 @@ __global__ void __launch_bounds__(384, 1)
                        const __grid_constant__ CUtensorMap tk0s,
                        const __grid_constant__ CUtensorMap tv0s,
                        const __grid_constant__ CUtensorMap tk1s,
-                       const __grid_constant__ CUtensorMap tv1s, const WinParams p) {
+                       const __grid_constant__ CUtensorMap tv1s,
+                       const __grid_constant__ CUtensorMap to, const WinParams p) {
   static_assert(D == 64 || D == 128, "head dim");
   extern __shared__ uint8_t smem_raw[];
   WinSmem<D>& sm = *reinterpret_cast<WinSmem<D>*>(
@@ -623,14 +625,35 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * inv);
           }
-          if (row < nq) {
-            uint32_t w[16];
+          uint32_t w[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]), __uint_as_float(rr[2 * j + 1]));
+          for (int j = 0; j < 16; ++j)
+            w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]), __uint_as_float(rr[2 * j + 1]));
+          if (p.o_tma) {
+            // the row's 16-byte pieces go to the tile's Q buffer (free: its last reader, S_x,
+            // completed before bar_o[x]) in the 128-byte swizzled layout of the output map
+            uint8_t* srow = sm.q[x] + (c >> 1) * BOX + row * 128;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<uint4*>(srow + ((((c & 1) * 4 + j) ^ (row & 7)) << 4)) =
+                  make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          } else if (row < nq) {
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
             for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          }
+        }
+        if (p.o_tma) {
+          // each warp stores its 32 rows (one box per 64 columns); rows past the frame fall
+          // outside the map's token extent P and are not written
+          fence_proxy_async_smem();
+          __syncwarp();
+          const int trow = (p.pair * pr + x) * 128 + quad * 32;
+          if (lane == 0 && trow < p.P) {
+            for (int cb = 0; cb < NBOX; ++cb)
+              tma_store_5d(&to, sm.q[x] + cb * BOX + quad * 32 * 128, cb * 64, h, trow, f_local, b);
+            bulk_commit();
+            bulk_wait_read_all();
           }
         }
       }
