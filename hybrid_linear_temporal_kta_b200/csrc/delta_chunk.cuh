@@ -287,13 +287,32 @@ __global__ void __launch_bounds__(128, 3) delta_prep_kernel(const DeltaParams p)
       const int t = idx / (C / 8), c = (idx % (C / 8)) * 8;
       *reinterpret_cast<uint4*>(&A[t * C + c]) = *reinterpret_cast<const uint4*>(&sm.aq[t * LDC + c]);
     }
+    // U'^T: transposed 8 x 8 blocks of U' (ldmatrix.trans) into a [D][C] tile over the free q / T
+    // region, its 16-byte pieces XOR-swizzled by row so that both the pair stores and the row
+    // reads are conflict-free, then whole rows to the workspace
+    static_assert(D * C * 2 <= sizeof(sm.q), "transpose tile");
+    uint8_t* ut = reinterpret_cast<uint8_t*>(sm.q);
+#pragma unroll
+    for (int tb = 2 * warp; tb < 2 * warp + 2; ++tb) {
+#pragma unroll
+      for (int jb = 0; jb < D / 32; ++jb) {
+        // matrix m = lane / 8 covers tokens 8 tb .. +7 and value columns 32 jb + 8 m .. +7; this
+        // lane receives tokens 8 tb + 2 (lane % 4), +1 of value column 32 jb + 8 m + lane / 4
+        uint32_t r[4];
+        ldsm_x4_t(r, &sm.v[(8 * tb + (lane & 7)) * LDK + 32 * jb + 8 * (lane >> 3)]);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int j = 32 * jb + 8 * m + (lane >> 2);
+          *reinterpret_cast<uint32_t*>(ut + j * (C * 2) + ((tb ^ (j & 7)) << 4) + 4 * (lane & 3)) = r[m];
+        }
+      }
+    }
+    __syncthreads();
     __nv_bfloat16* U = p.ws_U + wsi * D * C;
-    for (int idx = tid; idx < D * (C / 2); idx += 128) {
-      const int j = idx / (C / 2), t = (idx % (C / 2)) * 2;
-      __nv_bfloat162 pr;
-      pr.x = sm.v[t * LDK + j];
-      pr.y = sm.v[(t + 1) * LDK + j];
-      *reinterpret_cast<__nv_bfloat162*>(&U[j * C + t]) = pr;
+    for (int idx = tid; idx < D * (C / 8); idx += 128) {
+      const int j = idx / (C / 8), c = idx % (C / 8);
+      *reinterpret_cast<uint4*>(&U[j * C + c * 8]) =
+          *reinterpret_cast<const uint4*>(ut + j * (C * 2) + ((c ^ (j & 7)) << 4));
     }
     if (tid < C) p.ws_g[wsi * C + tid] = sm.lg[tid];
   }
