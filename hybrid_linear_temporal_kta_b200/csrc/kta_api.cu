@@ -340,17 +340,15 @@ kta_status launch_win_tc(const WinLaunch& L, cudaStream_t st) {
   if (nblk <= 0) return KTA_OK;
   if (nblk > 0x7fffffffLL) return fail(KTA_ERR_UNSUPPORTED, "too many tiles (%lld)", nblk);
   const size_t smem = kta::win_smem_bytes<D>();
-  if ((s = set_smem_attr(kta::win_attn_tc_kernel<D, false>, smem)) ||
-      (s = set_smem_attr(kta::win_attn_tc_kernel<D, true>, smem)))
-    return s;
+  // frames shorter than 120 keys (P a multiple of 8): a packed key tile may cross several frames
+  const bool mf = pk && L.P < 120;
+  auto kern = L.lse ? (mf ? kta::win_attn_tc_kernel<D, true, true> : kta::win_attn_tc_kernel<D, true, false>)
+                    : (mf ? kta::win_attn_tc_kernel<D, false, true> : kta::win_attn_tc_kernel<D, false, false>);
+  if ((s = set_smem_attr(kern, smem))) return s;
   {
     TraceScope ts("win_attn_tc", st);
-    if (L.lse)
-      kta::win_attn_tc_kernel<D, true><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
-          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, to, p);
-    else
-      kta::win_attn_tc_kernel<D, false><<<static_cast<unsigned>(nblk), 384, smem, st>>>(
-          tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s, tv1s, to, p);
+    kern<<<static_cast<unsigned>(nblk), 384, smem, st>>>(tq, tk0, tv0, tk1, tv1, tk0s, tv0s, tk1s,
+                                                         tv1s, to, p);
   }
   const cudaError_t le = cudaGetLastError();
   if (le != cudaSuccess) {

@@ -116,7 +116,9 @@ __device__ __forceinline__ void win_tile(int i, int f, int P, int W, int dil, in
 // packed: they form one sequence of nsp * P keys cut into 128-key tiles, so only the window's last
 // tile is ragged (per-frame tiles would leave a ragged tile in every frame). A packed tile takes
 // rows_a rows (a multiple of 8) from frame fr_a at row off_a and the rest from the first rows of
-// frame fr_b; nv keys of it are visible. Otherwise the tiles are win_tile's.
+// frame fr_b, when that rest fits in one frame (always for P >= 120; shorter frames may need
+// several, which the kernel's MF form loads box by box); nv keys of it are visible. Otherwise the
+// tiles are win_tile's.
 struct WinKTile {
   int fr_a, off_a, rows_a, fr_b, nv;
 };
@@ -187,8 +189,10 @@ constexpr size_t win_smem_bytes() {
 }
 
 // LSE: also store each row's base-2 log-sum-exp to p.lse (a separate instantiation, so that the
-// plain forward's code is unchanged).
-template <int D, bool LSE = false>
+// plain forward's code is unchanged). MF: frames shorter than 120 keys with P a multiple of 8, so
+// that a packed key tile may cross several frame boundaries (also a separate instantiation: the
+// extra loader path, inlined or called, slowed the hot loops of the common form by 2-4 %).
+template <int D, bool LSE = false, bool MF = false>
 __global__ void __launch_bounds__(384, 1)
     win_attn_tc_kernel(const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk0,
@@ -296,6 +300,31 @@ __global__ void __launch_bounds__(384, 1)
           const CUtensorMap* tm = is_v ? tv : tk;
           for (int c = 0; c < NBOX; ++c)
             tma_load_3d(sm.kv[slot] + c * BOX, tm, &sm.full[slot], c * 64, hk, krow);
+        } else if (MF) {
+          // a tile across one or more frame boundaries, in 8-row boxes (one 128-byte swizzle atom
+          // each; P is a multiple of 8, so a box never straddles a frame). The boxes step through
+          // the window's keys from row off_a of frame fr_a and move to the next visible frame,
+          // dil frames on, at each frame's end; boxes past the window's last key repeat its final
+          // rows (finite data, masked by nv).
+          const CUtensorMap* tm = is_v ? tvs : tks;
+          const int nsp = min(W, f / dil + 1);
+          int jj = (128 * kt) / p.P, row = t.off_a, fslot = t.fr_a % kmod;
+          for (int r = 0; r < 128; r += 8) {
+            const int src = (b * kbf + fslot) * p.P + row;
+            for (int c = 0; c < NBOX; ++c)
+              tma_load_3d(sm.kv[slot] + c * BOX + r * 128, tm, &sm.full[slot], c * 64, hk, src);
+            row += 8;
+            if (row == p.P) {
+              if (jj + 1 < nsp) {
+                ++jj;
+                row = 0;
+                fslot += dil;
+                while (fslot >= kmod) fslot -= kmod;
+              } else {
+                row = p.P - 8;
+              }
+            }
+          }
         } else {
           // a tile across two frames, in 8-row boxes (one 128-byte swizzle atom each)
           const CUtensorMap* tm = is_v ? tvs : tks;

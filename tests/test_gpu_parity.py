@@ -107,6 +107,11 @@ SOFTMAX_CASES = [
     (128, 1, 4, 33, 20, 1),   # W >= F: full frame-causal attention
     (64, 1, 7, 300, 1, 1),    # own frame only
     (128, 1, 13, 96, 3, 5),   # dilation larger than the window
+    # frames shorter than a key tile: a packed dilated window puts many frames in one tile
+    (128, 1, 12, 8, 4, 2),
+    (64, 2, 10, 16, 5, 2),
+    (128, 1, 30, 104, 8, 2),  # some packed tiles cross three frames
+    (128, 1, 6, 1, 3, 2),     # one-token frames (not packed: P is not a multiple of 8)
 ]
 
 
@@ -413,6 +418,32 @@ def test_stream_rollout_matches_full_forward(kta, dtype):
                            n_gla=2, W_swa=w.W_swa, W_dswa=w.W_dswa, dil=w.dil,
                            scale_softmax=w.scale_softmax)
     assert_heads_close(roll, ref, range(w.H), tol, what="stream vs oracle")
+    st.close()
+
+
+@pytest.mark.parametrize("P", [16, 40, 104])
+def test_stream_short_frames_match_full_forward(kta, P):
+    """Frames shorter than a key tile: the streamed SWA window is a ring of W slots, so its packed
+    tiles (and the dilated window's) span several frames. Softmax heads equal the full forward bit
+    for bit; every head is within the bf16 bound of the oracle."""
+    w = synth.STREAM_BF16.replace(F=14, P=P, n_swa=2, n_dswa=2, n_gla=2, W_swa=5, W_dswa=4, dil=2)
+    x = synth.make_inputs(w, B=2)
+    cfg = kta.cfg_from_workload(w, B=2)
+    q, k, v, a = dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["alpha"])
+    full = kta.hybrid_fwd(cfg, q, k, v, a)
+    st = kta.Stream(cfg)
+    outs = []
+    for f in range(w.F):
+        sl = slice(f * w.P, (f + 1) * w.P)
+        outs.append(st.step(q[:, sl].contiguous(), k[:, sl].contiguous(), v[:, sl].contiguous(),
+                            a[:, sl].contiguous()))
+    kta.device_status()
+    roll = torch.cat(outs, dim=1)
+    assert torch.equal(roll[:, :, :4], full[:, :, :4])
+    ref, _ = oracle.hybrid(x["q"], x["k"], x["v"], x["alpha"], None, P=w.P, n_swa=2, n_dswa=2,
+                           n_gla=2, W_swa=w.W_swa, W_dswa=w.W_dswa, dil=w.dil,
+                           scale_softmax=w.scale_softmax)
+    assert_heads_close(roll, ref, range(w.H), BF16_TOL, what=f"short-frame stream P={P}")
     st.close()
 
 
