@@ -140,9 +140,9 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
+def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+    current kernel sources and for this workload (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -150,6 +150,8 @@ def recorded_traffic(kernel: str):
         d = json.load(f)
     e = d.get(kernel)
     if not e or e.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    if e.get("config_workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -459,9 +461,9 @@ def run_kta(args):
     flops = softmax_flops(w)
     achieved = flops / t_launch / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = recorded_traffic("win_attn_tc")
+    traffic = recorded_traffic("win_attn_tc", w.name)
     # DRAM bytes of one GLA call (state pass + output pass) from the committed ncu summary
-    gla_parts = [recorded_traffic(k) for k in ("gla_tc_state", "gla_tc_out")]
+    gla_parts = [recorded_traffic(k, w.name) for k in ("gla_tc_state", "gla_tc_out")]
     gla_traffic = sum(gla_parts) if all(x is not None for x in gla_parts) else None
     t_gla = sum(v["ms"] for v in kern_gla.values()) / args.steps / 1e3
     launches = sum(v["launches"] for v in kern.values()) // args.steps * args.steps
