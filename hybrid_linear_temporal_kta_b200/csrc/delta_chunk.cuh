@@ -24,12 +24,13 @@
 //     Writes W [C][D], U'^T [D][C], Aq [C][C] (bf16) and the gates [C] (fp32) to a workspace.
 //   delta_scan_kernel (one CTA per (value block, sequence, head), chunks in order): a producer
 //     warp streams W, q, k, Aq, U'^T and the gates of the coming chunks into a ring of shared-
-//     memory stages with TMA (128-byte swizzle); each pair of consumer warps owns 16 value
+//     memory stages with TMA (128-byte swizzle); each pair of chain warps owns 16 value
 //     columns, each warp half of the key dims of their state rows S^T (16 x D/2, fp32, in
 //     registers), so the chunk-to-chunk chain stays in registers apart from one exchange of
 //     partial sums inside the pair:
-//       U^T = U'^T - S^T W^T,   S^T <- gamma_end S^T + (U^T diag(gamma_end / gamma)) K,
-//       o^T = (S_0^T q^T) diag(gamma) + U^T Aq^T   (S_0^T kept as bf16 fragments).
+//       U^T = U'^T - S^T W^T,   S^T <- gamma_end S^T + (U^T diag(gamma_end / gamma)) K;
+//     a pair of output warps per group takes S_0^T and U^T as bf16 fragments through shared
+//     memory and forms o^T = (S_0^T q^T) diag(gamma) + U^T Aq^T off that chain.
 #pragma once
 
 #include "kta_ptx.cuh"
@@ -332,9 +333,12 @@ template <int D, int VG, int NST>
 struct DeltaScanSmem {
   static constexpr int C = DELTA_C;
   static constexpr int VB = 16 * VG;      // value columns per CTA (VG groups of 16)
-  static constexpr int NCW = 2 * VG;      // consumer warps: two per group (key-dim halves)
+  static constexpr int NCW = 2 * VG;      // chain warps: two per group (key-dim halves)
+  static constexpr int NOW = 2 * VG;      // output warps: two per group (token halves)
   static constexpr int NBOX = D / 64;
-  static constexpr int XCH = C / 8 * 4 + C / 16 * 4;  // floats a lane hands its partner per chunk
+  static constexpr int NKH = D / 32;      // k steps over a key-dim half
+  static constexpr int NTP = C / 16;      // 16-token groups per chunk
+  static constexpr int XCH = C / 8 * 4;   // floats a chain lane hands its partner per chunk
   struct alignas(1024) Stage {
     __nv_bfloat16 w[NBOX * C * 64];
     __nv_bfloat16 q[NBOX * C * 64];
@@ -347,12 +351,18 @@ struct DeltaScanSmem {
       (3 * NBOX * C * 64 + C * 64 + VB * 64) * 2 + C * 4;  // bytes the TMA unit writes per stage
   Stage stage[NST];
   alignas(128) __nv_bfloat16 o[2][C * VB];  // output tiles [token][value column] for TMA stores
-  float xch[2][NCW][XCH][32];   // partial sums exchanged within a warp pair (by chunk parity)
+  float xch[2][NCW][XCH][32];   // partial sums of X exchanged within a chain pair (chunk parity)
+  // chain -> output warps, by chunk parity: S_0^T as bf16 A fragments (per group, key half and
+  // k step) and U^T as bf16 A fragments (per group and token group), one uint4 per lane
+  uint4 hs[2][VG][2][NKH][32];
+  uint4 hu[2][VG][NTP][32];
   int pair_ok[2][NCW];
   uint64_t full[NST];
   uint64_t empty[NST];
-  uint64_t ofull[2];            // consumers -> producer: output tile written
-  uint64_t ofree[2];            // producer -> consumers: output tile read by the TMA store
+  uint64_t hfull[2];            // chain -> output warps: the chunk's S_0^T and U^T are written
+  uint64_t hfree[2];            // output -> chain warps: read into registers
+  uint64_t ofull[2];            // output warps -> producer: output tile written
+  uint64_t ofree[2];            // producer -> output warps: output tile read by the TMA store
 };
 
 template <int D, int VG, int NST>
@@ -360,22 +370,24 @@ constexpr size_t delta_scan_smem_bytes() {
   return sizeof(DeltaScanSmem<D, VG, NST>) + 1024;  // + manual 1024-byte alignment
 }
 
-// Consumer warp 2g + hk owns value columns [16g, 16g+16) of the CTA's block and key dims
-// [hk D/2, (hk+1) D/2) of their state rows S^T. Per chunk the pair forms the key-dim partial
-// sums of X = S^T W^T and of S^T q^T, swaps them through shared memory (one pair barrier), and
-// then each warp updates its own key-dim half of S^T and finishes the outputs of its own half of
-// the chunk's tokens. The producer warp loads the stages and stores the output tiles (TMA).
+// Chain warp 2g + hk owns value columns [16g, 16g+16) of the CTA's block and key dims
+// [hk D/2, (hk+1) D/2) of their state rows S^T. Per chunk the pair forms the key-dim partial sums
+// of X = S^T W^T, swaps them through shared memory (one pair barrier), then each warp updates its
+// own key-dim half of S^T. Output warp 2g + ho of the same group takes the chunk's S_0^T and U^T
+// fragments from the chain pair through shared memory and forms the outputs of tokens
+// [ho C/2, (ho+1) C/2): (S_0^T q^T) diag(gamma) + U^T Aq^T, off the chunk-to-chunk chain. The
+// producer warp loads the stages and stores the output tiles (TMA).
 template <int D, int VG, int NST>
-__global__ void __launch_bounds__((2 * VG + 1) * 32, 1)
+__global__ void __launch_bounds__((4 * VG + 1) * 32, 1)
     delta_scan_kernel(const __grid_constant__ CUtensorMap tW, const __grid_constant__ CUtensorMap tQ,
                       const __grid_constant__ CUtensorMap tK, const __grid_constant__ CUtensorMap tA,
                       const __grid_constant__ CUtensorMap tU, const __grid_constant__ CUtensorMap tO,
                       const DeltaParams p) {
   using SM = DeltaScanSmem<D, VG, NST>;
-  constexpr int C = SM::C, VB = SM::VB, NCW = SM::NCW, NBOX = SM::NBOX;
-  constexpr int DH = D / 2;               // key dims per warp
-  constexpr int NKH = DH / 16;            // k steps over a key-dim half
-  constexpr int NTP = C / 16;             // 16-token groups per chunk
+  constexpr int C = SM::C, VB = SM::VB, NCW = SM::NCW, NOW = SM::NOW, NBOX = SM::NBOX;
+  constexpr int DH = D / 2;               // key dims per chain warp
+  constexpr int NKH = SM::NKH;            // k steps over a key-dim half
+  constexpr int NTP = SM::NTP;            // 16-token groups per chunk
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SM& sm = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -387,17 +399,19 @@ __global__ void __launch_bounds__((2 * VG + 1) * 32, 1)
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], NCW);
+      mbar_init(&sm.empty[s], NCW + NOW);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.ofull[i], NCW);
+      mbar_init(&sm.hfull[i], NCW);
+      mbar_init(&sm.hfree[i], NOW);
+      mbar_init(&sm.ofull[i], NOW);
       mbar_init(&sm.ofree[i], 1);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == NCW) {
+  if (warp == NCW + NOW) {
     // ---- producer: one lane loads the stages and stores the output tiles
     if (lane == 0) {
       prefetch_tmap(&tW);
@@ -441,160 +455,220 @@ __global__ void __launch_bounds__((2 * VG + 1) * 32, 1)
     return;
   }
 
-  // ---- consumers
-  const int grp = warp >> 1, hk = warp & 1, mate = warp ^ 1;
-  const int vr = 16 * grp + g4;           // this lane's value rows vr, vr + 8 (within the block)
-  const int jv = j0 + vr;
-  const int kb = hk * DH;                 // first key dim of this warp's half
-  const long long sb = static_cast<long long>(bh) * D * D;
-  // st[nt][r] = S^T[jv (+8 for r >= 2)][kb + 8 nt + 2 t4 + (r & 1)]
-  float st[DH / 8][4];
-#pragma unroll
-  for (int nt = 0; nt < DH / 8; ++nt)
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-      st[nt][r] = p.S0 ? p.S0[sb + (kb + nt * 8 + 2 * t4 + (r & 1)) * D + jv + (r >= 2 ? 8 : 0)] : 0.f;
-
   // lane row / column offsets of the ldmatrix address patterns
   const int nm_r = (lane & 7) + (lane >> 4) * 8, nm_c = ((lane >> 3) & 1) * 8;  // B stored [n][k]
   const int km_r = (lane & 7) + ((lane >> 3) & 1) * 8, km_c = (lane >> 4) * 8;  // B stored [k][n]
 
-  bool failed = false;
-  int c = 0;
-  for (; c < p.nch; ++c) {
-    const int s = c % NST;
-    const bool ok = !failed && mbar_wait(&sm.full[s], (c / NST) & 1);
-    float (*mine)[32] = sm.xch[c & 1][warp];
-    float (*theirs)[32] = sm.xch[c & 1][mate];
-    float xw[C / 8][4], ov[C / 8][4];
-    uint32_t sa[NKH][4];
-    const typename SM::Stage& S = sm.stage[s];
-    const uint8_t* Wb = reinterpret_cast<const uint8_t*>(S.w);
-    const uint8_t* Qb = reinterpret_cast<const uint8_t*>(S.q);
-    const uint8_t* Kb = reinterpret_cast<const uint8_t*>(S.k);
-    const uint8_t* Ab = reinterpret_cast<const uint8_t*>(S.aq);
-    const uint8_t* Ub = reinterpret_cast<const uint8_t*>(S.ut);
-    if (ok) {
-      // (a) this warp's half of S^T as bf16 A fragments (k = key dim)
-#pragma unroll
-      for (int kk = 0; kk < NKH; ++kk) {
-        sa[kk][0] = bf16x2(st[2 * kk][0], st[2 * kk][1]);
-        sa[kk][1] = bf16x2(st[2 * kk][2], st[2 * kk][3]);
-        sa[kk][2] = bf16x2(st[2 * kk + 1][0], st[2 * kk + 1][1]);
-        sa[kk][3] = bf16x2(st[2 * kk + 1][2], st[2 * kk + 1][3]);
-      }
-      // (b) key-dim partial sums of X = S^T W^T and of S^T q^T (n = token); the B fragments
-      // of the next k step are loaded while the current one's products issue
-#pragma unroll
-      for (int nt = 0; nt < C / 8; ++nt)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) xw[nt][r] = ov[nt][r] = 0.f;
-      {
-        uint32_t fw[2][NTP][4], fq[2][NTP][4];
-#pragma unroll
-        for (int np = 0; np < NTP; ++np) {
-          ldsm_x4(fw[0][np], Wb + swz<C>(np * 16 + nm_r, kb + nm_c));
-          ldsm_x4(fq[0][np], Qb + swz<C>(np * 16 + nm_r, kb + nm_c));
-        }
-#pragma unroll
-        for (int kk = 0; kk < NKH; ++kk) {
-          const int cur = kk & 1;
-          if (kk + 1 < NKH) {
-#pragma unroll
-            for (int np = 0; np < NTP; ++np) {
-              ldsm_x4(fw[cur ^ 1][np], Wb + swz<C>(np * 16 + nm_r, kb + (kk + 1) * 16 + nm_c));
-              ldsm_x4(fq[cur ^ 1][np], Qb + swz<C>(np * 16 + nm_r, kb + (kk + 1) * 16 + nm_c));
-            }
-          }
-#pragma unroll
-          for (int np = 0; np < NTP; ++np) {
-            mma16816(xw[2 * np], sa[kk], fw[cur][np][0], fw[cur][np][1]);
-            mma16816(xw[2 * np + 1], sa[kk], fw[cur][np][2], fw[cur][np][3]);
-            mma16816(ov[2 * np], sa[kk], fq[cur][np][0], fq[cur][np][1]);
-            mma16816(ov[2 * np + 1], sa[kk], fq[cur][np][2], fq[cur][np][3]);
-          }
-        }
-      }
-      // hand the partner its sums: all of X, and S^T q^T for the partner's half of the tokens
-#pragma unroll
-      for (int nt = 0; nt < C / 8; ++nt)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) mine[nt * 4 + r][lane] = xw[nt][r];
-#pragma unroll
-      for (int nt = 0; nt < C / 8; ++nt)
-        if (nt / (C / 16) != hk) {
-#pragma unroll
-          for (int r = 0; r < 4; ++r) mine[C / 2 + (nt % (C / 16)) * 4 + r][lane] = ov[nt][r];
-        }
-    }
-    if (lane == 0) sm.pair_ok[c & 1][warp] = ok ? 1 : 0;
-    named_bar_sync(2 + grp, 64);
-    if (!ok || !sm.pair_ok[c & 1][mate]) break;  // the same decision in both warps of the pair
-
-    // (c) U^T = U'^T - X  (value rows vr (+8), token columns)
-#pragma unroll
-    for (int nt = 0; nt < C / 8; ++nt) {
-      const int tc = nt * 8 + 2 * t4;
-      const float2 ua = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Ub + swz<VB>(vr, tc)));
-      const float2 ub = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Ub + swz<VB>(vr + 8, tc)));
-      xw[nt][0] = ua.x - (xw[nt][0] + theirs[nt * 4 + 0][lane]);
-      xw[nt][1] = ua.y - (xw[nt][1] + theirs[nt * 4 + 1][lane]);
-      xw[nt][2] = ub.x - (xw[nt][2] + theirs[nt * 4 + 2][lane]);
-      xw[nt][3] = ub.y - (xw[nt][3] + theirs[nt * 4 + 3][lane]);
-    }
-#pragma unroll
-    for (int nt = 0; nt < C / 8; ++nt)
-      if (nt / (C / 16) == hk) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) ov[nt][r] += theirs[C / 2 + (nt % (C / 16)) * 4 + r][lane];
-      }
-    // (d) U^T as A fragments (k = token): plain, and scaled by gamma_end / gamma_s
-    const float lgC = S.lg[C - 1];
-    uint32_t ua[NTP][4], ur[NTP][4];
-#pragma unroll
-    for (int kk = 0; kk < NTP; ++kk) {
-      const int ta = 16 * kk + 2 * t4, tb = ta + 8;
-      const float da0 = exp2f(lgC - S.lg[ta]), da1 = exp2f(lgC - S.lg[ta + 1]);
-      const float db0 = exp2f(lgC - S.lg[tb]), db1 = exp2f(lgC - S.lg[tb + 1]);
-      ua[kk][0] = bf16x2(xw[2 * kk][0], xw[2 * kk][1]);
-      ua[kk][1] = bf16x2(xw[2 * kk][2], xw[2 * kk][3]);
-      ua[kk][2] = bf16x2(xw[2 * kk + 1][0], xw[2 * kk + 1][1]);
-      ua[kk][3] = bf16x2(xw[2 * kk + 1][2], xw[2 * kk + 1][3]);
-      ur[kk][0] = bf16x2(xw[2 * kk][0] * da0, xw[2 * kk][1] * da1);
-      ur[kk][1] = bf16x2(xw[2 * kk][2] * da0, xw[2 * kk][3] * da1);
-      ur[kk][2] = bf16x2(xw[2 * kk + 1][0] * db0, xw[2 * kk + 1][1] * db1);
-      ur[kk][3] = bf16x2(xw[2 * kk + 1][2] * db0, xw[2 * kk + 1][3] * db1);
-    }
-    // (e) this warp's key dims of S^T = gamma_end S^T + Ur^T K  (n = key dim)
-    const float gC = exp2f(lgC);
+  if (warp < NCW) {
+    // ---- chain warps
+    const int grp = warp >> 1, hk = warp & 1, mate = warp ^ 1;
+    const int vr = 16 * grp + g4;           // this lane's value rows vr, vr + 8 (within the block)
+    const int jv = j0 + vr;
+    const int kb = hk * DH;                 // first key dim of this warp's half
+    const long long sb = static_cast<long long>(bh) * D * D;
+    // st[nt][r] = S^T[jv (+8 for r >= 2)][kb + 8 nt + 2 t4 + (r & 1)]
+    float st[DH / 8][4];
 #pragma unroll
     for (int nt = 0; nt < DH / 8; ++nt)
 #pragma unroll
-      for (int r = 0; r < 4; ++r) st[nt][r] *= gC;
-    {
-      uint32_t fk[2][NKH][4];
+      for (int r = 0; r < 4; ++r)
+        st[nt][r] = p.S0 ? p.S0[sb + (kb + nt * 8 + 2 * t4 + (r & 1)) * D + jv + (r >= 2 ? 8 : 0)] : 0.f;
+
+    bool failed = false;
+    int c = 0;
+    for (; c < p.nch; ++c) {
+      const int s = c % NST, hb = c & 1;
+      // the stage has landed, and the output warps have read the hand-over buffer of two chunks ago
+      const bool ok = !failed && mbar_wait(&sm.full[s], (c / NST) & 1) &&
+                      (c < 2 || mbar_wait(&sm.hfree[hb], ((c - 2) >> 1) & 1));
+      float (*mine)[32] = sm.xch[hb][warp];
+      float (*theirs)[32] = sm.xch[hb][mate];
+      float xw[C / 8][4];
+      const typename SM::Stage& S = sm.stage[s];
+      const uint8_t* Wb = reinterpret_cast<const uint8_t*>(S.w);
+      const uint8_t* Kb = reinterpret_cast<const uint8_t*>(S.k);
+      const uint8_t* Ub = reinterpret_cast<const uint8_t*>(S.ut);
+      if (ok) {
+        // (a) this warp's half of S^T (the chunk's start state) as bf16 A fragments (k = key
+        // dim), also handed to the output warps
+        uint32_t sa[NKH][4];
 #pragma unroll
-      for (int np = 0; np < NKH; ++np) ldsm_x4_t(fk[0][np], Kb + swz<C>(km_r, kb + np * 16 + km_c));
+        for (int kk = 0; kk < NKH; ++kk) {
+          sa[kk][0] = bf16x2(st[2 * kk][0], st[2 * kk][1]);
+          sa[kk][1] = bf16x2(st[2 * kk][2], st[2 * kk][3]);
+          sa[kk][2] = bf16x2(st[2 * kk + 1][0], st[2 * kk + 1][1]);
+          sa[kk][3] = bf16x2(st[2 * kk + 1][2], st[2 * kk + 1][3]);
+          sm.hs[hb][grp][hk][kk][lane] = make_uint4(sa[kk][0], sa[kk][1], sa[kk][2], sa[kk][3]);
+        }
+        // (b) key-dim partial sums of X = S^T W^T (n = token); the B fragments of the next k step
+        // are loaded while the current one's products issue
+#pragma unroll
+        for (int nt = 0; nt < C / 8; ++nt)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) xw[nt][r] = 0.f;
+        {
+          uint32_t fw[2][NTP][4];
+#pragma unroll
+          for (int np = 0; np < NTP; ++np) ldsm_x4(fw[0][np], Wb + swz<C>(np * 16 + nm_r, kb + nm_c));
+#pragma unroll
+          for (int kk = 0; kk < NKH; ++kk) {
+            const int cur = kk & 1;
+            if (kk + 1 < NKH) {
+#pragma unroll
+              for (int np = 0; np < NTP; ++np)
+                ldsm_x4(fw[cur ^ 1][np], Wb + swz<C>(np * 16 + nm_r, kb + (kk + 1) * 16 + nm_c));
+            }
+#pragma unroll
+            for (int np = 0; np < NTP; ++np) {
+              mma16816(xw[2 * np], sa[kk], fw[cur][np][0], fw[cur][np][1]);
+              mma16816(xw[2 * np + 1], sa[kk], fw[cur][np][2], fw[cur][np][3]);
+            }
+          }
+        }
+        // hand the partner this warp's sums of X
+#pragma unroll
+        for (int nt = 0; nt < C / 8; ++nt)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) mine[nt * 4 + r][lane] = xw[nt][r];
+      }
+      if (lane == 0) sm.pair_ok[hb][warp] = ok ? 1 : 0;
+      named_bar_sync(2 + grp, 64);
+      if (!ok || !sm.pair_ok[hb][mate]) break;  // the same decision in both warps of the pair
+
+      // (c) U^T = U'^T - X  (value rows vr (+8), token columns)
+#pragma unroll
+      for (int nt = 0; nt < C / 8; ++nt) {
+        const int tc = nt * 8 + 2 * t4;
+        const float2 ua = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Ub + swz<VB>(vr, tc)));
+        const float2 ub = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Ub + swz<VB>(vr + 8, tc)));
+        xw[nt][0] = ua.x - (xw[nt][0] + theirs[nt * 4 + 0][lane]);
+        xw[nt][1] = ua.y - (xw[nt][1] + theirs[nt * 4 + 1][lane]);
+        xw[nt][2] = ub.x - (xw[nt][2] + theirs[nt * 4 + 2][lane]);
+        xw[nt][3] = ub.y - (xw[nt][3] + theirs[nt * 4 + 3][lane]);
+      }
+      // (d) U^T as A fragments (k = token): plain (to the output warps, from one warp of the
+      // pair) and scaled by gamma_end / gamma_s (for the state update)
+      const float lgC = S.lg[C - 1];
+      uint32_t ur[NTP][4];
 #pragma unroll
       for (int kk = 0; kk < NTP; ++kk) {
-        const int cur = kk & 1;
-        if (kk + 1 < NTP) {
+        const int ta = 16 * kk + 2 * t4, tb = ta + 8;
+        const float da0 = exp2f(lgC - S.lg[ta]), da1 = exp2f(lgC - S.lg[ta + 1]);
+        const float db0 = exp2f(lgC - S.lg[tb]), db1 = exp2f(lgC - S.lg[tb + 1]);
+        if (hk == 0)
+          sm.hu[hb][grp][kk][lane] = make_uint4(bf16x2(xw[2 * kk][0], xw[2 * kk][1]),
+                                                bf16x2(xw[2 * kk][2], xw[2 * kk][3]),
+                                                bf16x2(xw[2 * kk + 1][0], xw[2 * kk + 1][1]),
+                                                bf16x2(xw[2 * kk + 1][2], xw[2 * kk + 1][3]));
+        ur[kk][0] = bf16x2(xw[2 * kk][0] * da0, xw[2 * kk][1] * da1);
+        ur[kk][1] = bf16x2(xw[2 * kk][2] * da0, xw[2 * kk][3] * da1);
+        ur[kk][2] = bf16x2(xw[2 * kk + 1][0] * db0, xw[2 * kk + 1][1] * db1);
+        ur[kk][3] = bf16x2(xw[2 * kk + 1][2] * db0, xw[2 * kk + 1][3] * db1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.hfull[hb]);
+      // (e) this warp's key dims of S^T = gamma_end S^T + Ur^T K  (n = key dim)
+      const float gC = exp2f(lgC);
 #pragma unroll
-          for (int np = 0; np < NKH; ++np)
-            ldsm_x4_t(fk[cur ^ 1][np], Kb + swz<C>((kk + 1) * 16 + km_r, kb + np * 16 + km_c));
+      for (int nt = 0; nt < DH / 8; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) st[nt][r] *= gC;
+      {
+        uint32_t fk[2][NKH][4];
+#pragma unroll
+        for (int np = 0; np < NKH; ++np) ldsm_x4_t(fk[0][np], Kb + swz<C>(km_r, kb + np * 16 + km_c));
+#pragma unroll
+        for (int kk = 0; kk < NTP; ++kk) {
+          const int cur = kk & 1;
+          if (kk + 1 < NTP) {
+#pragma unroll
+            for (int np = 0; np < NKH; ++np)
+              ldsm_x4_t(fk[cur ^ 1][np], Kb + swz<C>((kk + 1) * 16 + km_r, kb + np * 16 + km_c));
+          }
+#pragma unroll
+          for (int np = 0; np < NKH; ++np) {
+            mma16816(st[2 * np], ur[kk], fk[cur][np][0], fk[cur][np][1]);
+            mma16816(st[2 * np + 1], ur[kk], fk[cur][np][2], fk[cur][np][3]);
+          }
+        }
+      }
+      // every read of the stage by this warp is done
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+    }
+    if (p.S_out && c == p.nch) {
+#pragma unroll
+      for (int nt = 0; nt < DH / 8; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          p.S_out[sb + (kb + nt * 8 + 2 * t4 + (r & 1)) * D + jv + (r >= 2 ? 8 : 0)] = st[nt][r];
+    }
+    return;
+  }
+
+  // ---- output warps
+  const int ow = warp - NCW;
+  const int grp = ow >> 1, ho = ow & 1;
+  const int vr = 16 * grp + g4;
+  bool failed = false;
+  for (int c = 0; c < p.nch && !failed; ++c) {
+    const int s = c % NST, hb = c & 1;
+    if (!mbar_wait(&sm.full[s], (c / NST) & 1) || !mbar_wait(&sm.hfull[hb], (c >> 1) & 1)) break;
+    const typename SM::Stage& S = sm.stage[s];
+    const uint8_t* Qb = reinterpret_cast<const uint8_t*>(S.q);
+    const uint8_t* Ab = reinterpret_cast<const uint8_t*>(S.aq);
+    // the chunk's start state S_0^T (both key halves) and U^T, as A fragments
+    uint32_t sa[2 * NKH][4], ua[NTP][4];
+#pragma unroll
+    for (int kk = 0; kk < 2 * NKH; ++kk) {
+      const uint4 x = sm.hs[hb][grp][kk / NKH][kk % NKH][lane];
+      sa[kk][0] = x.x;
+      sa[kk][1] = x.y;
+      sa[kk][2] = x.z;
+      sa[kk][3] = x.w;
+    }
+#pragma unroll
+    for (int kk = 0; kk < NTP; ++kk) {
+      const uint4 x = sm.hu[hb][grp][kk][lane];
+      ua[kk][0] = x.x;
+      ua[kk][1] = x.y;
+      ua[kk][2] = x.z;
+      ua[kk][3] = x.w;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.hfree[hb]);
+    // (S_0^T q^T) for this warp's tokens [ho C/2, (ho+1) C/2) (n = token, k = key dim), the q
+    // fragments of the next k step loaded while the current one's products issue
+    constexpr int NPH = NTP / 2;            // 16-token groups per warp
+    float ov[2 * NPH][4];
+#pragma unroll
+    for (int nt = 0; nt < 2 * NPH; ++nt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) ov[nt][r] = 0.f;
+    {
+      uint32_t fq[2][NPH][4];
+#pragma unroll
+      for (int np = 0; np < NPH; ++np)
+        ldsm_x4(fq[0][np], Qb + swz<C>((ho * NPH + np) * 16 + nm_r, nm_c));
+#pragma unroll
+      for (int kk = 0; kk < 2 * NKH; ++kk) {
+        const int cur = kk & 1;
+        if (kk + 1 < 2 * NKH) {
+#pragma unroll
+          for (int np = 0; np < NPH; ++np)
+            ldsm_x4(fq[cur ^ 1][np], Qb + swz<C>((ho * NPH + np) * 16 + nm_r, (kk + 1) * 16 + nm_c));
         }
 #pragma unroll
-        for (int np = 0; np < NKH; ++np) {
-          mma16816(st[2 * np], ur[kk], fk[cur][np][0], fk[cur][np][1]);
-          mma16816(st[2 * np + 1], ur[kk], fk[cur][np][2], fk[cur][np][3]);
+        for (int np = 0; np < NPH; ++np) {
+          mma16816(ov[2 * np], sa[kk], fq[cur][np][0], fq[cur][np][1]);
+          mma16816(ov[2 * np + 1], sa[kk], fq[cur][np][2], fq[cur][np][3]);
         }
       }
     }
-    // (f) outputs of tokens [hk C/2, (hk+1) C/2): (S_0^T q^T) diag(gamma) + U^T Aq^T
+    // scale by gamma_t, then add U^T Aq^T (causal: token groups kk <= np)
 #pragma unroll
-    for (int nt = 0; nt < C / 8; ++nt) {
-      if (nt / (C / 16) != hk) continue;
-      const int tc = nt * 8 + 2 * t4;
+    for (int nt = 0; nt < 2 * NPH; ++nt) {
+      const int tc = (ho * NPH) * 16 + nt * 8 + 2 * t4;
       const float g0 = exp2f(S.lg[tc]), g1 = exp2f(S.lg[tc + 1]);
       ov[nt][0] *= g0;
       ov[nt][1] *= g1;
@@ -602,8 +676,8 @@ __global__ void __launch_bounds__((2 * VG + 1) * 32, 1)
       ov[nt][3] *= g1;
     }
 #pragma unroll
-    for (int np = 0; np < NTP; ++np) {
-      if (np / (NTP / 2) != hk) continue;
+    for (int npl = 0; npl < NPH; ++npl) {
+      const int np = ho * NPH + npl;
       uint32_t fa[NTP][4];
 #pragma unroll
       for (int kk = 0; kk < NTP; ++kk)
@@ -611,24 +685,23 @@ __global__ void __launch_bounds__((2 * VG + 1) * 32, 1)
 #pragma unroll
       for (int kk = 0; kk < NTP; ++kk) {
         if (kk > np) break;
-        mma16816(ov[2 * np], ua[kk], fa[kk][0], fa[kk][1]);
-        mma16816(ov[2 * np + 1], ua[kk], fa[kk][2], fa[kk][3]);
+        mma16816(ov[2 * npl], ua[kk], fa[kk][0], fa[kk][1]);
+        mma16816(ov[2 * npl + 1], ua[kk], fa[kk][2], fa[kk][3]);
       }
     }
-    // every read of the stage is done: hand it back to the producer
+    // every read of the stage by this warp is done
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[s]);
-    // (g) output tile [token][value column]: wait until the store of two chunks ago has read it
+    // output tile [token][value column]: wait until the store of two chunks ago has read it
     const int obi = c & 1;
     if (c >= 2 && !mbar_wait(&sm.ofree[obi], ((c - 2) >> 1) & 1)) {
-      failed = true;  // leaves at the next pair barrier
-      continue;
+      failed = true;
+      break;
     }
     __nv_bfloat16* ob = sm.o[obi];
 #pragma unroll
-    for (int nt = 0; nt < C / 8; ++nt) {
-      if (nt / (C / 16) != hk) continue;
-      const int tc = nt * 8 + 2 * t4;
+    for (int nt = 0; nt < 2 * NPH; ++nt) {
+      const int tc = (ho * NPH) * 16 + nt * 8 + 2 * t4;
       ob[tc * VB + vr] = __float2bfloat16_rn(ov[nt][0] * p.scale);
       ob[(tc + 1) * VB + vr] = __float2bfloat16_rn(ov[nt][1] * p.scale);
       ob[tc * VB + vr + 8] = __float2bfloat16_rn(ov[nt][2] * p.scale);
@@ -637,13 +710,6 @@ __global__ void __launch_bounds__((2 * VG + 1) * 32, 1)
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.ofull[obi]);
-  }
-  if (p.S_out && c == p.nch) {
-#pragma unroll
-    for (int nt = 0; nt < DH / 8; ++nt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-        p.S_out[sb + (kb + nt * 8 + 2 * t4 + (r & 1)) * D + jv + (r >= 2 ? 8 : 0)] = st[nt][r];
   }
 }
 

@@ -691,7 +691,7 @@ kta_status launch_delta_chunk(const LinLaunch& L, cudaStream_t st) {
   {
     TraceScope ts("delta_scan", st);
     kta::delta_scan_kernel<D, VG, NST>
-        <<<dim3(D / SS::VB, static_cast<unsigned>(BH)), (SS::NCW + 1) * 32, smem_s, st>>>(
+        <<<dim3(D / SS::VB, static_cast<unsigned>(BH)), (SS::NCW + SS::NOW + 1) * 32, smem_s, st>>>(
             tW, tQ, tK, tA, tU, tO, p);
   }
   KTA_CUDA(cudaGetLastError());
