@@ -36,6 +36,8 @@ def bf16(rng, shape):
     (64, 7, 130, 3, 2, (0, 2), 2),      # DSWA, 2-row tail tile
     (128, 4, 96, 8, 1, (0, 1), 1),      # one partial tile per frame, window past the start
     (128, 9, 256, 2, 3, (2, 4), 4),     # DSWA, whole tiles
+    (128, 12, 16, 4, 2, (0, 2), 2),     # frames shorter than a tile: the forward packs several
+    (64, 10, 8, 3, 1, (1, 2), 2),       # frames into one key tile
 ])
 def test_bf16_backward_matches_oracle(kta, d, F, P, W, dil, heads, Htot):
     rng = np.random.default_rng(d + F + P + W)

@@ -190,7 +190,10 @@ def test_bf16_dswa_equals_swa_on_page_reshape(kta):
                                            (64, 64, 64, 1, 2),
                                            # 40 sequence-heads: three segments, folded by the
                                            # output pass itself (no carry launch)
-                                           (128, 64, 700, 2, 20)])
+                                           (128, 64, 700, 2, 20),
+                                           # one token; one chunk and one token; a partial chunk
+                                           (128, 64, 1, 1, 2), (128, 64, 65, 2, 1),
+                                           (64, 32, 33, 1, 2), (128, 16, 15, 1, 1)])
 def test_bf16_gla_matches_oracle(kta, d, chunk, N, B, H):
     w = synth.HYBRID_BF16.replace(d=d, n_swa=0, n_dswa=0, n_gla=H, chunk=chunk)
     x = synth.make_inputs(w, N=N, B=B)
@@ -205,7 +208,7 @@ def test_bf16_gla_matches_oracle(kta, d, chunk, N, B, H):
 
 @pytest.mark.parametrize("d,chunk,N,B,H", [(128, 64, 1000, 2, 2), (128, 64, 50, 1, 3),
                                            (128, 64, 9000, 1, 2), (64, 32, 777, 2, 1),
-                                           (128, 16, 300, 1, 2)])
+                                           (128, 16, 300, 1, 2), (128, 64, 1, 1, 2)])
 def test_bf16_gla_end_state_only_matches_full_forward(kta, d, chunk, N, B, H):
     """kta_gla_chunk_state (state pass + segment fold, no outputs) against the full forward's
     S_out and the oracle, with a start state; one segment (N = 50) and many (N = 9000)."""
@@ -262,7 +265,10 @@ def test_bf16_gla_small_gates_match_oracle(kta, kind, d, chunk, N):
 
 @pytest.mark.parametrize("d,N,B,H,with_s0", [(128, 300, 2, 2, True), (64, 1000, 1, 3, False),
                                              (128, 4096, 1, 1, True), (128, 50, 3, 1, True),
-                                             (64, 640, 2, 5, True)])
+                                             (64, 640, 2, 5, True),
+                                             # one token; a chunk less one; a chunk and one
+                                             (128, 1, 1, 1, True), (128, 63, 2, 1, True),
+                                             (64, 65, 1, 2, False)])
 def test_bf16_delta_matches_oracle(kta, d, N, B, H, with_s0):
     w = synth.DELTA_BF16.replace(d=d, n_gla=H)
     x = synth.make_inputs(w, N=N, B=B)
