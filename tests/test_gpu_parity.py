@@ -427,11 +427,13 @@ def test_stream_rollout_matches_full_forward(kta, dtype):
     st.close()
 
 
-@pytest.mark.parametrize("P", [16, 40, 104])
+@pytest.mark.parametrize("P", [1, 7, 16, 40, 104])
 def test_stream_short_frames_match_full_forward(kta, P):
     """Frames shorter than a key tile: the streamed SWA window is a ring of W slots, so its packed
-    tiles (and the dilated window's) span several frames. Softmax heads equal the full forward bit
-    for bit; every head is within the bf16 bound of the oracle."""
+    tiles (and the dilated window's) span several frames. DSWA heads equal the full forward bit
+    for bit; so do SWA heads when P is a multiple of 8 (the ring's frames are then packed into the
+    full forward's tiles; otherwise each frame is its own span and the two agree within rounding).
+    Every head is within the bf16 bound of the oracle."""
     w = synth.STREAM_BF16.replace(F=14, P=P, n_swa=2, n_dswa=2, n_gla=2, W_swa=5, W_dswa=4, dil=2)
     x = synth.make_inputs(w, B=2)
     cfg = kta.cfg_from_workload(w, B=2)
@@ -445,7 +447,12 @@ def test_stream_short_frames_match_full_forward(kta, P):
                             a[:, sl].contiguous()))
     kta.device_status()
     roll = torch.cat(outs, dim=1)
-    assert torch.equal(roll[:, :, :4], full[:, :, :4])
+    assert torch.equal(roll[:, :, 2:4], full[:, :, 2:4])
+    if P % 8 == 0:
+        assert torch.equal(roll[:, :, :2], full[:, :, :2])
+    else:
+        assert_heads_close(roll, full.float().cpu().numpy().astype(np.float64), range(2), BF16_TOL,
+                           what=f"short-frame stream P={P} vs full")
     ref, _ = oracle.hybrid(x["q"], x["k"], x["v"], x["alpha"], None, P=w.P, n_swa=2, n_dswa=2,
                            n_gla=2, W_swa=w.W_swa, W_dswa=w.W_dswa, dil=w.dil,
                            scale_softmax=w.scale_softmax)
