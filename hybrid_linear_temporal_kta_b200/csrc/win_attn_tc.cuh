@@ -23,7 +23,8 @@
 //                the softmax wrote it over S, V MN-major). MMAs of one thread run in issue order,
 //                so S_X(i+1) overwrites P_X(i) only after PV_X(i) has read it, and the softmax of
 //                S_X(i+1) finds O_X stable.
-//   warps 2, 3   idle after set-up.
+//   warp 2       with a key split (below), the second producer: the second half's K / V.
+//   warp 3       idle after set-up.
 //   warps 4..7   softmax of tile A; warps 8..11 softmax of tile B: thread <-> query row (TMEM
 //                lane). Lazy rescale of O when the row max grows by more than 2^8; after the
 //                first tile the exponentials P = exp2(S*scale*log2e - m) are taken against the
@@ -31,8 +32,12 @@
 //                the max grew past that bound, so the max is off the critical path. P goes to
 //                TMEM as bf16 (scaling and row sums on packed fp32 pairs); one arrival per warp
 //                hands P to the MMA thread (128 arrivals on one barrier serialise); epilogue
-//                O / l -> bf16 -> global.
-// While the softmax of one tile runs, the tensor core works on the other tile's products.
+//                O / l -> bf16 -> the tile's Q buffer (free once its last product has run) ->
+//                one TMA store of 32 rows per warp (rows past the frame are outside the map).
+// While the softmax of one tile runs, the tensor core works on the other tile's products. A CTA
+// left with a single query tile (a ragged last tile, or every tile of a launch too small for
+// pairs) gives its two accumulators the two halves of that tile's key range instead and merges
+// the two partial results (running maxima, sums and O) before the store.
 // Every wait is bounded; on a timeout the CTA records it and unwinds to free its TMEM.
 #pragma once
 
